@@ -1,0 +1,98 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench.
+
+This module holds no attention arithmetic: it only draws random tensors (and
+builds the deterministic sinusoid input of the ddx issue #217 repro), so that
+the float64 oracle and the CUDA library see exactly the same bits.
+
+Draw order and distribution: one ``torch.Generator('cpu')`` seeded with the
+config's seed draws q, k, v, dO in that order, each ``randn(B, H, N, d)`` in
+float32. q and k are multiplied by ``qk_gain`` (0.5 for the 262,144-token
+case, 1.0 otherwise). For bf16 configs the float32 draws are rounded to
+bfloat16 (round-to-nearest-even, as ``Tensor.to(torch.bfloat16)`` rounds); the
+oracle then widens exactly those rounded values to float64.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class AttnConfig:
+    """One workload: shape [B, H, N, d], element type and seed."""
+
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    dtype: str  # "f32" or "bf16"
+    seed: int
+    qk_gain: float = 1.0
+    causal: bool = True
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def bwd_flops(self) -> float:
+        """Causal backward FLOPs, counted as 2.5x the causal forward's 4*B*H*N^2*d/2."""
+        return 5.0 * self.B * self.H * self.N * self.N * self.d
+
+    @property
+    def fwd_flops(self) -> float:
+        return 2.0 * self.B * self.H * self.N * self.N * self.d
+
+
+# The five workloads: a 256-token single head (fp32), the nanoGPT-shaped
+# batch of ddx issue #217 (12 sequences, 4 heads, 64 positions, 128 channels),
+# 1,024 tokens, 16,384 tokens x 32 heads, and 262,144 tokens (FlashBoB's length).
+CONFIGS = {
+    "c1": AttnConfig("c1", 1, 1, 256, 64, "f32", 0),
+    "c2_f32": AttnConfig("c2_f32", 12, 4, 64, 32, "f32", 1),
+    "c2_bf16": AttnConfig("c2_bf16", 12, 4, 64, 32, "bf16", 1),
+    "c3": AttnConfig("c3", 1, 1, 1024, 64, "bf16", 2),
+    "c4": AttnConfig("c4", 2, 16, 16384, 128, "bf16", 3),
+    "c5": AttnConfig("c5", 1, 4, 262144, 64, "bf16", 4, qk_gain=0.5),
+}
+
+
+def draw(B: int, H: int, N: int, d: int, seed: int, dtype: str = "f32",
+         qk_gain: float = 1.0):
+    """Return q, k, v, dO as CPU tensors of ``dtype`` ('f32' or 'bf16')."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = []
+    for name in ("q", "k", "v", "do"):
+        t = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
+        if name in ("q", "k") and qk_gain != 1.0:
+            t = t * qk_gain
+        out.append(t.to(torch.bfloat16) if dtype == "bf16" else t)
+    return tuple(out)
+
+
+def draw_config(cfg: AttnConfig):
+    return draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    """Widen a CPU tensor (f32 or bf16) to a float64 numpy array, exactly."""
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def ddx_issue217_input(S: int = 3, T: int = 8, H: int = 2, C: int = 4):
+    """The deterministic repro input of ddx issue #217.
+
+    q, k, v hold sin(n * 0.37 + phase) for n = 0 .. S*T*H*C-1 in (seq, pos,
+    head, channel) order, with phase 0, 1, 2. Returned as float64 arrays
+    permuted to this library's [B, H, N, d] layout (B = seq, N = pos).
+    """
+    n = np.arange(S * T * H * C, dtype=np.float64)
+    outs = []
+    for phase in (0.0, 1.0, 2.0):
+        x = np.sin(n * 0.37 + phase).reshape(S, T, H, C)
+        outs.append(np.ascontiguousarray(x.transpose(0, 2, 1, 3)))
+    return tuple(outs)

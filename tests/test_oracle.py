@@ -1,0 +1,313 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+None of these compare the oracle with itself: finite differences, closed
+forms, invariants, the pair count printed by ddx issue #217's repro and an
+independently written torch float64 autograd formula. The last group plants
+plausible mistakes in copies of the oracle's backward and checks that the
+finite-difference pin catches each of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention_f64 as A
+from seeded_inputs import ddx_issue217_input
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(seed, *shape):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def rel(a, b):
+    """Normwise relative error max|a-b| / max|b|."""
+    a, b = np.asarray(a), np.asarray(b)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-300))
+
+
+def loss_fn(q, k, v, do, scale, causal):
+    return float((do * A.forward_head(q, k, v, scale, causal)["O"]).sum())
+
+
+def fd_grads(q, k, v, do, scale, causal, h=1e-6):
+    """Central finite differences of L = sum(dO o O(q, k, v))."""
+    out = []
+    for which in range(3):
+        args = [q.copy(), k.copy(), v.copy()]
+        g = np.zeros_like(args[which])
+        for idx in np.ndindex(g.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            g[idx] = (loss_fn(*plus, do, scale, causal) - loss_fn(*minus, do, scale, causal)) / (2 * h)
+        out.append(g)
+    return out
+
+
+def tiny_case(seed=0, n=8, d=4):
+    return rnd(seed, n, d), rnd(seed + 1, n, d), rnd(seed + 2, n, d), rnd(seed + 3, n, d)
+
+
+# --------------------------------------------------------------------------
+# finite differences (B=1, H=1, N=8, d=4)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [True, False])
+def test_finite_differences(causal):
+    q, k, v, do = tiny_case()
+    scale = 0.5
+    r = A.backward_head(q, k, v, do, scale, causal)
+    fq, fk, fv = fd_grads(q, k, v, do, scale, causal)
+    for an, fd in ((r["dQ"], fq), (r["dK"], fk), (r["dV"], fv)):
+        assert np.all(np.abs(an - fd) <= 1e-7 * np.abs(fd).max() + 1e-9)
+
+
+# --------------------------------------------------------------------------
+# softmax normalisation and the causal filter
+# --------------------------------------------------------------------------
+def test_softmax_rows_sum_to_one_and_mask_is_exact():
+    q, k, v, _ = tiny_case(5, n=33, d=16)
+    f = A.forward_head(q, k, v, 0.25, causal=True)
+    P = f["P"]
+    assert np.abs(P.sum(axis=1) - 1).max() <= 1e-14
+    iu = np.triu_indices(33, 1)
+    assert np.all(P[iu] == 0.0)
+    il = np.tril_indices(33)
+    assert np.all(P[il] > 0.0)
+
+
+def test_lse_is_log_of_normaliser():
+    q, k, v, _ = tiny_case(6, n=20, d=8)
+    f = A.forward_head(q, k, v, 0.3, causal=True)
+    S = 0.3 * q @ k.T
+    for i in range(20):
+        assert abs(f["LSE"][i] - np.log(np.exp(S[i, : i + 1]).sum())) < 1e-13
+
+
+# --------------------------------------------------------------------------
+# invariance to a per-row shift of the scores
+# --------------------------------------------------------------------------
+def test_row_shift_invariance():
+    q, k, v, do = tiny_case(7, n=24, d=8)
+    c = rnd(11, 24) * 10
+    c[0], c[1] = 50.0, -50.0
+    a = A.backward_head(q, k, v, do, 0.4, True)
+    b = A.backward_head(q, k, v, do, 0.4, True, row_shift=c)
+    assert rel(b["fwd"]["O"], a["fwd"]["O"]) <= 1e-12
+    assert np.abs(b["fwd"]["LSE"] - c - a["fwd"]["LSE"]).max() <= 1e-12 * 50
+    for g in ("dQ", "dK", "dV"):
+        assert rel(b[g], a[g]) <= 1e-12
+
+
+# --------------------------------------------------------------------------
+# the shift's gradient cancels (ddx issue #243, item 1)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("ties", ["first", "split"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_with_shift_equals_without(ties, causal):
+    q, k, v, do = tiny_case(8, n=40, d=16)
+    a = A.backward_head(q, k, v, do, 0.25, causal)
+    b = A.backward_head_with_shift(q, k, v, do, 0.25, causal, ties=ties)
+    for g in ("dQ", "dK", "dV"):
+        assert rel(b[g], a[g]) <= 1e-12
+    # the routed max-terms are tiny rounding residue, not signal
+    assert np.abs(b["dm"]).max() <= 1e-13
+
+
+def test_with_shift_ties_split_equals_first():
+    # identical keys make every row's maximum tied
+    q, _, v, do = tiny_case(9, n=12, d=4)
+    k = np.tile(rnd(10, 1, 4), (12, 1))
+    a = A.backward_head_with_shift(q, k, v, do, 0.5, True, ties="first")
+    b = A.backward_head_with_shift(q, k, v, do, 0.5, True, ties="split")
+    for g in ("dQ", "dK", "dV"):
+        assert np.abs(a[g] - b[g]).max() <= 1e-12 * max(1.0, np.abs(a[g]).max())
+
+
+# --------------------------------------------------------------------------
+# closed forms
+# --------------------------------------------------------------------------
+def test_single_position():
+    q, k, v, do = tiny_case(12, n=1, d=8)
+    r = A.backward_head(q, k, v, do, 0.3, True)
+    assert np.array_equal(r["fwd"]["O"], v)
+    assert np.allclose(r["dV"], do, rtol=0, atol=1e-15)
+    assert np.abs(r["dQ"]).max() <= 1e-14 and np.abs(r["dK"]).max() <= 1e-14
+
+
+def test_zero_queries_give_prefix_means():
+    n, d = 17, 5
+    _, k, v, do = tiny_case(13, n=n, d=d)
+    q = np.zeros((n, d))
+    r = A.backward_head(q, k, v, do, 0.7, True)
+    f = r["fwd"]
+    for i in range(n):
+        assert np.allclose(f["P"][i, : i + 1], 1.0 / (i + 1), rtol=1e-14, atol=0)
+        assert np.allclose(f["O"][i], v[: i + 1].mean(axis=0), rtol=1e-13, atol=1e-15)
+        assert abs(f["LSE"][i] - np.log(i + 1)) <= 1e-14
+    want_dv = np.array([sum(do[i] / (i + 1) for i in range(j, n)) for j in range(n)])
+    assert np.allclose(r["dV"], want_dv, rtol=1e-13, atol=1e-15)
+
+
+def test_equal_value_rows_give_zero_score_gradients():
+    n, d = 21, 6
+    q, k, _, do = tiny_case(14, n=n, d=d)
+    v = np.tile(rnd(15, 1, d), (n, 1))
+    r = A.backward_head(q, k, v, do, 0.5, True)
+    assert np.allclose(r["fwd"]["O"], v, rtol=1e-14, atol=1e-14)
+    assert np.abs(r["dQ"]).max() <= 1e-13
+    assert np.abs(r["dK"]).max() <= 1e-13
+
+
+# --------------------------------------------------------------------------
+# row and column identities
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [True, False])
+def test_identities(causal):
+    q, k, v, do = tiny_case(16, n=50, d=12)
+    r = A.backward_head(q, k, v, do, 0.3, causal)
+    scale_g = np.abs(r["dK"]).max()
+    assert np.abs(r["dK"].sum(axis=0)).max() <= 1e-12 * 50 * scale_g
+    assert np.allclose(r["dV"].sum(axis=0), do.sum(axis=0), rtol=1e-12, atol=1e-12)
+    assert np.allclose(r["D"], r["D_rows"], rtol=1e-12, atol=1e-13)
+    assert np.abs(r["dS"].sum(axis=1)).max() <= 1e-13
+
+
+# --------------------------------------------------------------------------
+# independent float64 cross-check: torch autograd of a separately written formula
+# --------------------------------------------------------------------------
+def torch_reference(q, k, v, do, scale, causal):
+    q, k, v = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    s = (q @ k.transpose(-1, -2)) * scale
+    if causal:
+        n = q.shape[-2]
+        s = s.masked_fill(~torch.ones(n, n, dtype=torch.bool).tril(), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    (o * torch.tensor(do)).sum().backward()
+    return o.detach().numpy(), q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_torch_autograd_cross_check(causal):
+    B, H, N, d = 2, 3, 37, 16
+    q, k, v, do = (rnd(20 + t, B, H, N, d) for t in range(4))
+    out = A.backward(q, k, v, do, 0.25, causal)
+    o, gq, gk, gv = torch_reference(q, k, v, do, 0.25, causal)
+    assert rel(out["O"], o) <= 1e-12
+    assert rel(out["dQ"], gq) <= 1e-12
+    assert rel(out["dK"], gk) <= 1e-12
+    assert rel(out["dV"], gv) <= 1e-12
+
+
+# --------------------------------------------------------------------------
+# ddx issue #217's repro: its printed table sizes and its float64 JAX check
+# --------------------------------------------------------------------------
+def test_ddx_issue217_repro():
+    with open(os.path.join(GOLDEN, "ddx_issue217_repro.json")) as fh:
+        g = json.load(fh)
+    inp, printed = g["input"], g["printed"]
+    S, T, H, C = inp["S_sequences"], inp["T_positions"], inp["H_heads"], inp["C_channels"]
+    q, k, v = ddx_issue217_input(S, T, H, C)
+    assert q.shape == (S, H, T, C)
+    # the scores table keeps S*H*T(T+1)/2 rows
+    assert oracle.causal_pair_count(S, H, T) == printed["causal_score_rows"]
+    assert (S * H * T) ** 2 == printed["cross_product_rows"]
+    assert S * H * T * T == printed["seq_head_pos_pos"]
+    scale = 1.0 / inp["score_divisor"]
+    O, _ = A.forward(q, k, v, scale, True)
+    assert O.size == printed["saved_2_rows_attention_output"]
+    # loss sum(O^2)/2 => dO = O; check the gradient at the repro's tolerances
+    out = A.backward(q, k, v, O, scale, True)
+    _, gq, gk, gv = torch_reference(q, k, v, O, scale, True)
+    tol = printed["jax_check"]
+    for ours, ref in ((out["dQ"], gq), (out["dK"], gk), (out["dV"], gv)):
+        assert np.allclose(ours, ref, rtol=tol["rtol"], atol=tol["atol"])
+
+
+# --------------------------------------------------------------------------
+# row-wise, row-block and key-tail forms against the materialised head
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [True, False])
+def test_query_rows_and_row_blocks(causal):
+    n, d = 70, 8
+    q, k, v, do = tiny_case(30, n=n, d=d)
+    full = A.backward_head(q, k, v, do, 0.35, causal)
+    rows = [0, 1, 17, 63, 69]
+    qr = A.query_rows(q, k, v, do, 0.35, rows, causal)
+    assert rel(qr["dQ"], full["dQ"][rows]) <= 1e-12
+    assert rel(qr["O"], full["fwd"]["O"][rows]) <= 1e-12
+    assert np.allclose(qr["LSE"], full["fwd"]["LSE"][rows], rtol=1e-13)
+    assert np.allclose(qr["D"], full["D"][rows], rtol=1e-12, atol=1e-13)
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    for r0 in range(0, n, 16):
+        blk = A.backward_row_block(q, k, v, do, 0.35, r0, min(n, r0 + 16), causal)
+        dK += blk["dK"]
+        dV += blk["dV"]
+        assert rel(blk["dQ"], full["dQ"][r0:r0 + 16]) <= 1e-12
+    assert rel(dK, full["dK"]) <= 1e-12
+    assert rel(dV, full["dV"]) <= 1e-12
+    if causal:
+        tail = A.key_tail(q, k, v, do, 0.35, 50)
+        assert rel(tail["dK"], full["dK"][50:]) <= 1e-12
+        assert rel(tail["dV"], full["dV"][50:]) <= 1e-12
+
+
+def test_batched_equals_per_head_and_head_permutation():
+    B, H, N, d = 2, 3, 19, 4
+    q, k, v, do = (rnd(40 + t, B, H, N, d) for t in range(4))
+    out = A.backward(q, k, v, do, 0.5, True)
+    perm = [2, 0, 1]
+    outp = A.backward(q[:, perm], k[:, perm], v[:, perm], do[:, perm], 0.5, True)
+    for g in ("dQ", "dK", "dV", "O", "LSE"):
+        assert np.array_equal(outp[g], out[g][:, perm])
+
+
+# --------------------------------------------------------------------------
+# test of the tests: plausible mistakes planted in copies of the backward
+# --------------------------------------------------------------------------
+def _mutant(kind):
+    def bwd(q, k, v, do, scale, causal):
+        f = A.forward_head(q, k, v, scale, causal)
+        P, O = f["P"], f["O"]
+        dV = P.T @ do
+        dP = do @ v.T
+        D = (do * O).sum(axis=1)
+        if kind == "drop_D":
+            dS = P * dP
+        elif kind == "sign":
+            dS = P * (dP + D[:, None])
+        else:
+            dS = P * (dP - D[:, None])
+        dQ = scale * dS @ k
+        dK = scale * dS.T @ q
+        if kind == "transpose_dV":
+            dV = P @ do
+        if kind == "no_scale_dK":
+            dK = dS.T @ q
+        if kind == "swap_dQ_operand":
+            dQ = scale * dS.T @ k
+        return {"dQ": dQ, "dK": dK, "dV": dV}
+    return bwd
+
+
+@pytest.mark.parametrize("kind", ["drop_D", "sign", "transpose_dV", "no_scale_dK", "swap_dQ_operand"])
+def test_finite_differences_catch_planted_mistakes(kind):
+    q, k, v, do = tiny_case()
+    r = _mutant(kind)(q, k, v, do, 0.5, True)
+    fq, fk, fv = fd_grads(q, k, v, do, 0.5, True)
+    worst = max(rel(r["dQ"], fq), rel(r["dK"], fk), rel(r["dV"], fv))
+    assert worst > 1e-3
+
+
+def test_pair_count_catches_a_mask_without_diagonal(monkeypatch):
+    def strict(n_q, n_k, causal, q_offset=0):
+        i = q_offset + np.arange(n_q)[:, None]
+        return (i > np.arange(n_k)[None, :]) if causal else np.ones((n_q, n_k), bool)
+    monkeypatch.setattr(A, "keep_mask", strict)
+    assert A.causal_pair_count(3, 2, 8) != 216
