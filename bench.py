@@ -1,0 +1,402 @@
+"""Benchmark of the causal attention backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c4] [--impl reference]
+
+A step is one whole backward pass (attn_bwd: preprocess, main tile loop, dQ
+conversion) over one batch of seeded synthetic inputs already resident in
+HBM. The default workload is 2 sequences x 16 heads x 16,384 tokens x 128
+channels in bf16 (the long-sequence configuration on which the TFLOP/s target
+is stated). FLOPs are counted as 2.5x the causal forward's 4*B*H*N^2*d/2.
+
+Under torchrun each rank runs the same per-GPU workload on its own inputs
+(heads are independent; no collective on the data path): weak scaling, value =
+all ranks' FLOPs / max-over-ranks device time.
+
+`--impl reference` times the float64 CPU oracle instead (rank 0 only), on a
+bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from seeded_inputs import CONFIGS, draw  # noqa: E402
+
+METRIC = "causal attention backward TFLOP/s (bf16, 1×B200) and % of dense tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+MAIN_KERNEL_SOURCE = os.path.join(ROOT, "causal_softmax_attention_b200", "csrc",
+                                  "bwd_bf16_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bwd_main_dram_traffic.json")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in ("bwd_bf16_sm100.cu", "sm100.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "causal_softmax_attention_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic_per_launch(cfg):
+    """DRAM bytes per main-kernel launch from the committed ncu summary, scaled
+    to this workload by the causal tile pairs processed; None if the summary
+    is missing or was taken on a different kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as fh:
+        t = json.load(fh)
+    if t.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    if t.get("d") != cfg.d:
+        return None
+    T = math.ceil(cfg.N / 128)
+    pairs = cfg.B * cfg.H * T * (T + 1) / 2
+    return t["dram_bytes_per_tile_pair"] * pairs
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as fh:
+            rows = [r.strip().split(", ") for r in fh if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------- oracle arms
+def oracle_sample(cfg, budget_s: float, rows_per_block: int = 256):
+    """Time the float64 oracle on the last query-row blocks of head (0, 0)
+    until `budget_s` seconds of CPU work; returns (TFLOP/s, description)."""
+    import oracle
+    from seeded_inputs import as_f64
+    q, k, v, do = draw(1, 1, cfg.N, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)
+    qh, kh, vh, doh = (as_f64(t[0, 0]) for t in (q, k, v, do))
+    flops, elapsed, rows, r1 = 0.0, 0.0, 0, cfg.N
+    while elapsed < budget_s:
+        if r1 <= 0:  # whole head done: repeat from the end until the budget is spent
+            r1 = cfg.N
+        r0 = max(0, r1 - rows_per_block)
+        t0 = time.perf_counter()
+        oracle.backward_row_block(qh, kh, vh, doh, cfg.scale, r0, r1, causal=True)
+        elapsed += time.perf_counter() - t0
+        pairs = (r1 * (r1 + 1) - r0 * (r0 + 1)) / 2  # causal pairs of rows r0..r1-1
+        flops += 10.0 * cfg.d * pairs
+        rows += r1 - r0
+        r1 = r0
+    desc = (f"oracle backward_row_block (numpy float64) on {rows} query rows (last rows first) of one "
+            f"head of {cfg.name} (N={cfg.N}, d={cfg.d}): {flops / 10 / cfg.d:.3e} causal pairs "
+            f"in {elapsed:.1f} s")
+    return flops / elapsed / 1e12, desc, elapsed
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, budget / 4)
+    vals, descs, times = [], [], []
+    for _ in range(args.steps):
+        v, d, t = oracle_sample(cfg, budget)
+        vals.append(v)
+        descs.append(d)
+        times.append(t)
+    value = statistics.median(vals)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": descs[-1]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, n_gpus):
+    return {"workload": f"{cfg.name}: causal attention backward B={cfg.B} H={cfg.H} "
+                        f"N={cfg.N} d={cfg.d} {cfg.dtype}, q,k,v,dO ~ N(0,1)"
+                        + (f" (q,k x{cfg.qk_gain})" if cfg.qk_gain != 1.0 else "")
+                        + f", seed {cfg.seed}, scale 1/sqrt(d)",
+            "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "causal": True,
+            "global_batch": cfg.B * n_gpus, "seq_len": cfg.N,
+            "parallelism": f"independent replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush needed)"
+            if 5 * cfg.B * cfg.H * cfg.N * cfg.d * 2 > 126e6 else "L2 flushed between steps"}
+
+
+# --------------------------------------------------------------------- GPU arm
+def run_gpu(args, cfg, world, rank, local):
+    import causal_softmax_attention_b200 as csa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
+    q, k, v, do = draw(B, H, N, d, cfg.seed + 1000 * rank, cfg.dtype, cfg.qk_gain)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = csa.forward(qd, kd, vd, True, cfg.scale)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = csa.new_workspace(qd)
+    stream = torch.cuda.current_stream(dev)
+    small = 5 * B * H * N * d * 2 <= 126e6
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small else None
+
+    def step(ev_main=None):
+        if flush is not None:
+            flush.zero_()
+        csa.attn_bwd_preprocess(o, dod, lse, ws, stream)
+        if ev_main is not None:
+            ev_main[0].record(stream)
+        csa.attn_bwd_main(qd, kd, vd, dod, dq, dk, dv, ws, True, cfg.scale, stream)
+        if ev_main is not None:
+            ev_main[1].record(stream)
+        csa.attn_bwd_dq_convert(dq, ws, cfg.scale, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if csa.attn_last_status(ws) != 0:
+        raise RuntimeError("device status after warm-up: " + csa.status_string(csa.attn_last_status(ws)))
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mains = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_begin = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_begin.record(stream)
+        for s in range(args.steps):
+            starts[s].record(stream)
+            step(mains[s])
+            ends[s].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t_begin.elapsed_time(t_end)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    main_ms = [a.elapsed_time(b) for a, b in mains]
+    if flush is not None:
+        # remove the flush from the step time: time it alone
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        flush.zero_()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        total_ms -= args.steps * f0.elapsed_time(f1)
+    status = csa.attn_last_status(ws)
+    ms_per_step = max_over_ranks(total_ms / args.steps, world)
+    flops = cfg.bwd_flops
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- e2e through the public API with pinned host buffers
+    hq, hk, hv, ho, hdo = (t.cpu().pin_memory() for t in (qd, kd, vd, o, dod))
+    hlse = lse.cpu().pin_memory()
+    hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ho, hdo, hlse))
+    d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+
+    def e2e_step():
+        for h, dvc in ((hq, qd), (hk, kd), (hv, vd), (ho, o), (hdo, dod), (hlse, lse)):
+            dvc.copy_(h, non_blocking=True)
+        csa.attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, True, cfg.scale, stream)
+        for h, dvc in ((hdq, dq), (hdk, dk), (hdv, dv)):
+            h.copy_(dvc, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    main_avg = statistics.mean(main_ms)
+    achieved = flops / (main_avg * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = dram_traffic_per_launch(cfg)
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_dict(cfg, world),
+        "pct_of_dense_bf16_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "attn_bwd_bf16_sm100_kernel",
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": main_avg},
+        "stage_ms": {"step_median": statistics.median(step_ms), "main_median": statistics.median(main_ms),
+                     "pre_and_convert_median": statistics.median(step_ms) - statistics.median(main_ms)},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "device_status": csa.status_string(status),
+        "peak_memory_bytes": torch.cuda.max_memory_allocated(dev),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, desc, _ = oracle_sample(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c4", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, cfg, world, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,274 @@
+// C ABI of the library (declared in include/attn.h): argument checks, the
+// workspace layout, TMA tensor-map encoding and kernel dispatch. Everything
+// is enqueued on the caller's stream; nothing here allocates device memory.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "common.cuh"
+
+namespace csa {
+
+WorkspaceLayout workspace_layout(int B, int H, int N, int d, int dtype) {
+  WorkspaceLayout L{};
+  const size_t BH = static_cast<size_t>(B) * H;
+  L.Np = round_up(N, kTile);
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  L.status_off = 0;
+  L.lse_off = 256;
+  L.d_off = L.lse_off + up(BH * L.Np * sizeof(float));
+  L.dq_off = L.d_off + up(BH * L.Np * sizeof(float));
+  L.total = L.dq_off + (dtype == ATTN_BF16 ? up(BH * L.Np * d * sizeof(float)) : 0);
+  return L;
+}
+
+Workspace carve_workspace(void* base, const WorkspaceLayout& L) {
+  char* b = static_cast<char*>(base);
+  Workspace w;
+  w.status = reinterpret_cast<int*>(b + L.status_off);
+  w.lse_pad = reinterpret_cast<float*>(b + L.lse_off);
+  w.d_pad = reinterpret_cast<float*>(b + L.d_off);
+  w.dq_acc = reinterpret_cast<float*>(b + L.dq_off);
+  w.Np = L.Np;
+  return w;
+}
+
+}  // namespace csa
+
+namespace {
+
+using namespace csa;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape / pointer checks shared by every entry point.
+int check_shape(int B, int H, int N, int d, int dtype) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (dtype == ATTN_BF16 && d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype == ATTN_F32 && d > 128) return ATTN_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long T = (static_cast<long long>(N) + kTile - 1) / kTile;
+  if (BH > (1LL << 30) || BH * T > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+bool all_aligned(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p == nullptr || !aligned16(p)) return false;
+  return true;
+}
+
+// The tensor-core kernels are built for sm_100a only.
+int check_device_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return (major == 10 && minor == 0) ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [BH][N][d] bf16 array: box = 128 rows x min(d, 64) channels,
+// swizzled to match the UMMA canonical layout. Rows past N read as zero.
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int ch = d >= 64 ? 64 : d;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(ch), static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle swz =
+      ch * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+
+struct FaultInjection {
+  int armed = 0;
+  unsigned long long limit_ns = 0;
+};
+FaultInjection g_fault;
+std::mutex g_fault_mu;
+
+int check_ws(int B, int H, int N, int d, int dtype, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned16(ws)) return ATTN_ERR_INVALID;
+  if (ws_bytes < workspace_layout(B, H, N, d, dtype).total) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported dtype / head dimension";
+    case ATTN_ERR_CUDA: return "CUDA error (launch failed or device is not sm_100)";
+    case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
+  if (check_shape(B, H, N, d, dtype) != ATTN_OK) return 0;
+  return workspace_layout(B, H, N, d, dtype).total;
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, int causal, float scale, int dtype, void* stream) {
+  if (!all_aligned({q, k, v, o, lse})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (dtype == ATTN_F32)
+    return from_cuda(launch_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                    static_cast<const float*>(v), static_cast<float*>(o), lse, BH,
+                                    N, d, causal != 0, scale, s));
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  TmaMaps m;
+  if (!make_map(&m.a, q, BH, N, d) || !make_map(&m.b, k, BH, N, d) ||
+      !make_map(&m.c, v, BH, N, d))
+    return ATTN_ERR_CUDA;
+  int* status = fwd_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  return from_cuda(launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, s));
+}
+
+int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
+                        int d, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!all_aligned({o, dout, lse})) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  return from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, dtype == ATTN_BF16, ws,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                  void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                  int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!all_aligned({q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (dtype == ATTN_F32)
+    return from_cuda(launch_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                    static_cast<const float*>(v),
+                                    static_cast<const float*>(dout), static_cast<float*>(dq),
+                                    static_cast<float*>(dk), static_cast<float*>(dv), BH, N, d,
+                                    causal != 0, scale, ws, s));
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  TmaMaps m;
+  if (!make_map(&m.a, q, BH, N, d) || !make_map(&m.b, k, BH, N, d) ||
+      !make_map(&m.c, v, BH, N, d) || !make_map(&m.d, dout, BH, N, d))
+    return ATTN_ERR_CUDA;
+  int inject = 0;
+  unsigned long long limit = kWaitLimitNs;
+  {
+    std::lock_guard<std::mutex> g(g_fault_mu);
+    if (g_fault.armed) {
+      inject = 1;
+      limit = g_fault.limit_ns;
+      g_fault.armed = 0;
+    }
+  }
+  return from_cuda(launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject, s));
+}
+
+int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!all_aligned({dq})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if (dtype == ATTN_F32) return ATTN_OK;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  return from_cuda(launch_dq_convert(dq, B * H, N, d, scale, ws, static_cast<cudaStream_t>(stream)));
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+             int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+             void* stream) {
+  // Validate everything before the first launch so a bad call enqueues nothing.
+  if (!all_aligned({q, k, v, o, dout, lse, dq, dk, dv})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
+  st = attn_bwd_preprocess(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, stream);
+  if (st != ATTN_OK) return st;
+  st = attn_bwd_main(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
+                     workspace_bytes, stream);
+  if (st != ATTN_OK) return st;
+  return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
+}
+
+int attn_last_status(const void* workspace) {
+  if (workspace == nullptr) return ATTN_ERR_INVALID;
+  int v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return v;
+}
+
+int attn_fwd_last_status(void) {
+  int* p = fwd_status_ptr();
+  if (!p) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return v;
+}
+
+int attn_test_arm_timeout(unsigned long long wait_limit_ns) {
+  if (wait_limit_ns == 0) return ATTN_ERR_INVALID;
+  std::lock_guard<std::mutex> g(g_fault_mu);
+  g_fault.armed = 1;
+  g_fault.limit_ns = wait_limit_ns;
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,427 @@
+// Backward of causal softmax attention on the sm_100a tensor cores (tcgen05).
+//
+// One CTA per (key tile j of 128 keys, head bh). The CTA keeps K_j and V_j in
+// shared memory and walks the query tiles i that can see key tile j (i >= j
+// under the causal filter). For each query tile it recomputes the scores
+// instead of reading a stored N x N table (ddx issue #243, item 2):
+//
+//   S^T  = K_j Q_i^T                 (tcgen05 MMA -> TMEM, lanes = keys)
+//   P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)      (CUDA cores, MUFU)
+//   dP^T = V_j dO_i^T                (tcgen05 MMA -> TMEM)
+//   dS^T = P^T o (dP^T - D_i)        (CUDA cores; the max-shift's gradient is
+//                                     dropped, ddx issue #243, item 1)
+//   dV_j += P^T dO_i,  dK_j += dS^T Q_i   (tcgen05, accumulators stay in TMEM)
+//   dQ_i += dS K_j                   (tcgen05 -> TMEM -> fp32 red.add to HBM)
+//
+// These are the transposes of ddx PR #162 ("transpose p = w / z per score,
+// then p @ v"). Masked (j > i) scores are zeroed in registers on the diagonal
+// tile; tiles above the diagonal are never visited.
+//
+// Warp roles: warps 0-3 (128 threads, one TMEM lane = one key row or one
+// query row each) do the element-wise work and the epilogues; warp 4 issues
+// the TMA loads and the MMAs from one elected lane. All hand-offs are
+// mbarriers; every wait is bounded and reports a timeout in the status word.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+namespace {
+
+using namespace sm100;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int CH = D >= 64 ? 64 : D;   // TMA box width (elements)
+  static constexpr int NCH = D / CH;            // boxes per 128-row tile
+  static constexpr int ROWB = CH * 2;           // bytes per row inside a box
+  static constexpr int CHUNK = kTile * ROWB;    // bytes of one [128][CH] box
+  static constexpr int TILE = NCH * CHUNK;      // bytes of one [128][D] bf16 tile
+  static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr int STAGES = D == 128 ? 1 : 2;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + TILE;
+  static constexpr int Q_OFF = V_OFF + TILE;
+  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;
+  static constexpr int P_OFF = DO_OFF + STAGES * TILE;   // [128 keys][128 queries] bf16
+  static constexpr int DS_OFF = P_OFF + 32768;
+  static constexpr int LSE_OFF = DS_OFF + 32768;         // [STAGES][128] f32
+  static constexpr int DV_OFF = LSE_OFF + STAGES * 512;  // [STAGES][128] f32
+  static constexpr int BAR_OFF = DV_OFF + STAGES * 512;
+  static constexpr int MISC_OFF = BAR_OFF + 16 * 8;
+  static constexpr int BYTES = MISC_OFF + 64;
+  // + alignment slack; at least ~116 KB so that one CTA owns an SM's TMEM.
+  static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr uint32_t T_DQ = D == 128 ? 0 : 256 + 2 * D;
+  static constexpr uint32_t T_COLS = 512;
+};
+
+enum Bar { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_PFULL, B_DQFULL, B_DQEMPTY,
+           B_DONE, B_FINAL, B_COUNT };
+
+struct BwdParams {
+  const float* lse2;  // [BH][Np], LSE * log2(e), +inf past N
+  const float* dvec;  // [BH][Np], D, 0 past N
+  float* dq_acc;      // [BH][T][D/4][128][4]
+  __nv_bfloat16* dk;  // [BH][N][D]
+  __nv_bfloat16* dv;
+  int* status;
+  int N, Np, T, BH;
+  int causal;
+  float scale, scale_log2;
+  uint64_t wait_ns;
+  int inject_fault;   // 1: never signal the first score tile (tests the timeout path)
+};
+
+// Shared-memory address of K-major operand rows [128][D] stored as D/CH boxes,
+// advanced to the kk-th 16-element K step.
+template <int D>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
+  using L = BwdLayout<D>;
+  const int e = kk * 16;
+  const uint32_t addr = tile + (e / L::CH) * L::CHUNK + (e % L::CH) * 2;
+  return smem_desc(addr, 16, 8 * L::ROWB, L::SWZ);
+}
+
+// The same [128 rows][D] tile read as an MN-major B operand (rows = K,
+// columns = N), advanced to the kk-th 16-row K step.
+template <int D>
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
+  using L = BwdLayout<D>;
+  return smem_desc(tile + kk * 16 * L::ROWB, L::CHUNK, 8 * L::ROWB, L::SWZ);
+}
+
+// [128][128] bf16 tiles written by the compute warps (two 64-column boxes).
+__device__ __forceinline__ uint64_t desc_sq_kmajor(uint32_t tile, int kk) {
+  const int e = kk * 16;
+  return smem_desc(tile + (e / 64) * 16384 + (e % 64) * 2, 16, 1024, kSwizzle128B);
+}
+__device__ __forceinline__ uint64_t desc_sq_mnmajor(uint32_t tile, int kk) {
+  return smem_desc(tile + kk * 16 * 128, 16384, 1024, kSwizzle128B);
+}
+
+// Byte offset of the 16-byte group `g` (8 bf16 columns, 0..15) of row `r` in a
+// [128][128] SW128 tile.
+__device__ __forceinline__ uint32_t sq_offset(int r, int g) {
+  return (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__(160, 1)
+    attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  const volatile int* never = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);  // stays 0
+  const float* s_lse = reinterpret_cast<const float*>(smem + L::LSE_OFF);
+  const float* s_dv = reinterpret_cast<const float*>(smem + L::DV_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int jt = blockIdx.x / p.BH;  // longest-first: key tile 0 has the most query tiles
+  const int bh = blockIdx.x % p.BH;
+  const int j0 = jt * kTile;
+  const int i_begin = p.causal ? jt : 0;
+  const int n_iter = p.T - i_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[B_KV], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[B_QFULL + s], 1);
+      mbar_init(&bars[B_QEMPTY + s], 1);
+    }
+    mbar_init(&bars[B_SFULL], 1);
+    mbar_init(&bars[B_PFULL], 128);
+    mbar_init(&bars[B_DQFULL], 1);
+    mbar_init(&bars[B_DQEMPTY], 128);
+    mbar_init(&bars[B_DONE], 1);
+    mbar_init(&bars[B_FINAL], 1);
+    *abort_flag = 0;
+    *const_cast<volatile int*>(never) = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_base_slot, L::T_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicExch(p.status, kStatusTimeout);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------ TMA + MMA issuer
+    if (elect_one_sync()) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      prefetch_tensormap(&tm_do);
+      const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
+      const uint32_t sP = sbase + L::P_OFF, sdS = sbase + L::DS_OFF;
+      mbar_arrive_expect_tx(&bars[B_KV], 2 * L::TILE);
+      for (int c = 0; c < L::NCH; ++c) {
+        tma_load_3d(smem + L::K_OFF + c * L::CHUNK, &tm_k, &bars[B_KV], c * L::CH, j0, bh);
+        tma_load_3d(smem + L::V_OFF + c * L::CHUNK, &tm_v, &bars[B_KV], c * L::CH, j0, bh);
+      }
+      auto load_q = [&](int it) {
+        const int s = it % L::STAGES;
+        const int i0 = (i_begin + it) * kTile;
+        uint64_t* bar = &bars[B_QFULL + s];
+        mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
+        for (int c = 0; c < L::NCH; ++c) {
+          tma_load_3d(smem + L::Q_OFF + s * L::TILE + c * L::CHUNK, &tm_q, bar, c * L::CH, i0,
+                      bh);
+          tma_load_3d(smem + L::DO_OFF + s * L::TILE + c * L::CHUNK, &tm_do, bar, c * L::CH,
+                      i0, bh);
+        }
+        bulk_load(smem + L::LSE_OFF + s * 512, p.lse2 + static_cast<size_t>(bh) * p.Np + i0, 512,
+                  bar);
+        bulk_load(smem + L::DV_OFF + s * 512, p.dvec + static_cast<size_t>(bh) * p.Np + i0, 512,
+                  bar);
+      };
+      const int pre = n_iter < L::STAGES ? n_iter : L::STAGES;
+      int q_loaded = 0, q_waited = 0;
+      for (int it = 0; it < pre; ++it, ++q_loaded) load_q(it);
+
+      constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t ID_KV = idesc_bf16(128, D, false, true);
+      constexpr uint32_t ID_Q = idesc_bf16(128, D, true, true);
+      bool ok = mbar_wait(&bars[B_KV], 0, p.wait_ns, abort_flag);
+      const bool kv_waited = ok;
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int s = it % L::STAGES;
+        const uint32_t ph = (it / L::STAGES) & 1;
+        const uint32_t sQ = sbase + L::Q_OFF + s * L::TILE;
+        const uint32_t sdO = sbase + L::DO_OFF + s * L::TILE;
+        if (!(ok = mbar_wait(&bars[B_QFULL + s], ph, p.wait_ns, abort_flag))) break;
+        ++q_waited;
+        if (it > 0 && !(ok = mbar_wait(&bars[B_DQEMPTY], (it - 1) & 1, p.wait_ns, abort_flag)))
+          break;
+        tc_fence_after();
+        // S^T = K_j Q_i^T and dP^T = V_j dO_i^T (K = D)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + L::T_S, desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
+        if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
+        if (!(ok = mbar_wait(&bars[B_PFULL], it & 1, p.wait_ns, abort_flag))) break;
+        tc_fence_after();
+        // dV_j += P^T dO_i ; dK_j += dS^T Q_i   (K = 128 queries)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::T_DV, desc_sq_kmajor(sP, kk), desc_mnmajor<D>(sdO, kk), ID_KV,
+                 (it > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::T_DK, desc_sq_kmajor(sdS, kk), desc_mnmajor<D>(sQ, kk), ID_KV,
+                 (it > 0 || kk > 0));
+        // dQ_i = dS K_j   (K = 128 keys)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::T_DQ, desc_sq_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
+        mma_commit(&bars[B_DQFULL]);
+        mma_commit(&bars[B_QEMPTY + s]);
+        if (it + L::STAGES < n_iter) {
+          if (!(ok = mbar_wait(&bars[B_QEMPTY + s], ph, p.wait_ns, abort_flag))) break;
+          load_q(it + L::STAGES);
+          ++q_loaded;
+        }
+      }
+      if (ok) {
+        mma_commit(&bars[B_DONE]);
+      } else {
+        fail();
+        // Drain the loads still in flight (bounded) before the CTA exits.
+        if (!kv_waited) mbar_wait(&bars[B_KV], 0, p.wait_ns, never);
+        for (int w = q_waited; w < q_loaded; ++w)
+          mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_ns, never);
+      }
+      // Every MMA this thread issued has finished before TMEM is freed.
+      mma_commit(&bars[B_FINAL]);
+      mbar_wait(&bars[B_FINAL], 0, p.wait_ns, never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ element-wise warps 0-3
+    const int t = threadIdx.x;  // key row within the tile (S^T lanes), query row for dQ
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int key = j0 + t;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % L::STAGES;
+      const int i = i_begin + it;
+      const int i0 = i * kTile;
+      if (!(ok = mbar_wait(&bars[B_QFULL + s], (it / L::STAGES) & 1, p.wait_ns, abort_flag)))
+        break;
+      if (!(ok = mbar_wait(&bars[B_SFULL], it & 1, p.wait_ns, abort_flag))) break;
+      tc_fence_after();
+      const float* lse_s = s_lse + s * 128;
+      const float* d_s = s_dv + s * 128;
+      // queries with local index < thr are masked for this key row
+      const int thr = key >= p.N ? 128 : ((p.causal && i == jt) ? t : 0);
+      uint8_t* sP = smem + L::P_OFF;
+      uint8_t* sdS = smem + L::DS_OFF;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(lane_base + L::T_S + 32 * c, sr);
+        tmem_ld32(lane_base + L::T_DP + 32 * c, dr);
+        tmem_ld_wait();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const int q0 = 32 * c + u;
+          float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -lse_s[q0]));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -lse_s[q0 + 1]));
+          if (q0 < thr) p0 = 0.f;
+          if (q0 + 1 < thr) p1 = 0.f;
+          const float ds0 = p0 * (__uint_as_float(dr[u]) - d_s[q0]);
+          const float ds1 = p1 * (__uint_as_float(dr[u + 1]) - d_s[q0 + 1]);
+          pk[u / 2] = pack_bf16x2(p0, p1);
+          dk[u / 2] = pack_bf16x2(ds0, ds1);
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t off = sq_offset(t, 4 * c + v);
+          st_shared_v4(smem_u32(sP) + off, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          st_shared_v4(smem_u32(sdS) + off, dk[4 * v], dk[4 * v + 1], dk[4 * v + 2],
+                       dk[4 * v + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[B_PFULL]);
+      if (!(ok = mbar_wait(&bars[B_DQFULL], it & 1, p.wait_ns, abort_flag))) break;
+      tc_fence_after();
+      // dQ partial sums of query row i0 + t -> fp32 accumulator (tile-major layout)
+      const bool row_ok = i0 + t < p.N;
+      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + L::T_DQ + 32 * c, r);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(acc + (8 * c + v) * 512, __uint_as_float(r[4 * v]),
+                       __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                       __uint_as_float(r[4 * v + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_DQEMPTY]);
+    }
+    if (ok) ok = mbar_wait(&bars[B_DONE], 0, p.wait_ns, abort_flag);
+    if (!ok) {
+      fail();
+    } else {
+      tc_fence_after();
+      // Epilogue: dV_j and scale * dK_j rows -> bf16
+      if (key < p.N) {
+        __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + key) * D;
+        __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + key) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rv[32], rk[32];
+          tmem_ld32(lane_base + L::T_DV + 32 * c, rv);
+          tmem_ld32(lane_base + L::T_DK + 32 * c, rk);
+          tmem_ld_wait();
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 ov, ok4;
+            ov.x = pack_bf16x2(__uint_as_float(rv[8 * v + 0]), __uint_as_float(rv[8 * v + 1]));
+            ov.y = pack_bf16x2(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3]));
+            ov.z = pack_bf16x2(__uint_as_float(rv[8 * v + 4]), __uint_as_float(rv[8 * v + 5]));
+            ov.w = pack_bf16x2(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7]));
+            ok4.x = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 0]),
+                                p.scale * __uint_as_float(rk[8 * v + 1]));
+            ok4.y = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 2]),
+                                p.scale * __uint_as_float(rk[8 * v + 3]));
+            ok4.z = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 4]),
+                                p.scale * __uint_as_float(rk[8 * v + 5]));
+            ok4.w = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 6]),
+                                p.scale * __uint_as_float(rk[8 * v + 7]));
+            *reinterpret_cast<uint4*>(dv_row + 32 * c + 8 * v) = ov;
+            *reinterpret_cast<uint4*>(dk_row + 32 * c + 8 * v) = ok4;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::T_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, void* dv, int BH,
+                              int N, bool causal, float scale, uint64_t wait_ns, int inject,
+                              cudaStream_t s) {
+  using L = BwdLayout<D>;
+  auto kern = attn_bwd_bf16_sm100_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  BwdParams p;
+  p.lse2 = ws.lse_pad;
+  p.dvec = ws.d_pad;
+  p.dq_acc = ws.dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = ws.status;
+  p.N = N;
+  p.Np = ws.Np;
+  p.T = ws.Np / kTile;
+  p.BH = BH;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = wait_ns;
+  p.inject_fault = inject;
+  const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
+  kern<<<grid, 160, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
+                            int N, int d, bool causal, float scale, uint64_t wait_limit_ns,
+                            int inject_fault, cudaStream_t s) {
+  switch (d) {
+    case 32:
+      return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+                                   inject_fault, s);
+    case 64:
+      return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+                                   inject_fault, s);
+    case 128:
+      return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+                                    inject_fault, s);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace csa

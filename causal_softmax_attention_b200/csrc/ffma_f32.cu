@@ -1,0 +1,286 @@
+// fp32 forward and backward on the CUDA cores (FFMA), for small fp32 workloads.
+//
+// Same mathematics as the tensor-core path, entirely in fp32 with expf/logf:
+//   forward  S = scale Q K^T (causal filter i >= j), online max-shifted
+//            softmax, O = P V, LSE = m + ln z   (ddx issue #217 repro steps;
+//            LSE is ddx issue #243 item 2's saved number per row)
+//   backward P = exp(S - LSE) recomputed per score, dP = dO V^T,
+//            dS = P o (dP - D), dV = P^T dO, dK = scale dS^T Q, dQ = scale dS K
+//            (ddx PR #162 "What changed"; shift gradient dropped, issue #243
+//            item 1)
+//
+// Layout of the work: a row (query or key) is owned by TPR = DP/32 threads,
+// each holding 32 of its DP (d rounded up to 32/64/128) channels; dot
+// products are finished with TPR-wide shuffles. The other side streams
+// through shared memory in 32-row tiles. The backward runs two kernels, one
+// per key row (dK, dV) and one per query row (dQ), so no atomics are needed
+// and the results are deterministic.
+#include "common.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kRowsTile = 32;  // rows of the streamed side per shared-memory tile
+
+template <int TPR>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int off = 1; off < TPR; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// Loads rows [r0, r0 + 32) x channels [0, DP) of a [N][d] fp32 matrix into
+// shared memory, zero-filling rows >= N and channels >= d.
+template <int DP>
+__device__ __forceinline__ void load_tile(float (*dst)[DP], const float* src, int r0, int N,
+                                          int d) {
+  for (int idx = threadIdx.x; idx < kRowsTile * DP; idx += blockDim.x) {
+    const int r = idx / DP, c = idx % DP;
+    dst[r][c] = (r0 + r < N && c < d) ? src[static_cast<size_t>(r0 + r) * d + c] : 0.f;
+  }
+}
+
+template <int DP>
+__global__ void __launch_bounds__(128)
+    fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                   const float* __restrict__ v, float* __restrict__ o, float* __restrict__ lse,
+                   int N, int d, int causal, float scale) {
+  constexpr int TPR = DP / 32;
+  constexpr int R = 128 / TPR;  // rows per block
+  __shared__ float sK[kRowsTile][DP];
+  __shared__ float sV[kRowsTile][DP];
+  const int bh = blockIdx.y;
+  const int row = blockIdx.x * R + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
+  const float* qh = q + static_cast<size_t>(bh) * N * d;
+  const float* kh = k + static_cast<size_t>(bh) * N * d;
+  const float* vh = v + static_cast<size_t>(bh) * N * d;
+
+  float qr[32], acc[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const int ch = 32 * part + c;
+    qr[c] = (row < N && ch < d) ? qh[static_cast<size_t>(row) * d + ch] : 0.f;
+    acc[c] = 0.f;
+  }
+  float m = -INFINITY, z = 0.f;
+  const int last_row = min(N - 1, blockIdx.x * R + R - 1);
+  const int key_end = causal ? last_row + 1 : N;
+  for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
+    __syncthreads();
+    load_tile<DP>(sK, kh, k0, N, d);
+    load_tile<DP>(sV, vh, k0, N, d);
+    __syncthreads();
+    float s[kRowsTile];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kRowsTile; ++u) {
+      float part_dot = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) part_dot = fmaf(qr[c], sK[u][32 * part + c], part_dot);
+      const float dot = group_sum<TPR>(part_dot);
+      const int key = k0 + u;
+      const bool keep = key < N && (!causal || key <= row);
+      s[u] = keep ? dot * scale : -INFINITY;
+      mx = fmaxf(mx, s[u]);
+    }
+    const float m_new = fmaxf(m, mx);
+    if (m_new == -INFINITY) continue;  // nothing kept yet for this row
+    const float alpha = expf(m - m_new);
+    float zt = 0.f;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] *= alpha;
+#pragma unroll
+    for (int u = 0; u < kRowsTile; ++u) {
+      const float p = expf(s[u] - m_new);
+      zt += p;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = fmaf(p, sV[u][32 * part + c], acc[c]);
+    }
+    z = z * alpha + zt;
+    m = m_new;
+  }
+  if (row < N) {
+    const float inv = 1.f / z;
+    float* orow = o + (static_cast<size_t>(bh) * N + row) * d;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int ch = 32 * part + c;
+      if (ch < d) orow[ch] = acc[c] * inv;
+    }
+    if (part == 0) lse[static_cast<size_t>(bh) * N + row] = m + logf(z);
+  }
+}
+
+// dK, dV: one key row per thread group; query rows stream through shared memory.
+template <int DP>
+__global__ void __launch_bounds__(128)
+    bwd_dkdv_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                        const float* __restrict__ v, const float* __restrict__ dout,
+                        const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
+                        float* __restrict__ dk, float* __restrict__ dv, int N, int Np, int d,
+                        int causal, float scale) {
+  constexpr int TPR = DP / 32;
+  constexpr int R = 128 / TPR;
+  __shared__ float sQ[kRowsTile][DP];
+  __shared__ float sdO[kRowsTile][DP];
+  __shared__ float sL[kRowsTile], sD[kRowsTile];
+  const int bh = blockIdx.y;
+  const int key = blockIdx.x * R + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
+  const size_t off = static_cast<size_t>(bh) * N * d;
+  float kr[32], vr[32], gk[32], gv[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const int ch = 32 * part + c;
+    const bool in = key < N && ch < d;
+    kr[c] = in ? k[off + static_cast<size_t>(key) * d + ch] : 0.f;
+    vr[c] = in ? v[off + static_cast<size_t>(key) * d + ch] : 0.f;
+    gk[c] = gv[c] = 0.f;
+  }
+  const int first_key = blockIdx.x * R;
+  const int q_begin = causal ? (first_key / kRowsTile) * kRowsTile : 0;
+  for (int q0 = q_begin; q0 < N; q0 += kRowsTile) {
+    __syncthreads();
+    load_tile<DP>(sQ, q + off, q0, N, d);
+    load_tile<DP>(sdO, dout + off, q0, N, d);
+    if (threadIdx.x < kRowsTile) {
+      sL[threadIdx.x] = lse_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
+      sD[threadIdx.x] = d_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int u = 0; u < kRowsTile; ++u) {
+      const int qi = q0 + u;
+      float ps = 0.f, pd = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        ps = fmaf(sQ[u][32 * part + c], kr[c], ps);
+        pd = fmaf(sdO[u][32 * part + c], vr[c], pd);
+      }
+      const float s = group_sum<TPR>(ps) * scale;
+      const float dp = group_sum<TPR>(pd);
+      const bool keep = qi < N && key < N && (!causal || qi >= key);
+      const float p = keep ? expf(s - sL[u]) : 0.f;
+      const float ds = p * (dp - sD[u]);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        gv[c] = fmaf(p, sdO[u][32 * part + c], gv[c]);
+        gk[c] = fmaf(ds, sQ[u][32 * part + c], gk[c]);
+      }
+    }
+  }
+  if (key < N) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int ch = 32 * part + c;
+      if (ch < d) {
+        dk[off + static_cast<size_t>(key) * d + ch] = gk[c] * scale;
+        dv[off + static_cast<size_t>(key) * d + ch] = gv[c];
+      }
+    }
+  }
+}
+
+// dQ: one query row per thread group; key rows stream through shared memory.
+template <int DP>
+__global__ void __launch_bounds__(128)
+    bwd_dq_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                      const float* __restrict__ v, const float* __restrict__ dout,
+                      const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
+                      float* __restrict__ dq, int N, int Np, int d, int causal, float scale) {
+  constexpr int TPR = DP / 32;
+  constexpr int R = 128 / TPR;
+  __shared__ float sK[kRowsTile][DP];
+  __shared__ float sV[kRowsTile][DP];
+  const int bh = blockIdx.y;
+  const int row = blockIdx.x * R + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
+  const size_t off = static_cast<size_t>(bh) * N * d;
+  float qr[32], dor[32], g[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const int ch = 32 * part + c;
+    const bool in = row < N && ch < d;
+    qr[c] = in ? q[off + static_cast<size_t>(row) * d + ch] : 0.f;
+    dor[c] = in ? dout[off + static_cast<size_t>(row) * d + ch] : 0.f;
+    g[c] = 0.f;
+  }
+  const float Li = lse_pad[static_cast<size_t>(bh) * Np + min(row, Np - 1)];
+  const float Di = d_pad[static_cast<size_t>(bh) * Np + min(row, Np - 1)];
+  const int last_row = min(N - 1, blockIdx.x * R + R - 1);
+  const int key_end = causal ? last_row + 1 : N;
+  for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
+    __syncthreads();
+    load_tile<DP>(sK, k + off, k0, N, d);
+    load_tile<DP>(sV, v + off, k0, N, d);
+    __syncthreads();
+#pragma unroll 4
+    for (int u = 0; u < kRowsTile; ++u) {
+      const int key = k0 + u;
+      float ps = 0.f, pd = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        ps = fmaf(qr[c], sK[u][32 * part + c], ps);
+        pd = fmaf(dor[c], sV[u][32 * part + c], pd);
+      }
+      const float s = group_sum<TPR>(ps) * scale;
+      const float dp = group_sum<TPR>(pd);
+      const bool keep = row < N && key < N && (!causal || key <= row);
+      const float p = keep ? expf(s - Li) : 0.f;
+      const float ds = p * (dp - Di);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) g[c] = fmaf(ds, sK[u][32 * part + c], g[c]);
+    }
+  }
+  if (row < N) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int ch = 32 * part + c;
+      if (ch < d) dq[off + static_cast<size_t>(row) * d + ch] = g[c] * scale;
+    }
+  }
+}
+
+template <int DP>
+cudaError_t fwd_f32_dp(const float* q, const float* k, const float* v, float* o, float* lse,
+                       int BH, int N, int d, bool causal, float scale, cudaStream_t s) {
+  constexpr int R = 128 / (DP / 32);
+  dim3 grid((N + R - 1) / R, BH);
+  fwd_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, o, lse, N, d, causal, scale);
+  return cudaGetLastError();
+}
+
+template <int DP>
+cudaError_t bwd_f32_dp(const float* q, const float* k, const float* v, const float* dout,
+                       float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
+                       float scale, const Workspace& ws, cudaStream_t s) {
+  constexpr int R = 128 / (DP / 32);
+  dim3 grid((N + R - 1) / R, BH);
+  bwd_dkdv_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dk, dv, N,
+                                               ws.Np, d, causal, scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dq, N, ws.Np,
+                                             d, causal, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                           int BH, int N, int d, bool causal, float scale, cudaStream_t s) {
+  if (d <= 32) return fwd_f32_dp<32>(q, k, v, o, lse, BH, N, d, causal, scale, s);
+  if (d <= 64) return fwd_f32_dp<64>(q, k, v, o, lse, BH, N, d, causal, scale, s);
+  return fwd_f32_dp<128>(q, k, v, o, lse, BH, N, d, causal, scale, s);
+}
+
+cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
+                           float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
+                           float scale, const Workspace& ws, cudaStream_t s) {
+  if (d <= 32) return bwd_f32_dp<32>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
+  if (d <= 64) return bwd_f32_dp<64>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
+  return bwd_f32_dp<128>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
+}
+
+}  // namespace csa

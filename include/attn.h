@@ -1,0 +1,149 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) causal softmax attention library.
+ *
+ * The library computes batched, multi-head softmax attention (causal or full)
+ * and its backward pass, dQ, dK, dV from Q, K, V, O, dO and the per-row
+ * log-sum-exp. The scores are recomputed tile by tile inside the backward from
+ * Q, K and one saved number per row, LSE = m + log z, so no N x N tensor is
+ * ever written to device memory (ddx issue #243, "Attention's gradient: a
+ * softmax shift's backward computed twice, and recomputing scores instead of
+ * saving them", item 2). The max-shift's gradient is dropped, since it
+ * cancels in w / z (same issue, item 1); the backward uses the row term
+ * D_i = sum_c dO_ic O_ic instead.
+ *
+ * Layout. Every matrix argument is a DEVICE pointer to a contiguous
+ * [B][H][N][d] row-major array (batch, head, position, channel), of the
+ * element type `dtype` (ATTN_F32: float, ATTN_BF16: bfloat16 bits). LSE is a
+ * device [B][H][N] float array in natural-log units: LSE_i = m_i + ln z_i of
+ * the SCALED scores s_ij = scale * q_i . k_j (the scale is applied before the
+ * max, as in ddx issue #217's repro, `SUM(q.val * k.val) / 2.0`). With
+ * causal != 0 position i sees keys j <= i (diagonal included, the repro's
+ * `WHERE q.pos >= k.pos`); causal == 0 is full attention. N_q == N_k == N.
+ *
+ * Ownership. The caller allocates and frees every buffer, the backward's
+ * workspace included. The library never allocates or frees device memory,
+ * never synchronises the host with the device (except attn_last_status),
+ * and enqueues all work on `stream` (a cudaStream_t passed as void*; NULL is
+ * the legacy default stream).
+ *
+ * Errors. Arguments are checked before anything is launched:
+ *   null pointers, B, H, N <= 0, d <= 0, non-finite scale, pointers that are
+ *   not 16-byte aligned, a workspace smaller than attn_bwd_workspace_bytes
+ *     -> ATTN_ERR_INVALID
+ *   (dtype, d) outside the built set: bf16 with d in {32, 64, 128}, f32 with
+ *   1 <= d <= 128 -> ATTN_ERR_UNSUPPORTED
+ *   a failed launch or a non-sm_100 device -> ATTN_ERR_CUDA
+ * Device-side waits are bounded; a wait that runs out writes ATTN_ERR_TIMEOUT
+ * into a status word (the workspace's for the backward, a library-owned one
+ * for the forward) and the kernel returns without trapping. Input VALUES are
+ * not validated: NaN and infinities propagate as IEEE arithmetic carries them.
+ */
+#ifndef CSA_ATTN_H_
+#define CSA_ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = -1,
+  ATTN_ERR_UNSUPPORTED = -2,
+  ATTN_ERR_CUDA = -3,
+  ATTN_ERR_TIMEOUT = -4
+} attn_status;
+
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/*
+ * Forward: O = softmax(scale * Q K^T, causal filter) V and LSE = m + ln z per
+ * row (ddx issue #217's repro: the `scores`, `weights`, `norm` and `heads`
+ * steps; LSE is the saved number of ddx issue #243, item 2).
+ *   q, k, v : in,  [B][H][N][d] of dtype
+ *   o       : out, [B][H][N][d] of dtype
+ *   lse     : out, [B][H][N] float
+ * Returns an attn_status.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, int causal, float scale, int dtype, void* stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs for this shape: a status word, the
+ * row terms D and LSE (padded to whole 128-row tiles) and, for bf16, an fp32
+ * dQ accumulator. Returns 0 for arguments attn_bwd would reject.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int dtype);
+
+/*
+ * Backward: given dO = dL/dO, writes
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
+ *   dS = P o (dP - D),  dQ = scale dS K,  dK = scale dS^T Q
+ * (ddx PR #162, "perf(ddx-ad): transpose causal attention's contractions
+ * without their joins", "What changed": transpose p = w / z per score, then
+ * p @ v; ddx issue #243 items 1-2 for dropping the shift and using D).
+ *   q, k, v, o, dout : in,  [B][H][N][d] of dtype (o from attn_fwd)
+ *   lse              : in,  [B][H][N] float (from attn_fwd)
+ *   dq, dk, dv       : out, [B][H][N][d] of dtype
+ *   workspace        : device scratch of >= attn_bwd_workspace_bytes bytes,
+ *                      16-byte aligned; contents need not be initialised
+ * Runs three stream-ordered kernels: attn_bwd_preprocess, attn_bwd_main and
+ * (bf16 only) attn_bwd_dq_convert.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+             int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+             void* stream);
+
+/*
+ * The three stages attn_bwd runs, exposed so a caller can time or overlap them
+ * separately. Same arguments and checks as attn_bwd; they must be enqueued in
+ * this order on one stream with the same workspace.
+ *   preprocess : D_i = sum_c dO_ic O_ic, the padded LSE copy, zeroes the dQ
+ *                accumulator and the status word
+ *   main       : the tile loop (scores recomputed from Q, K, LSE; dV, dK; dQ
+ *                partial sums). For f32 it also writes dq.
+ *   dq_convert : dq = scale * accumulator, rounded to bf16 (bf16 only; a
+ *                no-op returning ATTN_OK for f32)
+ */
+int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
+                        int d, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                  void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                  int dtype, void* workspace, size_t workspace_bytes, void* stream);
+int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads the backward's device status word from `workspace` (synchronises the
+ * calling thread with the device). ATTN_OK, or ATTN_ERR_TIMEOUT if a bounded
+ * device wait ran out during the last attn_bwd on this workspace.
+ */
+int attn_last_status(const void* workspace);
+
+/*
+ * Same for the forward: reads (and clears) the library's forward status word
+ * on the current device. Synchronises.
+ */
+int attn_fwd_last_status(void);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(int status);
+
+/*
+ * Failure-detection hook for tests. Arms a one-shot fault for the NEXT bf16
+ * attn_bwd_main (or attn_bwd) call in this process: that launch withholds the
+ * signal that its first score tile is ready and runs its bounded waits with
+ * `wait_limit_ns` as the limit, so the waits run out, the kernel writes
+ * ATTN_ERR_TIMEOUT into the workspace status word, releases its tensor memory
+ * and returns. No fault, trap or unbounded wait is involved; the outputs of
+ * that call are undefined. Returns ATTN_ERR_INVALID for wait_limit_ns == 0.
+ */
+int attn_test_arm_timeout(unsigned long long wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_ATTN_H_ */

@@ -1,0 +1,121 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function that
+include/attn.h declares, sizes its workspace as documented and rejects bad
+arguments before touching the GPU (every call below returns during argument
+checking, so no CUDA call is made)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import causal_softmax_attention_b200 as csa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fname in os.listdir(os.path.join(ROOT, "include")):
+        if not fname.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fname)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(attn_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_last_status",
+                     "attn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(csa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(csa.EXPORTED) >= declared_functions()
+
+
+def test_status_strings():
+    assert csa.status_string(csa.ATTN_OK) == "ok"
+    assert "timed out" in csa.status_string(csa.ATTN_ERR_TIMEOUT)
+    assert csa.status_string(12345) == "unknown status"
+
+
+def up(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 1, 256, 64), (12, 4, 64, 32), (2, 16, 16384, 128),
+                                     (1, 4, 262144, 64), (3, 5, 1000, 128), (1, 1, 1, 32)])
+def test_workspace_bytes(B, H, N, d):
+    Np = (N + 127) // 128 * 128
+    rows = B * H * Np * 4
+    f32 = 256 + up(rows) + up(rows)
+    assert csa.attn_bwd_workspace_bytes(B, H, N, d, csa.ATTN_F32) == f32
+    assert csa.attn_bwd_workspace_bytes(B, H, N, d, csa.ATTN_BF16) == f32 + up(rows * d)
+
+
+def test_workspace_is_linear_in_n():
+    a = csa.attn_bwd_workspace_bytes(1, 4, 131072, 64, csa.ATTN_BF16)
+    b = csa.attn_bwd_workspace_bytes(1, 4, 262144, 64, csa.ATTN_BF16)
+    assert abs(b / a - 2.0) < 1e-3
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 1, 64, 64, 1), 0), ((1, 1, 0, 64, 1), 0), ((1, 1, 64, 48, 1), 0),
+    ((1, 1, 64, 256, 0), 0), ((1, 1, 64, 64, 7), 0)])
+def test_workspace_bytes_rejects(args, status):
+    assert csa.attn_bwd_workspace_bytes(*args) == status
+
+
+L = csa.library()
+A = 1 << 20  # a 16-byte aligned stand-in address; never dereferenced (calls fail in checks)
+
+
+def bwd(**over):
+    a = dict(q=A, k=A, v=A, o=A, do=A, lse=A, dq=A, dk=A, dv=A, B=1, H=1, N=64, d=64,
+             causal=1, scale=0.125, dt=csa.ATTN_BF16, ws=A, wsb=1 << 30, stream=None)
+    a.update(over)
+    return L.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                      a["dv"], a["B"], a["H"], a["N"], a["d"], a["causal"], a["scale"], a["dt"],
+                      a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), csa.ATTN_ERR_INVALID),
+    (dict(dv=None), csa.ATTN_ERR_INVALID),
+    (dict(k=A + 8), csa.ATTN_ERR_INVALID),
+    (dict(B=0), csa.ATTN_ERR_INVALID),
+    (dict(H=-1), csa.ATTN_ERR_INVALID),
+    (dict(N=0), csa.ATTN_ERR_INVALID),
+    (dict(scale=math.nan), csa.ATTN_ERR_INVALID),
+    (dict(scale=math.inf), csa.ATTN_ERR_INVALID),
+    (dict(d=48), csa.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256, dt=csa.ATTN_F32), csa.ATTN_ERR_UNSUPPORTED),
+    (dict(dt=3), csa.ATTN_ERR_UNSUPPORTED),
+    (dict(ws=None), csa.ATTN_ERR_INVALID),
+    (dict(wsb=100), csa.ATTN_ERR_INVALID),
+])
+def test_bwd_rejects_bad_arguments(over, status):
+    assert bwd(**over) == status
+
+
+def test_fwd_rejects_bad_arguments():
+    f = L.attn_fwd
+    assert f(None, A, A, A, A, 1, 1, 64, 64, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A + 4, 1, 1, 64, 64, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 96, 1, 0.125, 1, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(A, A, A, A, A, 1, 1, 64, 64, 1, math.nan, 1, None) == csa.ATTN_ERR_INVALID
+
+
+def test_stage_entry_points_reject_bad_arguments():
+    assert L.attn_bwd_preprocess(A, None, A, 1, 1, 64, 64, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+    assert L.attn_bwd_main(A, A, A, A, A, A, A, 1, 1, 64, 64, 1, 0.1, 1, A, 10, None) == csa.ATTN_ERR_INVALID
+    assert L.attn_bwd_dq_convert(A, 1, 1, 64, 40, 0.1, 1, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert L.attn_last_status(None) == csa.ATTN_ERR_INVALID
+    assert L.attn_test_arm_timeout(0) == csa.ATTN_ERR_INVALID

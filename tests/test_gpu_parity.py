@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64 oracle.
+
+Small and medium shapes are compared element by element over every output;
+the two long-sequence workloads (16,384 x 32 heads and 262,144 tokens) are
+compared on sampled query rows and on the last key rows, which the oracle
+computes one by one, plus identities that hold at any size.
+
+Tolerances (max |gpu - oracle| / max |oracle| per output): 1e-5 for the fp32
+path, 2e-2 for the bf16 path (bf16 inputs and outputs, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from seeded_inputs import CONFIGS, as_f64, draw
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+def rel(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
+
+
+@pytest.fixture(scope="module")
+def csa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import causal_softmax_attention_b200 as lib
+    return lib
+
+
+def run_gpu(csa, q, k, v, do, causal, scale):
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
+    o, lse = csa.forward(qd, kd, vd, causal, scale)
+    dq, dk, dv = csa.backward(qd, kd, vd, o, dod, lse, causal, scale)
+    torch.cuda.synchronize()
+    assert csa.attn_fwd_last_status() == 0
+    return {"O": o, "LSE": lse, "dQ": dq, "dK": dk, "dV": dv}
+
+
+def compare_full(csa, B, H, N, d, dtype, seed, causal=True, qk_gain=1.0):
+    q, k, v, do = draw(B, H, N, d, seed, dtype, qk_gain)
+    scale = d ** -0.5
+    g = run_gpu(csa, q, k, v, do, causal, scale)
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), scale, causal)
+    tol = TOL[dtype]
+    errs = {name: rel(as_f64(g[name].cpu()), ref[name]) for name in ("O", "dQ", "dK", "dV")}
+    lse_err = float(np.abs(as_f64(g["LSE"].cpu()) - ref["LSE"]).max())
+    for name, e in errs.items():
+        assert e <= tol, (name, e, errs)
+    assert lse_err <= (1e-5 if dtype == "f32" else 1e-3), lse_err
+    return errs
+
+
+# ------------------------------------------------------------------ the configs
+@pytest.mark.parametrize("name", ["c1", "c2_f32", "c2_bf16", "c3"])
+def test_config_parity(csa, name):
+    c = CONFIGS[name]
+    compare_full(csa, c.B, c.H, c.N, c.d, c.dtype, c.seed, c.causal, c.qk_gain)
+
+
+# ------------------------------------------------------------------ ragged / edge shapes
+@pytest.mark.parametrize("B,H,N,d,causal", [
+    (1, 2, 200, 64, True), (2, 1, 1000, 128, True), (1, 1, 1, 32, True),
+    (1, 1, 130, 128, True), (1, 1, 127, 64, True), (1, 3, 384, 32, False),
+    (2, 2, 257, 64, False), (1, 1, 129, 128, False), (3, 2, 640, 128, True),
+])
+def test_bf16_shapes(csa, B, H, N, d, causal):
+    compare_full(csa, B, H, N, d, "bf16", 100 + N, causal)
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", [
+    (1, 2, 100, 48, True), (1, 1, 1, 7, True), (2, 1, 70, 64, False), (1, 1, 300, 128, True),
+    (2, 3, 33, 1, True),
+])
+def test_f32_shapes(csa, B, H, N, d, causal):
+    compare_full(csa, B, H, N, d, "f32", 200 + N, causal)
+
+
+# ------------------------------------------------------------------ properties on the GPU
+def test_linearity_and_causality(csa):
+    B, H, N, d = 1, 2, 768, 64
+    q, k, v, do = draw(B, H, N, d, 7, "bf16")
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = csa.forward(qd, kd, vd)
+    g1 = csa.backward(qd, kd, vd, o, dod, lse)
+    g2 = csa.backward(qd, kd, vd, o, 2 * dod, lse)  # exact in bf16
+    for a, b in zip(g1, g2):
+        assert rel(as_f64(b.cpu()), 2 * as_f64(a.cpu())) <= 2e-2
+    i0 = 300
+    do0 = dod.clone()
+    do0[:, :, i0:] = 0
+    dq, dk, dv = csa.backward(qd, kd, vd, o, do0, lse)
+    assert torch.count_nonzero(dq[:, :, i0:]) == 0
+    assert torch.count_nonzero(dk[:, :, i0:]) == 0
+    assert torch.count_nonzero(dv[:, :, i0:]) == 0
+    # permuting heads permutes the outputs
+    perm = [1, 0]
+    op, lp = csa.forward(qd[:, perm].contiguous(), kd[:, perm].contiguous(), vd[:, perm].contiguous())
+    assert torch.equal(op, o[:, perm])
+    assert torch.equal(lp, lse[:, perm])
+
+
+def test_timeout_is_reported_and_context_survives(csa):
+    B, H, N, d = 1, 1, 256, 64
+    q, k, v, do = draw(B, H, N, d, 9, "bf16")
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = csa.forward(qd, kd, vd)
+    ws = csa.new_workspace(qd)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    assert csa.attn_test_arm_timeout(50_000_000) == csa.ATTN_OK  # 50 ms limit
+    csa.attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws)
+    assert csa.attn_last_status(ws) == csa.ATTN_ERR_TIMEOUT
+    # the next call is unaffected
+    csa.attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws)
+    assert csa.attn_last_status(ws) == csa.ATTN_OK
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), d ** -0.5, True)
+    assert rel(as_f64(dq.cpu()), ref["dQ"]) <= 2e-2
+
+
+def test_nonfinite_inputs_propagate(csa):
+    B, H, N, d = 1, 1, 256, 64
+    q, k, v, do = draw(B, H, N, d, 11, "bf16")
+    v[0, 0, 5, 3] = float("nan")
+    g = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    # row 5 of V reaches every O row that keeps key 5 (IEEE 0 * NaN may also
+    # reach the masked rows of the same tile; no claim is made about those)
+    assert torch.isnan(g["O"][0, 0, 5:, 3]).all()
+    assert not torch.isnan(g["O"][0, 0, :, :3]).any()
+
+
+# ------------------------------------------------------------------ full-size workloads
+def sampled_parity(csa, name, heads, n_rows=24, tail=128):
+    c = CONFIGS[name]
+    q, k, v, do = draw(c.B, c.H, c.N, c.d, c.seed, c.dtype, c.qk_gain)
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    g = run_gpu(csa, q, k, v, do, True, c.scale)
+    peak = torch.cuda.max_memory_allocated() - base
+    # memory is linear in N: inputs, outputs and workspace are O(B*H*N*d)
+    elems = c.B * c.H * c.N * c.d
+    assert peak <= elems * 2 * 12 + c.B * c.H * c.N * 64, peak
+    rng = np.random.default_rng(c.seed)
+    for (b, h) in heads:
+        rows = np.sort(np.concatenate([rng.choice(c.N, n_rows - 4, replace=False),
+                                       [0, 1, c.N // 2, c.N - 1]]))
+        qh, kh, vh, doh = (as_f64(t[b, h]) for t in (q, k, v, do))
+        r = oracle.query_rows(qh, kh, vh, doh, c.scale, rows, True)
+        gq = as_f64(g["dQ"][b, h].cpu())[rows]
+        assert rel(gq, r["dQ"]) <= TOL[c.dtype]
+        assert rel(as_f64(g["O"][b, h].cpu())[rows], r["O"]) <= TOL[c.dtype]
+        assert np.abs(as_f64(g["LSE"][b, h].cpu())[rows] - r["LSE"]).max() <= 1e-3
+        t = oracle.key_tail(qh, kh, vh, doh, c.scale, c.N - tail)
+        assert rel(as_f64(g["dK"][b, h].cpu())[-tail:], t["dK"]) <= TOL[c.dtype]
+        assert rel(as_f64(g["dV"][b, h].cpu())[-tail:], t["dV"]) <= TOL[c.dtype]
+    # identities over all positions: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
+    dk = g["dK"].double()
+    dv = g["dV"].double()
+    dod = do.to(dk.device).double()
+    assert (dk.sum(2).abs() <= 1e-2 * dk.abs().sum(2) + 1e-6).all()
+    assert ((dv.sum(2) - dod.sum(2)).abs() <= 1e-2 * dod.abs().sum(2) + 1e-3).all()
+    for t in g.values():
+        assert torch.isfinite(t).all()
+
+
+def test_long_sequence_16k_parity(csa):
+    sampled_parity(csa, "c4", heads=[(0, 0), (1, 15)])
+
+
+def test_long_sequence_262k_parity(csa):
+    sampled_parity(csa, "c5", heads=[(0, 0), (0, 3)], n_rows=16, tail=64)
