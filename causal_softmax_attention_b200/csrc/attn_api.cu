@@ -114,7 +114,7 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA
 
 struct FaultInjection {
   int armed = 0;
-  unsigned long long limit_ns = 0;
+  unsigned long long limit_cycles = 0;
 };
 FaultInjection g_fault;
 std::mutex g_fault_mu;
@@ -201,12 +201,12 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
       !make_map(&m.c, v, BH, N, d) || !make_map(&m.d, dout, BH, N, d))
     return ATTN_ERR_CUDA;
   int inject = 0;
-  unsigned long long limit = kWaitLimitNs;
+  unsigned long long limit = kWaitLimitCycles;
   {
     std::lock_guard<std::mutex> g(g_fault_mu);
     if (g_fault.armed) {
       inject = 1;
-      limit = g_fault.limit_ns;
+      limit = g_fault.limit_cycles;
       g_fault.armed = 0;
     }
   }
@@ -263,11 +263,11 @@ int attn_fwd_last_status(void) {
   return v;
 }
 
-int attn_test_arm_timeout(unsigned long long wait_limit_ns) {
-  if (wait_limit_ns == 0) return ATTN_ERR_INVALID;
+int attn_test_arm_timeout(unsigned long long wait_limit_cycles) {
+  if (wait_limit_cycles == 0) return ATTN_ERR_INVALID;
   std::lock_guard<std::mutex> g(g_fault_mu);
   g_fault.armed = 1;
-  g_fault.limit_ns = wait_limit_ns;
+  g_fault.limit_cycles = wait_limit_cycles;
   return ATTN_OK;
 }
 

@@ -72,7 +72,7 @@ struct BwdParams {
   int N, Np, T, BH;
   int causal;
   float scale, scale_log2;
-  uint64_t wait_ns;
+  uint64_t wait_cycles;
   int inject_fault;   // 1: never signal the first score tile (tests the timeout path)
 };
 
@@ -202,16 +202,16 @@ __global__ void __launch_bounds__(160, 1)
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_KV = idesc_bf16(128, D, false, true);
       constexpr uint32_t ID_Q = idesc_bf16(128, D, true, true);
-      bool ok = mbar_wait(&bars[B_KV], 0, p.wait_ns, abort_flag);
+      bool ok = mbar_wait(&bars[B_KV], 0, p.wait_cycles, abort_flag);
       const bool kv_waited = ok;
       for (int it = 0; ok && it < n_iter; ++it) {
         const int s = it % L::STAGES;
         const uint32_t ph = (it / L::STAGES) & 1;
         const uint32_t sQ = sbase + L::Q_OFF + s * L::TILE;
         const uint32_t sdO = sbase + L::DO_OFF + s * L::TILE;
-        if (!(ok = mbar_wait(&bars[B_QFULL + s], ph, p.wait_ns, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars[B_QFULL + s], ph, p.wait_cycles, abort_flag))) break;
         ++q_waited;
-        if (it > 0 && !(ok = mbar_wait(&bars[B_DQEMPTY], (it - 1) & 1, p.wait_ns, abort_flag)))
+        if (it > 0 && !(ok = mbar_wait(&bars[B_DQEMPTY], (it - 1) & 1, p.wait_cycles, abort_flag)))
           break;
         tc_fence_after();
         // S^T = K_j Q_i^T and dP^T = V_j dO_i^T (K = D)
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(160, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
         if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
-        if (!(ok = mbar_wait(&bars[B_PFULL], it & 1, p.wait_ns, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars[B_PFULL], it & 1, p.wait_cycles, abort_flag))) break;
         tc_fence_after();
         // dV_j += P^T dO_i ; dK_j += dS^T Q_i   (K = 128 queries)
 #pragma unroll
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(160, 1)
         mma_commit(&bars[B_DQFULL]);
         mma_commit(&bars[B_QEMPTY + s]);
         if (it + L::STAGES < n_iter) {
-          if (!(ok = mbar_wait(&bars[B_QEMPTY + s], ph, p.wait_ns, abort_flag))) break;
+          if (!(ok = mbar_wait(&bars[B_QEMPTY + s], ph, p.wait_cycles, abort_flag))) break;
           load_q(it + L::STAGES);
           ++q_loaded;
         }
@@ -250,13 +250,13 @@ __global__ void __launch_bounds__(160, 1)
       } else {
         fail();
         // Drain the loads still in flight (bounded) before the CTA exits.
-        if (!kv_waited) mbar_wait(&bars[B_KV], 0, p.wait_ns, never);
+        if (!kv_waited) mbar_wait(&bars[B_KV], 0, p.wait_cycles, never);
         for (int w = q_waited; w < q_loaded; ++w)
-          mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_ns, never);
+          mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_cycles, never);
       }
       // Every MMA this thread issued has finished before TMEM is freed.
       mma_commit(&bars[B_FINAL]);
-      mbar_wait(&bars[B_FINAL], 0, p.wait_ns, never);
+      mbar_wait(&bars[B_FINAL], 0, p.wait_cycles, never);
     }
     __syncwarp();
   } else {
@@ -264,14 +264,18 @@ __global__ void __launch_bounds__(160, 1)
     const int t = threadIdx.x;  // key row within the tile (S^T lanes), query row for dQ
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int key = j0 + t;
+    // Outcome of a wait, made uniform across the warp: the TMEM loads that
+    // follow are warp-collective, so a warp must never split on a timeout.
+    auto wait_w = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_cycles, abort_flag));
+    };
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % L::STAGES;
       const int i = i_begin + it;
       const int i0 = i * kTile;
-      if (!(ok = mbar_wait(&bars[B_QFULL + s], (it / L::STAGES) & 1, p.wait_ns, abort_flag)))
-        break;
-      if (!(ok = mbar_wait(&bars[B_SFULL], it & 1, p.wait_ns, abort_flag))) break;
+      if (!(ok = wait_w(&bars[B_QFULL + s], (it / L::STAGES) & 1))) break;
+      if (!(ok = wait_w(&bars[B_SFULL], it & 1))) break;
       tc_fence_after();
       const float* lse_s = s_lse + s * 128;
       const float* d_s = s_dv + s * 128;
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(160, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_PFULL]);
-      if (!(ok = mbar_wait(&bars[B_DQFULL], it & 1, p.wait_ns, abort_flag))) break;
+      if (!(ok = wait_w(&bars[B_DQFULL], it & 1))) break;
       tc_fence_after();
       // dQ partial sums of query row i0 + t -> fp32 accumulator (tile-major layout)
       const bool row_ok = i0 + t < p.N;
@@ -330,15 +334,17 @@ __global__ void __launch_bounds__(160, 1)
       tc_fence_before();
       mbar_arrive(&bars[B_DQEMPTY]);
     }
-    if (ok) ok = mbar_wait(&bars[B_DONE], 0, p.wait_ns, abort_flag);
+    if (ok) ok = wait_w(&bars[B_DONE], 0);
     if (!ok) {
       fail();
     } else {
       tc_fence_after();
-      // Epilogue: dV_j and scale * dK_j rows -> bf16
-      if (key < p.N) {
-        __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + key) * D;
-        __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + key) * D;
+      // Epilogue: dV_j and scale * dK_j rows -> bf16. Every lane takes part in
+      // the warp-collective TMEM loads; only the stores are predicated.
+      const bool key_ok = key < p.N;
+      __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
+      __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
+      {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rv[32], rk[32];
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(160, 1)
           tmem_ld32(lane_base + L::T_DK + 32 * c, rk);
           tmem_ld_wait();
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 4 && key_ok; ++v) {
             uint4 ov, ok4;
             ov.x = pack_bf16x2(__uint_as_float(rv[8 * v + 0]), __uint_as_float(rv[8 * v + 1]));
             ov.y = pack_bf16x2(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3]));
@@ -377,7 +383,7 @@ __global__ void __launch_bounds__(160, 1)
 
 template <int D>
 cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, void* dv, int BH,
-                              int N, bool causal, float scale, uint64_t wait_ns, int inject,
+                              int N, bool causal, float scale, uint64_t wait_cycles, int inject,
                               cudaStream_t s) {
   using L = BwdLayout<D>;
   auto kern = attn_bwd_bf16_sm100_kernel<D>;
@@ -397,7 +403,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.wait_ns = wait_ns;
+  p.wait_cycles = wait_cycles;
   p.inject_fault = inject;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
   kern<<<grid, 160, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
@@ -407,17 +413,17 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
 }  // namespace
 
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
-                            int N, int d, bool causal, float scale, uint64_t wait_limit_ns,
+                            int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
                             int inject_fault, cudaStream_t s) {
   switch (d) {
     case 32:
-      return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+      return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
                                    inject_fault, s);
     case 64:
-      return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+      return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
                                    inject_fault, s);
     case 128:
-      return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_ns,
+      return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
                                     inject_fault, s);
     default:
       return cudaErrorInvalidValue;

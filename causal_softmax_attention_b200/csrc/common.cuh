@@ -32,8 +32,9 @@ struct WorkspaceLayout {
 WorkspaceLayout workspace_layout(int B, int H, int N, int d, int dtype);
 Workspace carve_workspace(void* base, const WorkspaceLayout& L);
 
-// Per-launch wait limit for device-side bounded waits (nanoseconds).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Limit of one device-side bounded wait, in SM clock cycles (about 1.1 s at
+// 1.9 GHz; a healthy wait lasts microseconds).
+constexpr uint64_t kWaitLimitCycles = 1ull << 31;
 
 // ---- launchers (return cudaError_t from the launch) ----
 cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse, int BH, int N,
@@ -53,7 +54,7 @@ struct TmaMaps {
 cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
                             int d, bool causal, float scale, cudaStream_t s);
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
-                            int N, int d, bool causal, float scale, uint64_t wait_limit_ns,
+                            int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
                             int inject_fault, cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device

@@ -65,7 +65,7 @@ struct FwdParams {
   int N, T, BH;
   int causal;
   float scale_log2;
-  uint64_t wait_ns;
+  uint64_t wait_cycles;
 };
 
 template <int D>
@@ -162,14 +162,14 @@ __global__ void __launch_bounds__(160, 1)
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_O = idesc_bf16(128, D, false, true);
       const uint32_t sQ = sbase + L::Q_OFF, sP = sbase + L::P_OFF;
-      bool ok = mbar_wait(&bars[F_Q], 0, p.wait_ns, abort_flag);
+      bool ok = mbar_wait(&bars[F_Q], 0, p.wait_cycles, abort_flag);
       const bool q_waited = ok;
       for (int jt = 0; ok && jt < n_kv; ++jt) {
         const int s = jt & 1;
         const uint32_t ph = (jt >> 1) & 1;
         const uint32_t sK = sbase + L::K_OFF + s * L::TILE;
         const uint32_t sV = sbase + L::V_OFF + s * L::TILE;
-        if (!(ok = mbar_wait(&bars[F_KVFULL + s], ph, p.wait_ns, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars[F_KVFULL + s], ph, p.wait_cycles, abort_flag))) break;
         ++waited;
         // S may be overwritten once the row threads have read S(jt-1) (they
         // arrive on F_PFULL after that).
@@ -178,9 +178,9 @@ __global__ void __launch_bounds__(160, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_S, fdesc_kmajor<D>(sQ, kk), fdesc_kmajor<D>(sK, kk), ID_S, kk > 0);
         mma_commit(&bars[F_SFULL]);
-        if (!(ok = mbar_wait(&bars[F_PFULL], jt & 1, p.wait_ns, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars[F_PFULL], jt & 1, p.wait_cycles, abort_flag))) break;
         // O_j lands where the threads read O_(jt-1); they arrive on F_OREAD after.
-        if (jt > 0 && !(ok = mbar_wait(&bars[F_OREAD], (jt - 1) & 1, p.wait_ns, abort_flag)))
+        if (jt > 0 && !(ok = mbar_wait(&bars[F_OREAD], (jt - 1) & 1, p.wait_cycles, abort_flag)))
           break;
         tc_fence_after();
 #pragma unroll
@@ -189,19 +189,19 @@ __global__ void __launch_bounds__(160, 1)
         mma_commit(&bars[F_OFULL]);
         mma_commit(&bars[F_KVEMPTY + s]);
         if (jt + 2 < n_kv) {
-          if (!(ok = mbar_wait(&bars[F_KVEMPTY + s], ph, p.wait_ns, abort_flag))) break;
+          if (!(ok = mbar_wait(&bars[F_KVEMPTY + s], ph, p.wait_cycles, abort_flag))) break;
           load_kv(jt + 2);
           ++loaded;
         }
       }
       if (!ok) {
         fail();
-        if (!q_waited) mbar_wait(&bars[F_Q], 0, p.wait_ns, never);
+        if (!q_waited) mbar_wait(&bars[F_Q], 0, p.wait_cycles, never);
         for (int w = waited; w < loaded; ++w)
-          mbar_wait(&bars[F_KVFULL + (w & 1)], (w >> 1) & 1, p.wait_ns, never);
+          mbar_wait(&bars[F_KVFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
       }
       mma_commit(&bars[F_FINAL]);
-      mbar_wait(&bars[F_FINAL], 0, p.wait_ns, never);
+      mbar_wait(&bars[F_FINAL], 0, p.wait_cycles, never);
     }
     __syncwarp();
   } else {
@@ -212,6 +212,10 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
     for (int c = 0; c < D; ++c) o[c] = 0.f;
     float m = -INFINITY, z = 0.f;
+    // Wait outcomes are made warp-uniform: the TMEM loads are warp-collective.
+    auto wait_w = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_cycles, abort_flag));
+    };
     bool ok = true;
     uint8_t* sP = smem + L::P_OFF;
     for (int jt = 0; jt < n_kv; ++jt) {
@@ -219,7 +223,7 @@ __global__ void __launch_bounds__(160, 1)
       // keys with local index >= lim are excluded for this row
       int lim = p.N - j0;
       if (p.causal && qrow - j0 + 1 < lim) lim = qrow - j0 + 1;
-      if (!(ok = mbar_wait(&bars[F_SFULL], jt & 1, p.wait_ns, abort_flag))) break;
+      if (!(ok = wait_w(&bars[F_SFULL], jt & 1))) break;
       tc_fence_after();
       float mx = -INFINITY;
 #pragma unroll 1
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(160, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[F_PFULL]);
-      if (!(ok = mbar_wait(&bars[F_OFULL], jt & 1, p.wait_ns, abort_flag))) break;
+      if (!(ok = wait_w(&bars[F_OFULL], jt & 1))) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -315,7 +319,7 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
   p.BH = BH;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.wait_ns = kWaitLimitNs;
+  p.wait_cycles = kWaitLimitCycles;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
   kern<<<grid, 160, L::ALLOC, s>>>(m.a, m.b, m.c, p);
   return cudaGetLastError();

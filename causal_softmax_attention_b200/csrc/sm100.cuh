@@ -58,20 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on phase `parity`. Returns false if `limit_ns` of wall time
-// passed without the phase completing, or if another thread of the CTA has
-// raised `*abort`; the caller then reports a timeout instead of spinning
-// forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+// Bounded wait on phase `parity`. Returns false once `limit_cycles` SM clock
+// cycles have passed without the phase completing, or once another thread of
+// the CTA has raised `*abort`; the caller then reports a timeout instead of
+// spinning forever. The SM cycle counter is used because it always advances.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_cycles,
                                           const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+    if (static_cast<uint64_t>(clock64() - t0) > limit_cycles) return false;
   }
 }
 
@@ -162,8 +162,11 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
-// lane (warp's subpartition base + t), columns [col, col + 32).
+// lane (warp's subpartition base + t), columns [col, col + 32). The
+// instruction is warp-collective (.sync.aligned): every lane must execute it,
+// so the warp is reconverged first.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -182,6 +185,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"

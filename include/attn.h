@@ -134,13 +134,14 @@ const char* attn_status_string(int status);
 /*
  * Failure-detection hook for tests. Arms a one-shot fault for the NEXT bf16
  * attn_bwd_main (or attn_bwd) call in this process: that launch withholds the
- * signal that its first score tile is ready and runs its bounded waits with
- * `wait_limit_ns` as the limit, so the waits run out, the kernel writes
- * ATTN_ERR_TIMEOUT into the workspace status word, releases its tensor memory
- * and returns. No fault, trap or unbounded wait is involved; the outputs of
- * that call are undefined. Returns ATTN_ERR_INVALID for wait_limit_ns == 0.
+ * signal that its first score tile is ready and bounds each of its device
+ * waits by `wait_limit_cycles` SM clock cycles, so the waits run out, the
+ * kernel writes ATTN_ERR_TIMEOUT into the workspace status word, releases its
+ * tensor memory and returns. No fault, trap or unbounded wait is involved; the
+ * outputs of that call are undefined. Returns ATTN_ERR_INVALID for
+ * wait_limit_cycles == 0.
  */
-int attn_test_arm_timeout(unsigned long long wait_limit_ns);
+int attn_test_arm_timeout(unsigned long long wait_limit_cycles);
 
 #ifdef __cplusplus
 }

@@ -115,7 +115,7 @@ def test_timeout_is_reported_and_context_survives(csa):
     o, lse = csa.forward(qd, kd, vd)
     ws = csa.new_workspace(qd)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    assert csa.attn_test_arm_timeout(50_000_000) == csa.ATTN_OK  # 50 ms limit
+    assert csa.attn_test_arm_timeout(50_000_000) == csa.ATTN_OK  # ~25 ms of SM cycles
     csa.attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws)
     assert csa.attn_last_status(ws) == csa.ATTN_ERR_TIMEOUT
     # the next call is unaffected
