@@ -80,7 +80,7 @@ def dram_traffic_per_launch(cfg):
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -94,7 +94,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -108,7 +108,10 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and active throttle reasons of the samples taken
+        between host times t0 and t1 (the timed region), or of all samples."""
+        import datetime
         if self.proc is None or self.file is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.file.flush()
@@ -121,6 +124,12 @@ class ClockSampler:
             if len(r) < 9:
                 continue
             try:
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            if t0 is not None and ts is not None and not (t0 <= ts <= t1):
+                continue
+            try:
                 sm.append(float(r[1]))
                 smax = float(r[2])
                 power.append(float(r[3]))
@@ -131,8 +140,7 @@ class ClockSampler:
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": len(sm),
                 "power_w_max": max(power) if power else None}
 
@@ -276,6 +284,8 @@ def run_gpu(args, cfg, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        time.sleep(1.0)  # let nvidia-smi start sampling before the timed region
+        host_t0 = time.time()
         t_begin = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_begin.record(stream)
@@ -285,6 +295,8 @@ def run_gpu(args, cfg, world, rank, local):
             ends[s].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+        host_t1 = time.time()
+        time.sleep(0.25)
     barrier(world)
     total_ms = t_begin.elapsed_time(t_end)
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
@@ -337,7 +349,7 @@ def run_gpu(args, cfg, world, rank, local):
     achieved = flops / (main_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = dram_traffic_per_launch(cfg)
-    clk = clocks.summary()
+    clk = clocks.summary(host_t0, host_t1)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -370,7 +382,7 @@ def run_gpu(args, cfg, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="c4", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

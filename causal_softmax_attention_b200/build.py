@@ -1,6 +1,6 @@
 """Build the CUDA library in-tree: every csrc/*.cu for sm_100a -> libcsa_attn.so.
 
-    python -m causal_softmax_attention_b200.build        # or build() from Python
+    python causal_softmax_attention_b200/build.py [-v]     # or __graft_entry__.build()
 
 The shared library lands next to this file so that it travels with the
 source tree; object files go to _build/ (git-ignored).

@@ -58,6 +58,9 @@ CONFIGS = {
     "c3": AttnConfig("c3", 1, 1, 1024, 64, "bf16", 2),
     "c4": AttnConfig("c4", 2, 16, 16384, 128, "bf16", 3),
     "c5": AttnConfig("c5", 1, 4, 262144, 64, "bf16", 4, qk_gain=0.5),
+    # a quarter of c4 (8 heads): still larger than L2, small enough for a
+    # many-pass profiler capture
+    "prof_d128": AttnConfig("prof_d128", 1, 8, 16384, 128, "bf16", 5),
 }
 
 
