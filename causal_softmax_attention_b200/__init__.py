@@ -6,7 +6,7 @@ CUDA kernels. Tensor arguments are torch tensors (device memory and streams
 are torch's plumbing); raw-pointer variants take integers. If the shared
 library is missing, importing this package raises: there is no CPU fallback.
 
-Build the library with ``python -m causal_softmax_attention_b200.build``.
+Build the library with ``python causal_softmax_attention_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -37,7 +37,7 @@ class AttnError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m causal_softmax_attention_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python causal_softmax_attention_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -52,6 +52,7 @@ def _load() -> ctypes.CDLL:
         "attn_fwd_last_status": (i, []),
         "attn_status_string": (ctypes.c_char_p, [i]),
         "attn_test_arm_timeout": (i, [ctypes.c_ulonglong]),
+        "attn_bwd_noalloc": (i, [vp] * 9 + [i, i, i, i, i, f, i, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -63,7 +64,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
-            "attn_status_string", "attn_test_arm_timeout")
+            "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc")
 
 
 def library() -> ctypes.CDLL:

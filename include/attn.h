@@ -143,6 +143,35 @@ const char* attn_status_string(int status);
  */
 int attn_test_arm_timeout(unsigned long long wait_limit_cycles);
 
+/*
+ * Backward without any allocation, for callers that cannot call cudaMalloc:
+ * code running inside a host framework whose device memory is reserved by that
+ * framework's own pool (a plugin or custom operator that may not allocate),
+ * or latency-critical code that cannot afford an allocation, which may also
+ * synchronise the device. The pages have no counterpart: this is a
+ * deployment variant of attn_bwd, not part of the method.
+ *
+ * Same arguments, layout, results and checks as attn_bwd, minus the
+ * workspace: the scratch comes from a fixed device array of
+ * ATTN_BWD_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU
+ * that loads the library holds until the process exits. Shapes whose
+ * attn_bwd_workspace_bytes exceeds that size are rejected with
+ * ATTN_ERR_INVALID before anything is launched (for bf16 the need is about
+ * 4 * B * H * N * (d + 2) bytes).
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's
+ * contents (each call re-zeroes what must start at zero), so calls that
+ * overlap on the same GPU race: serialise them. Device-side timeouts are
+ * recorded in the array's status word, which this entry point does not
+ * expose. Returns an attn_status.
+ */
+#define ATTN_BWD_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                     int H, int N, int d, int causal, float scale, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
