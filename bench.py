@@ -152,13 +152,20 @@ def dist_env():
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Maximum of a per-rank time over all ranks (every rank takes part)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank processes its own copy of the workload, so the
+    job's throughput is all ranks' FLOPs over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
 def barrier(world: int):
@@ -312,7 +319,7 @@ def run_gpu(args, cfg, world, rank, local):
     status = csa.attn_last_status(ws)
     ms_per_step = max_over_ranks(total_ms / args.steps, world)
     flops = cfg.bwd_flops
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms_per_step)
 
     # ---- e2e through the public API with pinned host buffers
     hq, hk, hv, ho, hdo = (t.cpu().pin_memory() for t in (qd, kd, vd, o, dod))
@@ -340,7 +347,7 @@ def run_gpu(args, cfg, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(flops, world, e2e_ms)
 
     if rank != 0:
         return
