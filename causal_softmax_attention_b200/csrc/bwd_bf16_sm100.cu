@@ -6,21 +6,30 @@
 // instead of reading a stored N x N table (ddx issue #243, item 2):
 //
 //   S^T  = K_j Q_i^T                 (tcgen05 MMA -> TMEM, lanes = keys)
-//   P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)      (CUDA cores, MUFU)
+//   P^T  = exp2(S^T * scale*log2e - LSE_i*log2e) -> bf16, back into TMEM
 //   dP^T = V_j dO_i^T                (tcgen05 MMA -> TMEM)
-//   dS^T = P^T o (dP^T - D_i)        (CUDA cores; the max-shift's gradient is
-//                                     dropped, ddx issue #243, item 1)
-//   dV_j += P^T dO_i,  dK_j += dS^T Q_i   (tcgen05, accumulators stay in TMEM)
-//   dQ_i += dS K_j                   (tcgen05 -> TMEM -> fp32 red.add to HBM)
+//   dS^T = P^T o (dP^T - D_i)        (the max-shift's gradient is dropped,
+//                                     ddx issue #243, item 1) -> shared memory
+//   dV_j += P^T dO_i                 (tcgen05, A operand read from TMEM)
+//   dK_j += dS^T Q_i                 (tcgen05, accumulators stay in TMEM)
+//   dQ_i  = dS K_j                   (tcgen05 -> TMEM -> fp32 red.add to HBM)
 //
 // These are the transposes of ddx PR #162 ("transpose p = w / z per score,
 // then p @ v"). Masked (j > i) scores are zeroed in registers on the diagonal
 // tile; tiles above the diagonal are never visited.
 //
-// Warp roles: warps 0-3 (128 threads, one TMEM lane = one key row or one
-// query row each) do the element-wise work and the epilogues; warp 4 issues
-// the TMA loads and the MMAs from one elected lane. All hand-offs are
-// mbarriers; every wait is bounded and reports a timeout in the status word.
+// Warp roles (320 threads):
+//   warps 0-7  two element-wise warpgroups. Thread t of either group owns
+//              TMEM lane t (key j0+t for S^T / dP^T / dV / dK, query i0+t for
+//              dQ); group g handles query columns [64g, 64g+64) of each tile
+//              and half of the dQ / dK / dV channels.
+//   warp 8     MMA issuer (one elected lane).
+//   warp 9     TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
+//              the tile's LSE / D rows per query tile, two stages.
+// TMEM (512 columns): S^T [0,128) whose first columns receive P^T as bf16
+// (query q at column 64*(q/64) + (q%64)/2), dP^T [128,256), dV [256,256+d),
+// dK [256+d,256+2d); dQ over dP^T at d = 128, in its own columns otherwise.
+// Every hand-off is an mbarrier; every wait is bounded and reports a timeout.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -31,6 +40,11 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kComputeThreads = 256;  // warps 0-7
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr int kThreads = 320;
+
 template <int D>
 struct BwdLayout {
   static constexpr int CH = D >= 64 ? 64 : D;   // TMA box width (elements)
@@ -39,28 +53,35 @@ struct BwdLayout {
   static constexpr int CHUNK = kTile * ROWB;    // bytes of one [128][CH] box
   static constexpr int TILE = NCH * CHUNK;      // bytes of one [128][D] bf16 tile
   static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128B : kSwizzle64B;
-  static constexpr int STAGES = D == 128 ? 1 : 2;
+  static constexpr int STAGES = 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
-  static constexpr int Q_OFF = V_OFF + TILE;
-  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;
-  static constexpr int P_OFF = DO_OFF + STAGES * TILE;   // [128 keys][128 queries] bf16
-  static constexpr int DS_OFF = P_OFF + 32768;
-  static constexpr int LSE_OFF = DS_OFF + 32768;         // [STAGES][128] f32
-  static constexpr int DV_OFF = LSE_OFF + STAGES * 512;  // [STAGES][128] f32
+  static constexpr int Q_OFF = V_OFF + TILE;              // [STAGES] tiles
+  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;    // [STAGES] tiles
+  static constexpr int DS_OFF = DO_OFF + STAGES * TILE;   // [128 keys][128 queries] bf16
+  static constexpr int LSE_OFF = DS_OFF + 32768;          // [STAGES][128] f32
+  static constexpr int DV_OFF = LSE_OFF + STAGES * 512;   // [STAGES][128] f32
   static constexpr int BAR_OFF = DV_OFF + STAGES * 512;
-  static constexpr int MISC_OFF = BAR_OFF + 16 * 8;
+  static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
   static constexpr int BYTES = MISC_OFF + 64;
-  // + alignment slack; at least ~116 KB so that one CTA owns an SM's TMEM.
-  static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
+  // d = 128 fills the 227 KB window, so the window itself must be 1024-byte
+  // aligned (checked at run time); smaller d keep 1 KB of alignment slack and
+  // at least ~118 KB so that one CTA owns an SM's tensor memory.
+  static constexpr bool EXACT = D == 128;
+  static constexpr int ALLOC =
+      EXACT ? BYTES : ((BYTES + 1024) > 118 * 1024 ? BYTES + 1024 : 118 * 1024);
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr uint32_t T_DQ = D == 128 ? 0 : 256 + 2 * D;
+  static constexpr uint32_t T_DQ = D == 128 ? 128 : 256 + 2 * D;
+  static constexpr bool DQ_OVER_DP = D == 128;
   static constexpr uint32_t T_COLS = 512;
+  static constexpr int HALF_D = D / 2;  // dQ / dK / dV channels per element-wise group
 };
 
-enum Bar { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_PFULL, B_DQFULL, B_DQEMPTY,
-           B_DONE, B_FINAL, B_COUNT };
+enum Bar {
+  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DVDONE,
+  B_DQFULL, B_DQREAD, B_DONE, B_FINAL, B_COUNT
+};
 
 struct BwdParams {
   const float* lse2;  // [BH][Np], LSE * log2(e), +inf past N
@@ -76,8 +97,8 @@ struct BwdParams {
   int inject_fault;   // 1: never signal the first score tile (tests the timeout path)
 };
 
-// Shared-memory address of K-major operand rows [128][D] stored as D/CH boxes,
-// advanced to the kk-th 16-element K step.
+// K-major operand: rows [128][D] stored as D/CH swizzled boxes, advanced to
+// the kk-th 16-element K step.
 template <int D>
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
   using L = BwdLayout<D>;
@@ -86,39 +107,44 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
   return smem_desc(addr, 16, 8 * L::ROWB, L::SWZ);
 }
 
-// The same [128 rows][D] tile read as an MN-major B operand (rows = K,
-// columns = N), advanced to the kk-th 16-row K step.
+// The same [128 rows][D] tile read as an MN-major operand (rows = K,
+// columns = M or N), advanced to the kk-th 16-row K step.
 template <int D>
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
   using L = BwdLayout<D>;
   return smem_desc(tile + kk * 16 * L::ROWB, L::CHUNK, 8 * L::ROWB, L::SWZ);
 }
 
-// [128][128] bf16 tiles written by the compute warps (two 64-column boxes).
-__device__ __forceinline__ uint64_t desc_sq_kmajor(uint32_t tile, int kk) {
+// The [128 keys][128 queries] dS tile (two 64-query boxes, 128B swizzle).
+__device__ __forceinline__ uint64_t desc_ds_kmajor(uint32_t tile, int kk) {
   const int e = kk * 16;
   return smem_desc(tile + (e / 64) * 16384 + (e % 64) * 2, 16, 1024, kSwizzle128B);
 }
-__device__ __forceinline__ uint64_t desc_sq_mnmajor(uint32_t tile, int kk) {
+__device__ __forceinline__ uint64_t desc_ds_mnmajor(uint32_t tile, int kk) {
   return smem_desc(tile + kk * 16 * 128, 16384, 1024, kSwizzle128B);
 }
 
-// Byte offset of the 16-byte group `g` (8 bf16 columns, 0..15) of row `r` in a
-// [128][128] SW128 tile.
-__device__ __forceinline__ uint32_t sq_offset(int r, int g) {
+// Byte offset of 16-byte group `g` (8 bf16 columns, 0..15) of row `r` in the
+// dS tile.
+__device__ __forceinline__ uint32_t ds_offset(int r, int g) {
   return (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4);
 }
 
+// TMEM column of the bf16 P^T pair holding query q (q even).
+__host__ __device__ constexpr uint32_t p_col(int q) { return 64 * (q >> 6) + ((q & 63) >> 1); }
+
 template <int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
                                const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   using L = BwdLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = L::EXACT ? smem_raw
+                           : reinterpret_cast<uint8_t*>(
+                                 (reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                 ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
@@ -128,12 +154,18 @@ __global__ void __launch_bounds__(160, 1)
   const float* s_dv = reinterpret_cast<const float*>(smem + L::DV_OFF);
 
   const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
   const int jt = blockIdx.x / p.BH;  // longest-first: key tile 0 has the most query tiles
   const int bh = blockIdx.x % p.BH;
   const int j0 = jt * kTile;
   const int i_begin = p.causal ? jt : 0;
   const int n_iter = p.T - i_begin;
+
+  // Swizzled operands need a 1024-byte aligned window; nothing has been
+  // issued yet, so a misaligned window is reported and every thread returns.
+  if ((sbase & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(p.status, -3);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_KV], 1);
@@ -142,9 +174,12 @@ __global__ void __launch_bounds__(160, 1)
       mbar_init(&bars[B_QEMPTY + s], 1);
     }
     mbar_init(&bars[B_SFULL], 1);
-    mbar_init(&bars[B_PFULL], 128);
+    mbar_init(&bars[B_DPFULL], 1);
+    mbar_init(&bars[B_PFULL], kComputeThreads);
+    mbar_init(&bars[B_DSFULL], kComputeThreads);
+    mbar_init(&bars[B_DVDONE], 1);
     mbar_init(&bars[B_DQFULL], 1);
-    mbar_init(&bars[B_DQEMPTY], 128);
+    mbar_init(&bars[B_DQREAD], kComputeThreads);
     mbar_init(&bars[B_DONE], 1);
     mbar_init(&bars[B_FINAL], 1);
     *abort_flag = 0;
@@ -165,22 +200,25 @@ __global__ void __launch_bounds__(160, 1)
     atomicExch(p.status, kStatusTimeout);
   };
 
-  if (warp == 4) {
-    // ------------------------------------------------ TMA + MMA issuer
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       prefetch_tensormap(&tm_do);
-      const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
-      const uint32_t sP = sbase + L::P_OFF, sdS = sbase + L::DS_OFF;
       mbar_arrive_expect_tx(&bars[B_KV], 2 * L::TILE);
       for (int c = 0; c < L::NCH; ++c) {
         tma_load_3d(smem + L::K_OFF + c * L::CHUNK, &tm_k, &bars[B_KV], c * L::CH, j0, bh);
         tma_load_3d(smem + L::V_OFF + c * L::CHUNK, &tm_v, &bars[B_KV], c * L::CH, j0, bh);
       }
-      auto load_q = [&](int it) {
-        const int s = it % L::STAGES;
+      bool ok = true;
+      int issued = 0;
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it & 1;
+        if (it >= 2 &&
+            !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
+          break;
         const int i0 = (i_begin + it) * kTile;
         uint64_t* bar = &bars[B_QFULL + s];
         mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
@@ -194,65 +232,72 @@ __global__ void __launch_bounds__(160, 1)
                   bar);
         bulk_load(smem + L::DV_OFF + s * 512, p.dvec + static_cast<size_t>(bh) * p.Np + i0, 512,
                   bar);
-      };
-      const int pre = n_iter < L::STAGES ? n_iter : L::STAGES;
-      int q_loaded = 0, q_waited = 0;
-      for (int it = 0; it < pre; ++it, ++q_loaded) load_q(it);
-
+        ++issued;
+      }
+      if (!ok) fail();
+      // Every load issued has landed before the CTA can exit (bounded).
+      mbar_wait(&bars[B_KV], 0, p.wait_cycles, never);
+      for (int w = issued > 2 ? issued - 2 : 0; w < issued; ++w)
+        mbar_wait(&bars[B_QFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issuer
+    if (elect_one_sync()) {
+      const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sdS = sbase + L::DS_OFF;
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_KV = idesc_bf16(128, D, false, true);
       constexpr uint32_t ID_Q = idesc_bf16(128, D, true, true);
-      bool ok = mbar_wait(&bars[B_KV], 0, p.wait_cycles, abort_flag);
-      const bool kv_waited = ok;
+      auto wait = [&](int b, uint32_t parity) {
+        return mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag);
+      };
+      bool ok = wait(B_KV, 0);
       for (int it = 0; ok && it < n_iter; ++it) {
-        const int s = it % L::STAGES;
-        const uint32_t ph = (it / L::STAGES) & 1;
+        const int s = it & 1;
         const uint32_t sQ = sbase + L::Q_OFF + s * L::TILE;
         const uint32_t sdO = sbase + L::DO_OFF + s * L::TILE;
-        if (!(ok = mbar_wait(&bars[B_QFULL + s], ph, p.wait_cycles, abort_flag))) break;
-        ++q_waited;
-        if (it > 0 && !(ok = mbar_wait(&bars[B_DQEMPTY], (it - 1) & 1, p.wait_cycles, abort_flag)))
-          break;
+        if (!(ok = wait(B_QFULL + s, (it >> 1) & 1))) break;
+        // S^T overwrites the P^T columns that dV(it-1) read.
+        if (it > 0 && !(ok = wait(B_DVDONE, (it - 1) & 1))) break;
         tc_fence_after();
-        // S^T = K_j Q_i^T and dP^T = V_j dO_i^T (K = D)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_S, desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
+        if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
+        // At d = 128 dP^T overwrites dQ(it-1), which must have been read out.
+        if (L::DQ_OVER_DP && it > 0 && !(ok = wait(B_DQREAD, (it - 1) & 1))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
-        if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
-        if (!(ok = mbar_wait(&bars[B_PFULL], it & 1, p.wait_cycles, abort_flag))) break;
+        mma_commit(&bars[B_DPFULL]);
+        // dV_j += P^T dO_i, P^T read from TMEM (K = 128 queries, 16 per step)
+        if (!(ok = wait(B_PFULL, it & 1))) break;
         tc_fence_after();
-        // dV_j += P^T dO_i ; dK_j += dS^T Q_i   (K = 128 queries)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DV, desc_sq_kmajor(sP, kk), desc_mnmajor<D>(sdO, kk), ID_KV,
+          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(sdO, kk), ID_KV,
                  (it > 0 || kk > 0));
+        mma_commit(&bars[B_DVDONE]);
+        // dK_j += dS^T Q_i ; dQ_i = dS K_j   (dS from shared memory)
+        if (!(ok = wait(B_DSFULL, it & 1))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DK, desc_sq_kmajor(sdS, kk), desc_mnmajor<D>(sQ, kk), ID_KV,
+          mma_ss(tmem + L::T_DK, desc_ds_kmajor(sdS, kk), desc_mnmajor<D>(sQ, kk), ID_KV,
                  (it > 0 || kk > 0));
-        // dQ_i = dS K_j   (K = 128 keys)
+        if (!L::DQ_OVER_DP && it > 0 && !(ok = wait(B_DQREAD, (it - 1) & 1))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DQ, desc_sq_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
+          mma_ss(tmem + L::T_DQ, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
         mma_commit(&bars[B_DQFULL]);
         mma_commit(&bars[B_QEMPTY + s]);
-        if (it + L::STAGES < n_iter) {
-          if (!(ok = mbar_wait(&bars[B_QEMPTY + s], ph, p.wait_cycles, abort_flag))) break;
-          load_q(it + L::STAGES);
-          ++q_loaded;
-        }
       }
       if (ok) {
         mma_commit(&bars[B_DONE]);
       } else {
         fail();
-        // Drain the loads still in flight (bounded) before the CTA exits.
-        if (!kv_waited) mbar_wait(&bars[B_KV], 0, p.wait_cycles, never);
-        for (int w = q_waited; w < q_loaded; ++w)
-          mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_cycles, never);
       }
       // Every MMA this thread issued has finished before TMEM is freed.
       mma_commit(&bars[B_FINAL]);
@@ -260,115 +305,158 @@ __global__ void __launch_bounds__(160, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ element-wise warps 0-3
-    const int t = threadIdx.x;  // key row within the tile (S^T lanes), query row for dQ
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------ element-wise warps 0-7
+    const int t = threadIdx.x & 127;  // TMEM lane: key row (S^T, dV, dK) / query row (dQ)
+    const int g = threadIdx.x >> 7;   // query columns [64g, 64g+64), channels [g*D/2, ...)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int key = j0 + t;
-    // Outcome of a wait, made uniform across the warp: the TMEM loads that
+    // Outcome of a wait, made uniform across the warp: the TMEM accesses that
     // follow are warp-collective, so a warp must never split on a timeout.
-    auto wait_w = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_cycles, abort_flag));
+    auto wait_w = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
     };
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
-      const int s = it % L::STAGES;
+      const int s = it & 1;
       const int i = i_begin + it;
       const int i0 = i * kTile;
-      if (!(ok = wait_w(&bars[B_QFULL + s], (it / L::STAGES) & 1))) break;
-      if (!(ok = wait_w(&bars[B_SFULL], it & 1))) break;
-      tc_fence_after();
+      if (!(ok = wait_w(B_QFULL + s, (it >> 1) & 1))) break;  // LSE_i, D_i in shared memory
       const float* lse_s = s_lse + s * 128;
       const float* d_s = s_dv + s * 128;
       // queries with local index < thr are masked for this key row
       const int thr = key >= p.N ? 128 : ((p.causal && i == jt) ? t : 0);
-      uint8_t* sP = smem + L::P_OFF;
-      uint8_t* sdS = smem + L::DS_OFF;
+
+      // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e), written back as bf16
+      if (!(ok = wait_w(B_SFULL, it & 1))) break;
+      tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(lane_base + L::T_S + 32 * c, sr);
-        tmem_ld32(lane_base + L::T_DP + 32 * c, dr);
+      for (int c = 0; c < 2; ++c) {
+        const int qb = 64 * g + 32 * c;
+        uint32_t sr[32];
+        tmem_ld32(lane_base + L::T_S + qb, sr);
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int u = 0; u < 32; u += 2) {
-          const int q0 = 32 * c + u;
+          const int q0 = qb + u;
           float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -lse_s[q0]));
           float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -lse_s[q0 + 1]));
           if (q0 < thr) p0 = 0.f;
           if (q0 + 1 < thr) p1 = 0.f;
-          const float ds0 = p0 * (__uint_as_float(dr[u]) - d_s[q0]);
-          const float ds1 = p1 * (__uint_as_float(dr[u + 1]) - d_s[q0 + 1]);
           pk[u / 2] = pack_bf16x2(p0, p1);
+        }
+        // columns [p_col(qb), +16) lie inside this group's already-read S^T columns
+        tmem_st16(lane_base + L::T_S + p_col(qb), pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[B_PFULL]);
+
+      // ---- dS^T = P^T o (dP^T - D) -> shared memory (bf16)
+      if (!(ok = wait_w(B_DPFULL, it & 1))) break;
+      tc_fence_after();
+      uint8_t* sdS = smem + L::DS_OFF;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const int qb = 64 * g + 32 * c;
+        uint32_t dr[32], pr[16];
+        tmem_ld32(lane_base + L::T_DP + qb, dr);
+        tmem_ld16(lane_base + L::T_S + p_col(qb), pr);
+        tmem_ld_wait();
+        uint32_t dk[16];
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const int q0 = qb + u;
+          const float2 pp = unpack_bf16x2(pr[u / 2]);
+          const float ds0 = pp.x * (__uint_as_float(dr[u]) - d_s[q0]);
+          const float ds1 = pp.y * (__uint_as_float(dr[u + 1]) - d_s[q0 + 1]);
           dk[u / 2] = pack_bf16x2(ds0, ds1);
         }
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint32_t off = sq_offset(t, 4 * c + v);
-          st_shared_v4(smem_u32(sP) + off, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          st_shared_v4(smem_u32(sdS) + off, dk[4 * v], dk[4 * v + 1], dk[4 * v + 2],
-                       dk[4 * v + 3]);
-        }
+        for (int v = 0; v < 4; ++v)
+          st_shared_v4(smem_u32(sdS) + ds_offset(t, qb / 8 + v), dk[4 * v], dk[4 * v + 1],
+                       dk[4 * v + 2], dk[4 * v + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL]);
-      if (!(ok = wait_w(&bars[B_DQFULL], it & 1))) break;
+      mbar_arrive(&bars[B_DSFULL]);
+
+      // ---- dQ partial sums of query row i0 + t -> fp32 accumulator
+      if (!(ok = wait_w(B_DQFULL, it & 1))) break;
       tc_fence_after();
-      // dQ partial sums of query row i0 + t -> fp32 accumulator (tile-major layout)
       const bool row_ok = i0 + t < p.N;
       float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
+      if constexpr (L::HALF_D >= 32) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + L::T_DQ + 32 * c, r);
+        for (int c = 0; c < L::HALF_D / 32; ++c) {
+          const int ch = g * L::HALF_D + 32 * c;
+          uint32_t r[32];
+          tmem_ld32(lane_base + L::T_DQ + ch, r);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              red_add_v4(acc + (ch / 4 + v) * 512, __uint_as_float(r[4 * v]),
+                         __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                         __uint_as_float(r[4 * v + 3]));
+          }
+        }
+      } else {
+        const int ch = g * L::HALF_D;
+        uint32_t r[16];
+        tmem_ld16(lane_base + L::T_DQ + ch, r);
         tmem_ld_wait();
         if (row_ok) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(acc + (8 * c + v) * 512, __uint_as_float(r[4 * v]),
+          for (int v = 0; v < 4; ++v)
+            red_add_v4(acc + (ch / 4 + v) * 512, __uint_as_float(r[4 * v]),
                        __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
                        __uint_as_float(r[4 * v + 3]));
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars[B_DQEMPTY]);
+      mbar_arrive(&bars[B_DQREAD]);
     }
-    if (ok) ok = wait_w(&bars[B_DONE], 0);
+    if (ok) ok = wait_w(B_DONE, 0);
     if (!ok) {
       fail();
     } else {
       tc_fence_after();
-      // Epilogue: dV_j and scale * dK_j rows -> bf16. Every lane takes part in
-      // the warp-collective TMEM loads; only the stores are predicated.
+      // Epilogue: dV_j and scale * dK_j rows -> bf16, group g writing channels
+      // [g*D/2, (g+1)*D/2). All lanes load; only the stores are predicated.
       const bool key_ok = key < p.N;
       __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
       __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
-      {
+      constexpr int W = L::HALF_D >= 32 ? 32 : 16;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rv[32], rk[32];
-          tmem_ld32(lane_base + L::T_DV + 32 * c, rv);
-          tmem_ld32(lane_base + L::T_DK + 32 * c, rk);
-          tmem_ld_wait();
+      for (int c = 0; c < L::HALF_D / W; ++c) {
+        const int ch = g * L::HALF_D + W * c;
+        uint32_t rv[W], rk[W];
+        if constexpr (W == 32) {
+          tmem_ld32(lane_base + L::T_DV + ch, rv);
+          tmem_ld32(lane_base + L::T_DK + ch, rk);
+        } else {
+          tmem_ld16(lane_base + L::T_DV + ch, rv);
+          tmem_ld16(lane_base + L::T_DK + ch, rk);
+        }
+        tmem_ld_wait();
 #pragma unroll
-          for (int v = 0; v < 4 && key_ok; ++v) {
-            uint4 ov, ok4;
-            ov.x = pack_bf16x2(__uint_as_float(rv[8 * v + 0]), __uint_as_float(rv[8 * v + 1]));
-            ov.y = pack_bf16x2(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3]));
-            ov.z = pack_bf16x2(__uint_as_float(rv[8 * v + 4]), __uint_as_float(rv[8 * v + 5]));
-            ov.w = pack_bf16x2(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7]));
-            ok4.x = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 0]),
-                                p.scale * __uint_as_float(rk[8 * v + 1]));
-            ok4.y = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 2]),
-                                p.scale * __uint_as_float(rk[8 * v + 3]));
-            ok4.z = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 4]),
-                                p.scale * __uint_as_float(rk[8 * v + 5]));
-            ok4.w = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 6]),
-                                p.scale * __uint_as_float(rk[8 * v + 7]));
-            *reinterpret_cast<uint4*>(dv_row + 32 * c + 8 * v) = ov;
-            *reinterpret_cast<uint4*>(dk_row + 32 * c + 8 * v) = ok4;
-          }
+        for (int v = 0; v < W / 8 && key_ok; ++v) {
+          uint4 ov, ok4;
+          ov.x = pack_bf16x2(__uint_as_float(rv[8 * v + 0]), __uint_as_float(rv[8 * v + 1]));
+          ov.y = pack_bf16x2(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3]));
+          ov.z = pack_bf16x2(__uint_as_float(rv[8 * v + 4]), __uint_as_float(rv[8 * v + 5]));
+          ov.w = pack_bf16x2(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7]));
+          ok4.x = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 0]),
+                              p.scale * __uint_as_float(rk[8 * v + 1]));
+          ok4.y = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 2]),
+                              p.scale * __uint_as_float(rk[8 * v + 3]));
+          ok4.z = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 4]),
+                              p.scale * __uint_as_float(rk[8 * v + 5]));
+          ok4.w = pack_bf16x2(p.scale * __uint_as_float(rk[8 * v + 6]),
+                              p.scale * __uint_as_float(rk[8 * v + 7]));
+          *reinterpret_cast<uint4*>(dv_row + ch + 8 * v) = ov;
+          *reinterpret_cast<uint4*>(dk_row + ch + 8 * v) = ok4;
         }
       }
     }
@@ -386,6 +474,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
                               int N, bool causal, float scale, uint64_t wait_cycles, int inject,
                               cudaStream_t s) {
   using L = BwdLayout<D>;
+  static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = attn_bwd_bf16_sm100_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
@@ -406,7 +495,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.wait_cycles = wait_cycles;
   p.inject_fault = inject;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
-  kern<<<grid, 160, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
+  kern<<<grid, kThreads, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
   return cudaGetLastError();
 }
 
