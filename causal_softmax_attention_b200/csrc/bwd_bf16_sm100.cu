@@ -9,26 +9,37 @@
 //   P^T  = exp2(S^T * scale*log2e - LSE_i*log2e) -> bf16, back into TMEM
 //   dP^T = V_j dO_i^T                (tcgen05 MMA -> TMEM)
 //   dS^T = P^T o (dP^T - D_i)        (the max-shift's gradient is dropped,
-//                                     ddx issue #243, item 1) -> shared memory
+//                                     ddx issue #243, item 1) -> bf16, into
+//                                     TMEM and into shared memory
 //   dV_j += P^T dO_i                 (tcgen05, A operand read from TMEM)
-//   dK_j += dS^T Q_i                 (tcgen05, accumulators stay in TMEM)
-//   dQ_i  = dS K_j                   (tcgen05 -> TMEM -> fp32 red.add to HBM)
+//   dK_j += dS^T Q_i                 (tcgen05, A operand read from TMEM;
+//                                     accumulators stay in TMEM)
+//   dQ_i  = dS K_j                   (tcgen05, A = the shared-memory dS tile
+//                                     read transposed -> TMEM -> fp32 red.add)
 //
 // These are the transposes of ddx PR #162 ("transpose p = w / z per score,
 // then p @ v"). Masked (j > i) scores are zeroed in registers on the diagonal
 // tile; tiles above the diagonal are never visited.
 //
-// Warp roles (320 threads):
-//   warps 0-7  two element-wise warpgroups. Thread t of either group owns
-//              TMEM lane t (key j0+t for S^T / dP^T / dV / dK, query i0+t for
-//              dQ); group g handles query columns [64g, 64g+64) of each tile
-//              and half of the dQ / dK / dV channels.
-//   warp 8     MMA issuer (one elected lane).
-//   warp 9     TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
-//              the tile's LSE / D rows per query tile, two stages.
-// TMEM (512 columns): S^T [0,128) whose first columns receive P^T as bf16
-// (query q at column 64*(q/64) + (q%64)/2), dP^T [128,256), dV [256,256+d),
-// dK [256+d,256+2d); dQ over dP^T at d = 128, in its own columns otherwise.
+// Warp roles (448 threads):
+//   warps 0-7   two element-wise warpgroups. Thread t of either group owns
+//               TMEM lane t (key j0+t for S^T / dP^T / dV / dK); group g
+//               handles query columns [64g, 64g+64) of each tile and half of
+//               the dK / dV channels in the epilogue.
+//   warp 8      MMA issuer (one elected lane).
+//   warp 9      TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
+//               the tile's LSE / D rows per query tile, two stages.
+//   warps 10-13 dQ warpgroup: thread (warp%4)*32 + lane owns query row i0 +
+//               that lane of the dQ tile; it copies the row out of TMEM,
+//               releases the columns, then adds it into the fp32 accumulator
+//               with red.global.add, so the atomics stay off the path of the
+//               element-wise warps and the MMAs.
+// TMEM (512 columns): S^T [0,128), whose columns then receive P^T and dS^T
+// as bf16 (query q's P at column 64*(q/64) + (q%64)/2, its dS 32 columns
+// further), dP^T [128,256), dV [256,256+d), dK [256+d,256+2d); dQ over dP^T
+// at d = 128, in its own columns otherwise. Shared-memory traffic is the
+// scarce resource (four of the five MMAs read 128 B/clk at this tile shape),
+// so P and dS feed their MMAs from TMEM wherever the operand shape allows.
 // Every hand-off is an mbarrier; every wait is bounded and reports a timeout.
 #include <cuda_bf16.h>
 
@@ -43,7 +54,9 @@ using namespace sm100;
 constexpr int kComputeThreads = 256;  // warps 0-7
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kDqWarp0 = 10;          // warps 10-13
+constexpr int kDqThreads = 128;
+constexpr int kThreads = 448;
 
 template <int D>
 struct BwdLayout {
@@ -75,11 +88,12 @@ struct BwdLayout {
   static constexpr uint32_t T_DQ = D == 128 ? 128 : 256 + 2 * D;
   static constexpr bool DQ_OVER_DP = D == 128;
   static constexpr uint32_t T_COLS = 512;
-  static constexpr int HALF_D = D / 2;  // dQ / dK / dV channels per element-wise group
+  static constexpr int HALF_D = D / 2;  // dK / dV channels per element-wise group
+  static constexpr int DQ_PASSES = D > 64 ? 2 : 1;  // TMEM read passes of the dQ warps
 };
 
 enum Bar {
-  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DVDONE,
+  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DKDONE,
   B_DQFULL, B_DQREAD, B_DONE, B_FINAL, B_COUNT
 };
 
@@ -115,11 +129,8 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
   return smem_desc(tile + kk * 16 * L::ROWB, L::CHUNK, 8 * L::ROWB, L::SWZ);
 }
 
-// The [128 keys][128 queries] dS tile (two 64-query boxes, 128B swizzle).
-__device__ __forceinline__ uint64_t desc_ds_kmajor(uint32_t tile, int kk) {
-  const int e = kk * 16;
-  return smem_desc(tile + (e / 64) * 16384 + (e % 64) * 2, 16, 1024, kSwizzle128B);
-}
+// The [128 keys][128 queries] dS tile (two 64-query boxes, 128B swizzle),
+// read as the MN-major A operand of dQ = dS K (M = queries, K = keys).
 __device__ __forceinline__ uint64_t desc_ds_mnmajor(uint32_t tile, int kk) {
   return smem_desc(tile + kk * 16 * 128, 16384, 1024, kSwizzle128B);
 }
@@ -130,11 +141,12 @@ __device__ __forceinline__ uint32_t ds_offset(int r, int g) {
   return (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4);
 }
 
-// TMEM column of the bf16 P^T pair holding query q (q even).
+// TMEM columns of the bf16 pairs holding query q (q even) of P^T and dS^T.
 __host__ __device__ constexpr uint32_t p_col(int q) { return 64 * (q >> 6) + ((q & 63) >> 1); }
+__host__ __device__ constexpr uint32_t ds_col(int q) { return p_col(q) + 32; }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(128)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
@@ -177,9 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_DPFULL], 1);
     mbar_init(&bars[B_PFULL], kComputeThreads);
     mbar_init(&bars[B_DSFULL], kComputeThreads);
-    mbar_init(&bars[B_DVDONE], 1);
+    mbar_init(&bars[B_DKDONE], 1);
     mbar_init(&bars[B_DQFULL], 1);
-    mbar_init(&bars[B_DQREAD], kComputeThreads);
+    mbar_init(&bars[B_DQREAD], kDqThreads);
     mbar_init(&bars[B_DONE], 1);
     mbar_init(&bars[B_FINAL], 1);
     *abort_flag = 0;
@@ -257,8 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sQ = sbase + L::Q_OFF + s * L::TILE;
         const uint32_t sdO = sbase + L::DO_OFF + s * L::TILE;
         if (!(ok = wait(B_QFULL + s, (it >> 1) & 1))) break;
-        // S^T overwrites the P^T columns that dV(it-1) read.
-        if (it > 0 && !(ok = wait(B_DVDONE, (it - 1) & 1))) break;
+        // S^T overwrites the P^T / dS^T columns that dV(it-1) and dK(it-1)
+        // read; dK(it-1) was issued after dV(it-1).
+        if (it > 0 && !(ok = wait(B_DKDONE, (it - 1) & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -278,14 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(sdO, kk), ID_KV,
                  (it > 0 || kk > 0));
-        mma_commit(&bars[B_DVDONE]);
-        // dK_j += dS^T Q_i ; dQ_i = dS K_j   (dS from shared memory)
+        // dK_j += dS^T Q_i (dS^T from TMEM) ; dQ_i = dS K_j (dS from shared memory)
         if (!(ok = wait(B_DSFULL, it & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DK, desc_ds_kmajor(sdS, kk), desc_mnmajor<D>(sQ, kk), ID_KV,
+          mma_ts(tmem + L::T_DK, tmem + L::T_S + ds_col(16 * kk), desc_mnmajor<D>(sQ, kk), ID_KV,
                  (it > 0 || kk > 0));
+        mma_commit(&bars[B_DKDONE]);
         if (!L::DQ_OVER_DP && it > 0 && !(ok = wait(B_DQREAD, (it - 1) & 1))) break;
         tc_fence_after();
 #pragma unroll
@@ -304,6 +317,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[B_FINAL], 0, p.wait_cycles, never);
     }
     __syncwarp();
+  } else if (warp >= kDqWarp0) {
+    // ------------------------------------------------ dQ warpgroup (warps 10-13)
+    const int t = ((warp & 3) << 5) | (threadIdx.x & 31);  // TMEM lane = query row
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    auto wait_w = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
+    };
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int i = i_begin + it;
+      if (!(ok = wait_w(B_DQFULL, it & 1))) break;
+      tc_fence_after();
+      const bool row_ok = i * kTile + t < p.N;
+      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
+      // At most 64 channels per pass: 128 registers a thread is the ceiling
+      // for 14 warps (four of them share one SM sub-partition's 16K registers).
+#pragma unroll
+      for (int h = 0; h < L::DQ_PASSES; ++h) {
+        constexpr int W = D / L::DQ_PASSES;
+        uint32_t r[W];
+#pragma unroll
+        for (int c = 0; c < W; c += 16)
+          tmem_ld16(lane_base + L::T_DQ + h * W + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        tmem_ld_wait();
+        if (h == L::DQ_PASSES - 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_DQREAD]);  // the dQ columns are free again
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < W / 4; ++v)
+            red_add_v4(acc + (h * W / 4 + v) * 512, __uint_as_float(r[4 * v]),
+                       __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                       __uint_as_float(r[4 * v + 3]));
+        }
+      }
+    }
+    if (!ok) fail();
   } else {
     // ------------------------------------------------ element-wise warps 0-7
     const int t = threadIdx.x & 127;  // TMEM lane: key row (S^T, dV, dK) / query row (dQ)
@@ -337,13 +388,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
+        for (int u = 0; u < 32; u += 4) {
           const int q0 = qb + u;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -lse_s[q0]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -lse_s[q0 + 1]));
+          // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q0);
+          float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -l4.x));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -l4.y));
+          float p2 = ex2_approx(fmaf(__uint_as_float(sr[u + 2]), p.scale_log2, -l4.z));
+          float p3 = ex2_approx(fmaf(__uint_as_float(sr[u + 3]), p.scale_log2, -l4.w));
           if (q0 < thr) p0 = 0.f;
           if (q0 + 1 < thr) p1 = 0.f;
+          if (q0 + 2 < thr) p2 = 0.f;
+          if (q0 + 3 < thr) p3 = 0.f;
           pk[u / 2] = pack_bf16x2(p0, p1);
+          pk[u / 2 + 1] = pack_bf16x2(p2, p3);
         }
         // columns [p_col(qb), +16) lie inside this group's already-read S^T columns
         tmem_st16(lane_base + L::T_S + p_col(qb), pk);
@@ -365,57 +423,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         uint32_t dk[16];
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
+        for (int u = 0; u < 32; u += 4) {
           const int q0 = qb + u;
-          const float2 pp = unpack_bf16x2(pr[u / 2]);
-          const float ds0 = pp.x * (__uint_as_float(dr[u]) - d_s[q0]);
-          const float ds1 = pp.y * (__uint_as_float(dr[u + 1]) - d_s[q0 + 1]);
-          dk[u / 2] = pack_bf16x2(ds0, ds1);
+          const float4 d4 = *reinterpret_cast<const float4*>(d_s + q0);
+          const float2 pa = unpack_bf16x2(pr[u / 2]);
+          const float2 pb = unpack_bf16x2(pr[u / 2 + 1]);
+          dk[u / 2] = pack_bf16x2(pa.x * (__uint_as_float(dr[u]) - d4.x),
+                                  pa.y * (__uint_as_float(dr[u + 1]) - d4.y));
+          dk[u / 2 + 1] = pack_bf16x2(pb.x * (__uint_as_float(dr[u + 2]) - d4.z),
+                                      pb.y * (__uint_as_float(dr[u + 3]) - d4.w));
         }
+        // dS^T for dK (TMEM A operand); these S^T columns were read in the P pass
+        tmem_st16(lane_base + L::T_S + ds_col(qb), dk);
+        // dS for dQ (shared memory, read transposed by the MMA)
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           st_shared_v4(smem_u32(sdS) + ds_offset(t, qb / 8 + v), dk[4 * v], dk[4 * v + 1],
                        dk[4 * v + 2], dk[4 * v + 3]);
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_DSFULL]);
 
-      // ---- dQ partial sums of query row i0 + t -> fp32 accumulator
-      if (!(ok = wait_w(B_DQFULL, it & 1))) break;
-      tc_fence_after();
-      const bool row_ok = i0 + t < p.N;
-      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
-      if constexpr (L::HALF_D >= 32) {
-#pragma unroll 1
-        for (int c = 0; c < L::HALF_D / 32; ++c) {
-          const int ch = g * L::HALF_D + 32 * c;
-          uint32_t r[32];
-          tmem_ld32(lane_base + L::T_DQ + ch, r);
-          tmem_ld_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              red_add_v4(acc + (ch / 4 + v) * 512, __uint_as_float(r[4 * v]),
-                         __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
-                         __uint_as_float(r[4 * v + 3]));
-          }
-        }
-      } else {
-        const int ch = g * L::HALF_D;
-        uint32_t r[16];
-        tmem_ld16(lane_base + L::T_DQ + ch, r);
-        tmem_ld_wait();
-        if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            red_add_v4(acc + (ch / 4 + v) * 512, __uint_as_float(r[4 * v]),
-                       __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
-                       __uint_as_float(r[4 * v + 3]));
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_DQREAD]);
     }
     if (ok) ok = wait_w(B_DONE, 0);
     if (!ok) {
