@@ -21,27 +21,31 @@
 // then p @ v"). Masked (j > i) scores are zeroed in registers on the diagonal
 // tile; tiles above the diagonal are never visited.
 //
-// Warp roles (448 threads):
+// Warp roles (512 threads, four warpgroups):
 //   warps 0-7   two element-wise warpgroups. Thread t of either group owns
-//               TMEM lane t (key j0+t for S^T / dP^T / dV / dK); group g
-//               handles query columns [64g, 64g+64) of each tile and half of
-//               the dK / dV channels in the epilogue.
-//   warp 8      MMA issuer (one elected lane).
-//   warp 9      TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
+//               TMEM lane t (key j0+t); group g handles query columns
+//               [64g, 64g+64) of each tile and half of the dK / dV channels
+//               in the epilogue. P stays in registers between the P and dS
+//               passes.
+//   warps 8-11  dQ warpgroup: thread (warp%4)*32 + lane owns query row i0 +
+//               that lane; it copies the whole dQ row out of TMEM, releases
+//               the columns, then adds the row into the fp32 accumulator with
+//               red.global.add while the next tiles are computed.
+//   warp 12     MMA issuer (one elected lane).
+//   warp 13     TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
 //               the tile's LSE / D rows per query tile, two stages.
-//   warps 10-13 dQ warpgroup: thread (warp%4)*32 + lane owns query row i0 +
-//               that lane of the dQ tile; it copies the row out of TMEM,
-//               releases the columns, then adds it into the fp32 accumulator
-//               with red.global.add, so the atomics stay off the path of the
-//               element-wise warps and the MMAs.
-// TMEM (512 columns): S^T [0,128), whose columns then receive P^T and dS^T
-// as bf16 (query q's P at column 64*(q/64) + (q%64)/2, its dS 32 columns
-// further), dP^T [128,256), dV [256,256+d), dK [256+d,256+2d); dQ over dP^T
-// at d = 128, in its own columns otherwise. Shared-memory traffic is the
-// scarce resource (four of the five MMAs read 128 B/clk at this tile shape),
-// so P and dS feed their MMAs from TMEM wherever the operand shape allows.
+//   warps 14-15 idle (they complete the fourth warpgroup, which setmaxnreg
+//               needs to move registers to the dQ and element-wise warps).
+// TMEM (512 columns): region A [0,128) holds S^T, then P^T as bf16 (query q
+// at column 64*(q/64) + (q%64)/2); region B [128,256) holds dP^T, then dS^T as
+// bf16 in the same packing; dV [256,256+d), dK [256+d,256+2d). dQ takes
+// region B at d = 128 (after dK has read dS^T) and two buffers of its own at
+// smaller d. Because P^T and dS^T live in different regions, S^T of the next
+// tile only waits for dV and runs while the element-wise warps compute dS.
 // Every hand-off is an mbarrier; every wait is bounded and reports a timeout.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -52,11 +56,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kComputeThreads = 256;  // warps 0-7
-constexpr int kMmaWarp = 8;
-constexpr int kTmaWarp = 9;
-constexpr int kDqWarp0 = 10;          // warps 10-13
+constexpr int kDqWarp0 = 8;           // warps 8-11
 constexpr int kDqThreads = 128;
-constexpr int kThreads = 448;
+constexpr int kMmaWarp = 12;
+constexpr int kTmaWarp = 13;
+constexpr int kThreads = 512;
+// Registers per thread after the split. Each SM sub-partition runs one warp
+// of every warpgroup and holds 16K registers = 512 per lane, so the four
+// budgets must add up to at most 512 (the launch gives 128 to each).
+constexpr uint32_t kRegsCompute = 136, kRegsDq = 144, kRegsCtl = 96;
+static_assert(2 * kRegsCompute + kRegsDq + kRegsCtl <= 512, "register split exceeds the SM");
+// Pause after each 16-byte dQ reduction of a dQ thread (see the dQ warps).
+constexpr unsigned kRedPaceNs = 40;
 
 template <int D>
 struct BwdLayout {
@@ -85,17 +96,19 @@ struct BwdLayout {
       EXACT ? BYTES : ((BYTES + 1024) > 118 * 1024 ? BYTES + 1024 : 118 * 1024);
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr uint32_t T_DQ = D == 128 ? 128 : 256 + 2 * D;
   static constexpr bool DQ_OVER_DP = D == 128;
+  static constexpr int DQ_BUFS = DQ_OVER_DP ? 1 : 2;
+  static constexpr uint32_t T_DQ = DQ_OVER_DP ? T_DP : 256 + 2 * D;  // buffer b at T_DQ + b*D
   static constexpr uint32_t T_COLS = 512;
   static constexpr int HALF_D = D / 2;  // dK / dV channels per element-wise group
-  static constexpr int DQ_PASSES = D > 64 ? 2 : 1;  // TMEM read passes of the dQ warps
+  static_assert(DQ_OVER_DP || T_DQ + DQ_BUFS * D <= T_COLS, "TMEM columns exceeded");
 };
 
 enum Bar {
-  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DKDONE,
-  B_DQFULL, B_DQREAD, B_DONE, B_FINAL, B_COUNT
+  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DVDONE,
+  B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2, B_DONE = B_DQREAD + 2, B_FINAL, B_COUNT
 };
+static_assert(B_COUNT <= 32, "barrier slots");
 
 struct BwdParams {
   const float* lse2;  // [BH][Np], LSE * log2(e), +inf past N
@@ -105,6 +118,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int* status;
   int N, Np, T, BH;
+  int G;              // heads per scheduling group (see the CTA order in the kernel)
   int causal;
   float scale, scale_log2;
   uint64_t wait_cycles;
@@ -146,7 +160,7 @@ __host__ __device__ constexpr uint32_t p_col(int q) { return 64 * (q >> 6) + ((q
 __host__ __device__ constexpr uint32_t ds_col(int q) { return p_col(q) + 32; }
 
 template <int D>
-__global__ void __maxnreg__(128)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
@@ -166,8 +180,17 @@ __global__ void __maxnreg__(128)
   const float* s_dv = reinterpret_cast<const float*>(smem + L::DV_OFF);
 
   const int warp = threadIdx.x >> 5;
-  const int jt = blockIdx.x / p.BH;  // longest-first: key tile 0 has the most query tiles
-  const int bh = blockIdx.x % p.BH;
+  // CTA order: heads in groups of G, the groups one after another; inside a
+  // group, key tiles longest-first (key tile 0 has the most query tiles),
+  // heads interleaved. The CTAs in flight then touch only a few heads' Q, dO
+  // and dQ accumulator, which stay in L2 while every key tile of those heads
+  // passes over them; the last group may be smaller.
+  const int per_group = p.T * p.G;
+  const int g0 = (blockIdx.x / per_group) * p.G;
+  const int r = blockIdx.x % per_group;
+  const int gs = min(p.G, p.BH - g0);
+  const int jt = r / gs;
+  const int bh = g0 + r % gs;
   const int j0 = jt * kTile;
   const int i_begin = p.causal ? jt : 0;
   const int n_iter = p.T - i_begin;
@@ -184,14 +207,15 @@ __global__ void __maxnreg__(128)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_QFULL + s], 1);
       mbar_init(&bars[B_QEMPTY + s], 1);
+      mbar_init(&bars[B_DQFULL + s], 1);
+      mbar_init(&bars[B_DQREAD + s], kDqThreads);
     }
     mbar_init(&bars[B_SFULL], 1);
     mbar_init(&bars[B_DPFULL], 1);
     mbar_init(&bars[B_PFULL], kComputeThreads);
     mbar_init(&bars[B_DSFULL], kComputeThreads);
+    mbar_init(&bars[B_DVDONE], 1);
     mbar_init(&bars[B_DKDONE], 1);
-    mbar_init(&bars[B_DQFULL], 1);
-    mbar_init(&bars[B_DQREAD], kDqThreads);
     mbar_init(&bars[B_DONE], 1);
     mbar_init(&bars[B_FINAL], 1);
     *abort_flag = 0;
@@ -212,6 +236,11 @@ __global__ void __maxnreg__(128)
     atomicExch(p.status, kStatusTimeout);
   };
 
+  // Registers move from the control warpgroup (warps 12-15) to the others;
+  // each budget is set at the head of its role's branch so that the compiler
+  // allocates that branch's code against it.
+  if (warp >= kMmaWarp) {
+    regs_dec<kRegsCtl>();
   if (warp == kTmaWarp) {
     // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
@@ -255,6 +284,9 @@ __global__ void __maxnreg__(128)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
+    // Issue order per query tile i: dV(i), S(i+1), dK(i), dQ(i), dP(i+1); S(0)
+    // and dP(0) before the loop. Each wait guards one TMEM or shared-memory
+    // region against the MMA that overwrites it.
     if (elect_one_sync()) {
       const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sdS = sbase + L::DS_OFF;
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
@@ -263,49 +295,80 @@ __global__ void __maxnreg__(128)
       auto wait = [&](int b, uint32_t parity) {
         return mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag);
       };
-      bool ok = wait(B_KV, 0);
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int s = it & 1;
-        const uint32_t sQ = sbase + L::Q_OFF + s * L::TILE;
-        const uint32_t sdO = sbase + L::DO_OFF + s * L::TILE;
-        if (!(ok = wait(B_QFULL + s, (it >> 1) & 1))) break;
-        // S^T overwrites the P^T / dS^T columns that dV(it-1) and dK(it-1)
-        // read; dK(it-1) was issued after dV(it-1).
-        if (it > 0 && !(ok = wait(B_DKDONE, (it - 1) & 1))) break;
-        tc_fence_after();
+      auto stage_q = [&](int it) { return sbase + L::Q_OFF + (it & 1) * L::TILE; };
+      auto stage_do = [&](int it) { return sbase + L::DO_OFF + (it & 1) * L::TILE; };
+      // S^T(it) = K_j Q_i^T -> region A
+      auto issue_s = [&](int it) {
+        const uint32_t sQ = stage_q(it);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_S, desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
         if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
-        // At d = 128 dP^T overwrites dQ(it-1), which must have been read out.
-        if (L::DQ_OVER_DP && it > 0 && !(ok = wait(B_DQREAD, (it - 1) & 1))) break;
-        tc_fence_after();
+      };
+      // dP^T(it) = V_j dO_i^T -> region B
+      auto issue_dp = [&](int it) {
+        const uint32_t sdO = stage_do(it);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
         mma_commit(&bars[B_DPFULL]);
-        // dV_j += P^T dO_i, P^T read from TMEM (K = 128 queries, 16 per step)
+      };
+      bool ok = wait(B_KV, 0) && wait(B_QFULL, 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int s = it & 1;
+        const bool more = it + 1 < n_iter;
+        // dV_j += P^T dO_i, P^T read from region A (K = 128 queries, 16 per step)
         if (!(ok = wait(B_PFULL, it & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(sdO, kk), ID_KV,
-                 (it > 0 || kk > 0));
-        // dK_j += dS^T Q_i (dS^T from TMEM) ; dQ_i = dS K_j (dS from shared memory)
+          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(stage_do(it), kk),
+                 ID_KV, (it > 0 || kk > 0));
+        mma_commit(&bars[B_DVDONE]);
+        if (more) {
+          // S^T(it+1) overwrites P^T(it), which dV(it) reads.
+          if (!(ok = wait(B_QFULL + (s ^ 1), ((it + 1) >> 1) & 1))) break;
+          if (!(ok = wait(B_DVDONE, it & 1))) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
+        // dK_j += dS^T Q_i, dS^T read from region B
         if (!(ok = wait(B_DSFULL, it & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DK, tmem + L::T_S + ds_col(16 * kk), desc_mnmajor<D>(sQ, kk), ID_KV,
-                 (it > 0 || kk > 0));
+          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col(16 * kk), desc_mnmajor<D>(stage_q(it), kk),
+                 ID_KV, (it > 0 || kk > 0));
         mma_commit(&bars[B_DKDONE]);
-        if (!L::DQ_OVER_DP && it > 0 && !(ok = wait(B_DQREAD, (it - 1) & 1))) break;
+        // dQ_i = dS K_j (dS from shared memory)
+        const int b = it % L::DQ_BUFS;
+        if (L::DQ_OVER_DP) {
+          if (!(ok = wait(B_DKDONE, it & 1))) break;  // dQ(it) overwrites dS^T(it)
+        } else if (it >= L::DQ_BUFS) {
+          if (!(ok = wait(B_DQREAD + b, (it / L::DQ_BUFS - 1) & 1))) break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DQ, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
-        mma_commit(&bars[B_DQFULL]);
+          mma_ss(tmem + L::T_DQ + b * D, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q,
+                 kk > 0);
+        mma_commit(&bars[B_DQFULL + b]);
         mma_commit(&bars[B_QEMPTY + s]);
+        if (more) {
+          // dP^T(it+1) overwrites region B: dQ(it) at d = 128, dS^T(it) otherwise.
+          if (L::DQ_OVER_DP) {
+            if (!(ok = wait(B_DQREAD, it & 1))) break;
+          } else {
+            if (!(ok = wait(B_DKDONE, it & 1))) break;
+          }
+          tc_fence_after();
+          issue_dp(it + 1);
+        }
       }
       if (ok) {
         mma_commit(&bars[B_DONE]);
@@ -317,8 +380,10 @@ __global__ void __maxnreg__(128)
       mbar_wait(&bars[B_FINAL], 0, p.wait_cycles, never);
     }
     __syncwarp();
+  }
   } else if (warp >= kDqWarp0) {
-    // ------------------------------------------------ dQ warpgroup (warps 10-13)
+    regs_inc<kRegsDq>();
+    // ------------------------------------------------ dQ warpgroup (warps 8-11)
     const int t = ((warp & 3) << 5) | (threadIdx.x & 31);  // TMEM lane = query row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     auto wait_w = [&](int b, uint32_t parity) {
@@ -327,40 +392,40 @@ __global__ void __maxnreg__(128)
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_begin + it;
-      if (!(ok = wait_w(B_DQFULL, it & 1))) break;
+      const int b = it % L::DQ_BUFS;
+      if (!(ok = wait_w(B_DQFULL + b, (it / L::DQ_BUFS) & 1))) break;
       tc_fence_after();
-      const bool row_ok = i * kTile + t < p.N;
-      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
-      // At most 64 channels per pass: 128 registers a thread is the ceiling
-      // for 14 warps (four of them share one SM sub-partition's 16K registers).
+      // The whole row first, so the columns are released before the atomics.
+      uint32_t r[D];
 #pragma unroll
-      for (int h = 0; h < L::DQ_PASSES; ++h) {
-        constexpr int W = D / L::DQ_PASSES;
-        uint32_t r[W];
+      for (int c = 0; c < D; c += 32)
+        tmem_ld32(lane_base + L::T_DQ + b * D + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[B_DQREAD + b]);
+      if (i * kTile + t < p.N) {
+        float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
+        // Metered: a burst of reductions fills the sub-partition's memory
+        // instruction queue, and the element-wise warps' TMEM and shared-memory
+        // accesses then wait behind it. Spaced out, the reductions of one tile
+        // drain during the next tile's work.
 #pragma unroll
-        for (int c = 0; c < W; c += 16)
-          tmem_ld16(lane_base + L::T_DQ + h * W + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
-        tmem_ld_wait();
-        if (h == L::DQ_PASSES - 1) {
-          tc_fence_before();
-          mbar_arrive(&bars[B_DQREAD]);  // the dQ columns are free again
-        }
-        if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < W / 4; ++v)
-            red_add_v4(acc + (h * W / 4 + v) * 512, __uint_as_float(r[4 * v]),
-                       __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
-                       __uint_as_float(r[4 * v + 3]));
+        for (int v = 0; v < D / 4; ++v) {
+          red_add_v4(acc + v * 512, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          __nanosleep(kRedPaceNs);
         }
       }
     }
     if (!ok) fail();
   } else {
+    regs_inc<kRegsCompute>();
     // ------------------------------------------------ element-wise warps 0-7
-    const int t = threadIdx.x & 127;  // TMEM lane: key row (S^T, dV, dK) / query row (dQ)
+    const int t = threadIdx.x & 127;  // TMEM lane: key row
     const int g = threadIdx.x >> 7;   // query columns [64g, 64g+64), channels [g*D/2, ...)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int key = j0 + t;
+    const int qb = 64 * g;
     // Outcome of a wait, made uniform across the warp: the TMEM accesses that
     // follow are warp-collective, so a warp must never split on a timeout.
     auto wait_w = [&](int b, uint32_t parity) {
@@ -370,25 +435,23 @@ __global__ void __maxnreg__(128)
     for (int it = 0; it < n_iter; ++it) {
       const int s = it & 1;
       const int i = i_begin + it;
-      const int i0 = i * kTile;
       if (!(ok = wait_w(B_QFULL + s, (it >> 1) & 1))) break;  // LSE_i, D_i in shared memory
       const float* lse_s = s_lse + s * 128;
       const float* d_s = s_dv + s * 128;
       // queries with local index < thr are masked for this key row
       const int thr = key >= p.N ? 128 : ((p.causal && i == jt) ? t : 0);
 
-      // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e), written back as bf16
+      // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e) -> bf16 into region A
       if (!(ok = wait_w(B_SFULL, it & 1))) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const int qb = 64 * g + 32 * c;
-        uint32_t sr[32];
-        tmem_ld32(lane_base + L::T_S + qb, sr);
+      uint32_t pk[32];  // this thread's 64 P values as bf16 pairs, kept for the dS pass
+      {
+        uint32_t sr[64];
+        tmem_ld32(lane_base + L::T_S + qb, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(lane_base + L::T_S + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
         tmem_ld_wait();
-        uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
+        for (int u = 0; u < 64; u += 4) {
           const int q0 = qb + u;
           // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q0);
@@ -403,49 +466,49 @@ __global__ void __maxnreg__(128)
           pk[u / 2] = pack_bf16x2(p0, p1);
           pk[u / 2 + 1] = pack_bf16x2(p2, p3);
         }
-        // columns [p_col(qb), +16) lie inside this group's already-read S^T columns
-        tmem_st16(lane_base + L::T_S + p_col(qb), pk);
       }
+      // both S^T chunks were read above, so the packed P may overwrite them
+      tmem_st16(lane_base + L::T_S + p_col(qb), *reinterpret_cast<uint32_t(*)[16]>(pk));
+      tmem_st16(lane_base + L::T_S + p_col(qb + 32), *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[B_PFULL]);
 
-      // ---- dS^T = P^T o (dP^T - D) -> shared memory (bf16)
+      // ---- dS^T = P^T o (dP^T - D) -> bf16 into region B and shared memory
       if (!(ok = wait_w(B_DPFULL, it & 1))) break;
       tc_fence_after();
-      uint8_t* sdS = smem + L::DS_OFF;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const int qb = 64 * g + 32 * c;
-        uint32_t dr[32], pr[16];
-        tmem_ld32(lane_base + L::T_DP + qb, dr);
-        tmem_ld16(lane_base + L::T_S + p_col(qb), pr);
+      uint32_t dk[32];
+      {
+        uint32_t dr[64];
+        tmem_ld32(lane_base + L::T_DP + qb, *reinterpret_cast<uint32_t(*)[32]>(dr));
+        tmem_ld32(lane_base + L::T_DP + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(dr + 32));
         tmem_ld_wait();
-        uint32_t dk[16];
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
+        for (int u = 0; u < 64; u += 4) {
           const int q0 = qb + u;
           const float4 d4 = *reinterpret_cast<const float4*>(d_s + q0);
-          const float2 pa = unpack_bf16x2(pr[u / 2]);
-          const float2 pb = unpack_bf16x2(pr[u / 2 + 1]);
+          const float2 pa = unpack_bf16x2(pk[u / 2]);
+          const float2 pb = unpack_bf16x2(pk[u / 2 + 1]);
           dk[u / 2] = pack_bf16x2(pa.x * (__uint_as_float(dr[u]) - d4.x),
                                   pa.y * (__uint_as_float(dr[u + 1]) - d4.y));
           dk[u / 2 + 1] = pack_bf16x2(pb.x * (__uint_as_float(dr[u + 2]) - d4.z),
                                       pb.y * (__uint_as_float(dr[u + 3]) - d4.w));
         }
-        // dS^T for dK (TMEM A operand); these S^T columns were read in the P pass
-        tmem_st16(lane_base + L::T_S + ds_col(qb), dk);
-        // dS for dQ (shared memory, read transposed by the MMA)
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          st_shared_v4(smem_u32(sdS) + ds_offset(t, qb / 8 + v), dk[4 * v], dk[4 * v + 1],
-                       dk[4 * v + 2], dk[4 * v + 3]);
       }
+      // dS^T for dK (TMEM A operand); both dP^T chunks were read above
+      tmem_st16(lane_base + L::T_DP + p_col(qb), *reinterpret_cast<uint32_t(*)[16]>(dk));
+      tmem_st16(lane_base + L::T_DP + p_col(qb + 32), *reinterpret_cast<uint32_t(*)[16]>(dk + 16));
+      // dS for dQ (shared memory, read transposed by the MMA). dQ(it-1) has
+      // finished reading the previous tile: dP^T(it) was issued after it.
+      uint8_t* sdS = smem + L::DS_OFF;
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        st_shared_v4(smem_u32(sdS) + ds_offset(t, qb / 8 + v), dk[4 * v], dk[4 * v + 1],
+                     dk[4 * v + 2], dk[4 * v + 3]);
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_DSFULL]);
-
     }
     if (ok) ok = wait_w(B_DONE, 0);
     if (!ok) {
@@ -519,6 +582,14 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.Np = ws.Np;
   p.T = ws.Np / kTile;
   p.BH = BH;
+  // Heads per group: as many as fit, with their Q and dO tiles (bf16) and dQ
+  // accumulator (fp32), in about a third of L2.
+  int dev = 0, l2 = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
+    l2 = 126 << 20;
+  const size_t head_bytes = static_cast<size_t>(ws.Np) * D * 8;
+  p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
