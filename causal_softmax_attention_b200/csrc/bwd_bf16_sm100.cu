@@ -66,6 +66,8 @@ constexpr int kThreads = 512;
 // budgets must add up to at most 512 (the launch gives 128 to each).
 constexpr uint32_t kRegsCompute = 136, kRegsDq = 144, kRegsCtl = 96;
 static_assert(2 * kRegsCompute + kRegsDq + kRegsCtl <= 512, "register split exceeds the SM");
+// Pause after each 16-byte dQ reduction of a dQ thread (see the dQ warps).
+constexpr unsigned kRedPaceNs = 40;
 
 template <int D>
 struct BwdLayout {
@@ -75,22 +77,15 @@ struct BwdLayout {
   static constexpr int CHUNK = kTile * ROWB;    // bytes of one [128][CH] box
   static constexpr int TILE = NCH * CHUNK;      // bytes of one [128][D] bf16 tile
   static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128B : kSwizzle64B;
-  static constexpr int Q_STAGES = 2;            // Q_i (with LSE_i, D_i): read by S(i) and dK(i)
-  // dO_i is read by dP(i) and dV(i) only; dO_{i+1} is needed after dQ(i), so
-  // one buffer suffices where shared memory is short (d = 128).
-  static constexpr int DO_STAGES = D == 128 ? 1 : 2;
-  static constexpr int DQ_PASS_CH = D >= 64 ? 64 : D;    // dQ channels staged per bulk reduction
-  static constexpr int DQ_PASSES = D / DQ_PASS_CH;
-  static constexpr int STG_BYTES = DQ_PASS_CH * kTile * 4;
+  static constexpr int STAGES = 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
-  static constexpr int Q_OFF = V_OFF + TILE;                // [Q_STAGES] tiles
-  static constexpr int DO_OFF = Q_OFF + Q_STAGES * TILE;    // [DO_STAGES] tiles
-  static constexpr int DS_OFF = DO_OFF + DO_STAGES * TILE;  // [128 keys][128 queries] bf16
-  static constexpr int STG_OFF = DS_OFF + 32768;            // dQ staging, [DQ_PASS_CH/4][128][4] f32
-  static constexpr int LSE_OFF = STG_OFF + STG_BYTES;       // [Q_STAGES][128] f32
-  static constexpr int DV_OFF = LSE_OFF + Q_STAGES * 512;   // [Q_STAGES][128] f32
-  static constexpr int BAR_OFF = DV_OFF + Q_STAGES * 512;
+  static constexpr int Q_OFF = V_OFF + TILE;              // [STAGES] tiles
+  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;    // [STAGES] tiles
+  static constexpr int DS_OFF = DO_OFF + STAGES * TILE;   // [128 keys][128 queries] bf16
+  static constexpr int LSE_OFF = DS_OFF + 32768;          // [STAGES][128] f32
+  static constexpr int DV_OFF = LSE_OFF + STAGES * 512;   // [STAGES][128] f32
+  static constexpr int BAR_OFF = DV_OFF + STAGES * 512;
   static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
   static constexpr int BYTES = MISC_OFF + 64;
   // d = 128 fills the 227 KB window, so the window itself must be 1024-byte
@@ -110,9 +105,8 @@ struct BwdLayout {
 };
 
 enum Bar {
-  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL,
-  B_PFULL, B_DSFULL, B_DVDONE, B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2,
-  B_STGFREE = B_DQREAD + 2, B_STGREADY, B_DONE, B_FINAL, B_COUNT
+  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DVDONE,
+  B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2, B_DONE = B_DQREAD + 2, B_FINAL, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
@@ -213,13 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_QFULL + s], 1);
       mbar_init(&bars[B_QEMPTY + s], 1);
-      mbar_init(&bars[B_DOFULL + s], 1);
-      mbar_init(&bars[B_DOEMPTY + s], 1);
       mbar_init(&bars[B_DQFULL + s], 1);
       mbar_init(&bars[B_DQREAD + s], kDqThreads);
     }
-    mbar_init(&bars[B_STGFREE], 1);
-    mbar_init(&bars[B_STGREADY], kDqThreads);
     mbar_init(&bars[B_SFULL], 1);
     mbar_init(&bars[B_DPFULL], 1);
     mbar_init(&bars[B_PFULL], kComputeThreads);
@@ -264,46 +254,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(smem + L::V_OFF + c * L::CHUNK, &tm_v, &bars[B_KV], c * L::CH, j0, bh);
       }
       bool ok = true;
-      int q_issued = 0, do_issued = 0;
+      int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
-        const int i0 = (i_begin + it) * kTile;
-        // Q_i, LSE_i, D_i: stage it % 2, free once dK(i-2) has completed
-        const int s = it % L::Q_STAGES;
-        if (it >= L::Q_STAGES &&
-            !(ok = mbar_wait(&bars[B_QEMPTY + s], (it / L::Q_STAGES - 1) & 1, p.wait_cycles,
-                             abort_flag)))
+        const int s = it & 1;
+        if (it >= 2 &&
+            !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
           break;
+        const int i0 = (i_begin + it) * kTile;
         uint64_t* bar = &bars[B_QFULL + s];
-        mbar_arrive_expect_tx(bar, L::TILE + 2 * 512);
-        for (int c = 0; c < L::NCH; ++c)
+        mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
+        for (int c = 0; c < L::NCH; ++c) {
           tma_load_3d(smem + L::Q_OFF + s * L::TILE + c * L::CHUNK, &tm_q, bar, c * L::CH, i0,
                       bh);
+          tma_load_3d(smem + L::DO_OFF + s * L::TILE + c * L::CHUNK, &tm_do, bar, c * L::CH,
+                      i0, bh);
+        }
         bulk_load(smem + L::LSE_OFF + s * 512, p.lse2 + static_cast<size_t>(bh) * p.Np + i0, 512,
                   bar);
         bulk_load(smem + L::DV_OFF + s * 512, p.dvec + static_cast<size_t>(bh) * p.Np + i0, 512,
                   bar);
-        ++q_issued;
-        // dO_i: stage it % DO_STAGES, free once dV(i - DO_STAGES) has completed
-        const int t = it % L::DO_STAGES;
-        if (it >= L::DO_STAGES &&
-            !(ok = mbar_wait(&bars[B_DOEMPTY + t], (it / L::DO_STAGES - 1) & 1, p.wait_cycles,
-                             abort_flag)))
-          break;
-        bar = &bars[B_DOFULL + t];
-        mbar_arrive_expect_tx(bar, L::TILE);
-        for (int c = 0; c < L::NCH; ++c)
-          tma_load_3d(smem + L::DO_OFF + t * L::TILE + c * L::CHUNK, &tm_do, bar, c * L::CH, i0,
-                      bh);
-        ++do_issued;
+        ++issued;
       }
       if (!ok) fail();
       // Every load issued has landed before the CTA can exit (bounded).
       mbar_wait(&bars[B_KV], 0, p.wait_cycles, never);
-      for (int w = q_issued > L::Q_STAGES ? q_issued - L::Q_STAGES : 0; w < q_issued; ++w)
-        mbar_wait(&bars[B_QFULL + w % L::Q_STAGES], (w / L::Q_STAGES) & 1, p.wait_cycles, never);
-      for (int w = do_issued > L::DO_STAGES ? do_issued - L::DO_STAGES : 0; w < do_issued; ++w)
-        mbar_wait(&bars[B_DOFULL + w % L::DO_STAGES], (w / L::DO_STAGES) & 1, p.wait_cycles,
-                  never);
+      for (int w = issued > 2 ? issued - 2 : 0; w < issued; ++w)
+        mbar_wait(&bars[B_QFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -319,11 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait = [&](int b, uint32_t parity) {
         return mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag);
       };
-      auto stage_q = [&](int it) { return sbase + L::Q_OFF + (it % L::Q_STAGES) * L::TILE; };
-      auto stage_do = [&](int it) { return sbase + L::DO_OFF + (it % L::DO_STAGES) * L::TILE; };
-      auto wait_do = [&](int it) {
-        return wait(B_DOFULL + it % L::DO_STAGES, (it / L::DO_STAGES) & 1);
-      };
+      auto stage_q = [&](int it) { return sbase + L::Q_OFF + (it & 1) * L::TILE; };
+      auto stage_do = [&](int it) { return sbase + L::DO_OFF + (it & 1) * L::TILE; };
       // S^T(it) = K_j Q_i^T -> region A
       auto issue_s = [&](int it) {
         const uint32_t sQ = stage_q(it);
@@ -340,13 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
         mma_commit(&bars[B_DPFULL]);
       };
-      bool ok = wait(B_KV, 0) && wait(B_QFULL, 0) && wait_do(0);
+      bool ok = wait(B_KV, 0) && wait(B_QFULL, 0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
       for (int it = 0; ok && it < n_iter; ++it) {
+        const int s = it & 1;
         const bool more = it + 1 < n_iter;
         // dV_j += P^T dO_i, P^T read from region A (K = 128 queries, 16 per step)
         if (!(ok = wait(B_PFULL, it & 1))) break;
@@ -356,10 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(stage_do(it), kk),
                  ID_KV, (it > 0 || kk > 0));
         mma_commit(&bars[B_DVDONE]);
-        mma_commit(&bars[B_DOEMPTY + it % L::DO_STAGES]);  // dP(it) and dV(it) read dO_i
         if (more) {
           // S^T(it+1) overwrites P^T(it), which dV(it) reads.
-          if (!(ok = wait(B_QFULL + (it + 1) % L::Q_STAGES, ((it + 1) / L::Q_STAGES) & 1))) break;
+          if (!(ok = wait(B_QFULL + (s ^ 1), ((it + 1) >> 1) & 1))) break;
           if (!(ok = wait(B_DVDONE, it & 1))) break;
           tc_fence_after();
           issue_s(it + 1);
@@ -372,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col(16 * kk), desc_mnmajor<D>(stage_q(it), kk),
                  ID_KV, (it > 0 || kk > 0));
         mma_commit(&bars[B_DKDONE]);
-        mma_commit(&bars[B_QEMPTY + it % L::Q_STAGES]);  // S(it) and dK(it) read Q_i
         // dQ_i = dS K_j (dS from shared memory)
         const int b = it % L::DQ_BUFS;
         if (L::DQ_OVER_DP) {
@@ -386,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + L::T_DQ + b * D, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q,
                  kk > 0);
         mma_commit(&bars[B_DQFULL + b]);
+        mma_commit(&bars[B_QEMPTY + s]);
         if (more) {
           // dP^T(it+1) overwrites region B: dQ(it) at d = 128, dS^T(it) otherwise.
           if (L::DQ_OVER_DP) {
@@ -393,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             if (!(ok = wait(B_DKDONE, it & 1))) break;
           }
-          if (!(ok = wait_do(it + 1))) break;
           tc_fence_after();
           issue_dp(it + 1);
         }
@@ -412,27 +384,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kDqWarp0) {
     regs_inc<kRegsDq>();
     // ------------------------------------------------ dQ warpgroup (warps 8-11)
-    // Each tile's dQ rows go TMEM -> registers -> a shared-memory staging
-    // buffer laid out like the accumulator tile, and one thread hands the
-    // buffer to the TMA engine as a bulk f32 add-reduction into the fp32
-    // accumulator in global memory. The reductions then never occupy the
-    // warps' memory-instruction queues (a burst of per-thread red.add there
-    // stalls the element-wise warps' TMEM and shared-memory accesses).
     const int t = ((warp & 3) << 5) | (threadIdx.x & 31);  // TMEM lane = query row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const bool leader = threadIdx.x == kDqWarp0 * 32;
-    float* stg = reinterpret_cast<float*>(smem + L::STG_OFF);
     auto wait_w = [&](int b, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
     };
-    if (leader) mbar_arrive(&bars[B_STGFREE]);  // the staging buffer starts free
     bool ok = true;
-    for (int it = 0; ok && it < n_iter; ++it) {
+    for (int it = 0; it < n_iter; ++it) {
       const int i = i_begin + it;
       const int b = it % L::DQ_BUFS;
       if (!(ok = wait_w(B_DQFULL + b, (it / L::DQ_BUFS) & 1))) break;
       tc_fence_after();
-      // The whole row first, so the columns are released at once.
+      // The whole row first, so the columns are released before the atomics.
       uint32_t r[D];
 #pragma unroll
       for (int c = 0; c < D; c += 32)
@@ -440,31 +403,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars[B_DQREAD + b]);
-      // Accumulator tile (bh, i): [D/4][128 rows][4] floats, pass h = channels
-      // [h*W, (h+1)*W), contiguous. Rows past N are zero (P = 0 there).
-      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512;
+      if (i * kTile + t < p.N) {
+        float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
+        // Metered: a burst of reductions fills the sub-partition's memory
+        // instruction queue, and the element-wise warps' TMEM and shared-memory
+        // accesses then wait behind it. Spaced out, the reductions of one tile
+        // drain during the next tile's work.
 #pragma unroll
-      for (int h = 0; h < L::DQ_PASSES; ++h) {
-        constexpr int W = L::DQ_PASS_CH;
-        const int k = it * L::DQ_PASSES + h;  // staging use number
-        if (!(ok = wait_w(B_STGFREE, k & 1))) break;
-        const uint32_t dst = smem_u32(stg) + t * 16;
-#pragma unroll
-        for (int v = 0; v < W / 4; ++v)
-          st_shared_v4(dst + v * 2048, r[h * W + 4 * v], r[h * W + 4 * v + 1],
-                       r[h * W + 4 * v + 2], r[h * W + 4 * v + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(&bars[B_STGREADY]);
-        if (leader) {
-          if (!(ok = mbar_wait(&bars[B_STGREADY], k & 1, p.wait_cycles, abort_flag))) break;
-          bulk_reduce_add_f32(acc + h * (W / 4) * 512, stg, L::STG_BYTES);
-          bulk_commit();
-          bulk_wait_read_all();
-          mbar_arrive(&bars[B_STGFREE]);
+        for (int v = 0; v < D / 4; ++v) {
+          red_add_v4(acc + v * 512, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          __nanosleep(kRedPaceNs);
         }
       }
     }
-    if (leader) bulk_wait_all();  // the reductions are done before the CTA exits
     if (!ok) fail();
   } else {
     regs_inc<kRegsCompute>();

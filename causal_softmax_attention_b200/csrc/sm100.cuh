@@ -106,29 +106,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Bulk reduction shared -> global: dst[k] += src[k] (f32) over `bytes`
-// (16-byte aligned addresses, a multiple of 16 bytes), performed by the TMA
-// engine at L2. Tracked by bulk groups of the issuing thread.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc,
-                                                    uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   gdst),
-               "r"(smem_u32(ssrc)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Waits until every committed bulk group of this thread has finished reading
-// its shared-memory source (the source may then be overwritten).
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Waits until every committed bulk group of this thread has completed.
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // ---------------------------------------------------------------- tcgen05
 // Allocation: executed by one whole warp; the TMEM base address is written to
 // shared memory at `dst`.
