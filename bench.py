@@ -349,6 +349,19 @@ def run_gpu(args, cfg, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e_value = whole_job_tflops(flops, world, e2e_ms)
 
+    # ---- the forward that produces O and LSE (not part of the timed step):
+    # its own CUDA-event time on the same stream, same inputs, outputs reused.
+    fwd_iters = 5
+    for _ in range(2):
+        csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(fwd_iters):
+        csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = max_over_ranks(f0.elapsed_time(f1) / fwd_iters, world)
+
     if rank != 0:
         return
     peaks, peak_kind = load_peaks()
@@ -374,6 +387,11 @@ def run_gpu(args, cfg, world, rank, local):
                      "pre_and_convert_median": statistics.median(step_ms) - statistics.median(main_ms)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "forward": {"kernel": "attn_fwd_bf16_sm100_kernel", "ms": fwd_ms,
+                    "tflops": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12,
+                    "frac": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12 / peak,
+                    "flops_convention": "causal forward 4*B*H*N^2*d/2",
+                    "note": "measured outside the timed backward step"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "device_status": csa.status_string(status),
