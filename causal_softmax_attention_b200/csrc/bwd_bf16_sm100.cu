@@ -61,11 +61,18 @@ constexpr int kDqThreads = 128;
 constexpr int kMmaWarp = 12;
 constexpr int kTmaWarp = 13;
 constexpr int kThreads = 512;
+constexpr uint32_t kLaunchRegs = 65536 / kThreads;  // registers a thread holds at launch
 // Registers per thread after the split. Each SM sub-partition runs one warp
 // of every warpgroup and holds 16K registers = 512 per lane, so the four
 // budgets must add up to at most 512 (the launch gives 128 to each).
-constexpr uint32_t kRegsCompute = 136, kRegsDq = 144, kRegsCtl = 96;
-static_assert(2 * kRegsCompute + kRegsDq + kRegsCtl <= 512, "register split exceeds the SM");
+// The dQ warps hold a whole row of up to 128 values.
+template <int D>
+struct RegSplit {
+  static constexpr uint32_t kCompute = 136;
+  static constexpr uint32_t kDq = 144;
+  static constexpr uint32_t kCtl = 96;
+  static_assert(2 * kCompute + kDq + kCtl <= 512, "register split exceeds the SM");
+};
 // Pause after each 16-byte dQ reduction of a dQ thread (see the dQ warps).
 constexpr unsigned kRedPaceNs = 40;
 
@@ -159,6 +166,31 @@ __device__ __forceinline__ uint32_t ds_offset(int r, int g) {
 __host__ __device__ constexpr uint32_t p_col(int q) { return 64 * (q >> 6) + ((q & 63) >> 1); }
 __host__ __device__ constexpr uint32_t ds_col(int q) { return p_col(q) + 32; }
 
+// P for this thread's key row over 64 queries: p_u = 2^(S_u * scale*log2e -
+// LSE_u*log2e), packed as bf16 pairs. Queries u < thr are masked (kMasked);
+// off the diagonal tile nothing is, and the compare-and-select is skipped.
+template <bool kMasked>
+__device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[64], const float* lse,
+                                              float scale_log2, int thr, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int u = 0; u < 64; u += 4) {
+    // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
+    const float4 l4 = *reinterpret_cast<const float4*>(lse + u);
+    float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), scale_log2, -l4.x));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), scale_log2, -l4.y));
+    float p2 = ex2_approx(fmaf(__uint_as_float(sr[u + 2]), scale_log2, -l4.z));
+    float p3 = ex2_approx(fmaf(__uint_as_float(sr[u + 3]), scale_log2, -l4.w));
+    if (kMasked) {
+      if (u < thr) p0 = 0.f;
+      if (u + 1 < thr) p1 = 0.f;
+      if (u + 2 < thr) p2 = 0.f;
+      if (u + 3 < thr) p3 = 0.f;
+    }
+    pk[u / 2] = pack_bf16x2(p0, p1);
+    pk[u / 2 + 1] = pack_bf16x2(p2, p3);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -240,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // each budget is set at the head of its role's branch so that the compiler
   // allocates that branch's code against it.
   if (warp >= kMmaWarp) {
-    regs_dec<kRegsCtl>();
+    regs_to<RegSplit<D>::kCtl, kLaunchRegs>();
   if (warp == kTmaWarp) {
     // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
@@ -382,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   } else if (warp >= kDqWarp0) {
-    regs_inc<kRegsDq>();
+    regs_to<RegSplit<D>::kDq, kLaunchRegs>();
     // ------------------------------------------------ dQ warpgroup (warps 8-11)
     const int t = ((warp & 3) << 5) | (threadIdx.x & 31);  // TMEM lane = query row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -400,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32)
         tmem_ld32(lane_base + L::T_DQ + b * D + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
-      tmem_ld_wait();
+      tmem_ld_wait(r);
       tc_fence_before();
       mbar_arrive(&bars[B_DQREAD + b]);
       if (i * kTile + t < p.N) {
@@ -419,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) fail();
   } else {
-    regs_inc<kRegsCompute>();
+    regs_to<RegSplit<D>::kCompute, kLaunchRegs>();
     // ------------------------------------------------ element-wise warps 0-7
     const int t = threadIdx.x & 127;  // TMEM lane: key row
     const int g = threadIdx.x >> 7;   // query columns [64g, 64g+64), channels [g*D/2, ...)
@@ -449,23 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sr[64];
         tmem_ld32(lane_base + L::T_S + qb, *reinterpret_cast<uint32_t(*)[32]>(sr));
         tmem_ld32(lane_base + L::T_S + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-        tmem_ld_wait();
-#pragma unroll
-        for (int u = 0; u < 64; u += 4) {
-          const int q0 = qb + u;
-          // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q0);
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -l4.x));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -l4.y));
-          float p2 = ex2_approx(fmaf(__uint_as_float(sr[u + 2]), p.scale_log2, -l4.z));
-          float p3 = ex2_approx(fmaf(__uint_as_float(sr[u + 3]), p.scale_log2, -l4.w));
-          if (q0 < thr) p0 = 0.f;
-          if (q0 + 1 < thr) p1 = 0.f;
-          if (q0 + 2 < thr) p2 = 0.f;
-          if (q0 + 3 < thr) p3 = 0.f;
-          pk[u / 2] = pack_bf16x2(p0, p1);
-          pk[u / 2 + 1] = pack_bf16x2(p2, p3);
-        }
+        tmem_ld_wait(sr);
+        // Only the diagonal tile and the key tile past N mask anything.
+        if (__any_sync(0xffffffffu, thr > qb))
+          p_from_scores<true>(sr, lse_s + qb, p.scale_log2, thr - qb, pk);
+        else
+          p_from_scores<false>(sr, lse_s + qb, p.scale_log2, 0, pk);
       }
       // both S^T chunks were read above, so the packed P may overwrite them
       tmem_st16(lane_base + L::T_S + p_col(qb), *reinterpret_cast<uint32_t(*)[16]>(pk));
@@ -482,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t dr[64];
         tmem_ld32(lane_base + L::T_DP + qb, *reinterpret_cast<uint32_t(*)[32]>(dr));
         tmem_ld32(lane_base + L::T_DP + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(dr + 32));
-        tmem_ld_wait();
+        tmem_ld_wait(dr);
 #pragma unroll
         for (int u = 0; u < 64; u += 4) {
           const int q0 = qb + u;
@@ -532,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(lane_base + L::T_DV + ch, rv);
           tmem_ld16(lane_base + L::T_DK + ch, rk);
         }
-        tmem_ld_wait();
+        tmem_ld_wait(rv, rk);
 #pragma unroll
         for (int v = 0; v < W / 8 && key_ok; ++v) {
           uint4 ov, ok4;
@@ -571,6 +592,16 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   auto kern = attn_bwd_bf16_sm100_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
+  // The setmaxnreg split redistributes exactly the registers the block is
+  // launched with; with fewer at launch the increases could never be served.
+  static const cudaError_t regs_ok = [&]() {
+    cudaFuncAttributes fa;
+    const cudaError_t r = cudaFuncGetAttributes(&fa, kern);
+    if (r != cudaSuccess) return r;
+    return fa.numRegs == static_cast<int>(kLaunchRegs) ? cudaSuccess
+                                                       : cudaErrorInvalidConfiguration;
+  }();
+  if (regs_ok != cudaSuccess) return regs_ok;
   BwdParams p;
   p.lse2 = ws.lse_pad;
   p.dvec = ws.d_pad;

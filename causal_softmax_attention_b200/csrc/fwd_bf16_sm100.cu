@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(160, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(lane_base + L::T_S + 32 * c, r);
-        tmem_ld_wait();
+        tmem_ld_wait(r);
 #pragma unroll
         for (int u = 0; u < 32; ++u)
           if (32 * c + u < lim) mx = fmaxf(mx, __uint_as_float(r[u]));
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(160, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(lane_base + L::T_S + 32 * c, r);
-        tmem_ld_wait();
+        tmem_ld_wait(r);
         uint32_t pk[16];
 #pragma unroll
         for (int u = 0; u < 32; u += 2) {
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(160, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(lane_base + L::T_O + 32 * c, r);
-        tmem_ld_wait();
+        tmem_ld_wait(r);
 #pragma unroll
         for (int u = 0; u < 32; ++u) o[32 * c + u] = fmaf(o[32 * c + u], alpha, __uint_as_float(r[u]));
       }

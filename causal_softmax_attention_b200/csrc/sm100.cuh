@@ -196,6 +196,34 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.ld writes its destination registers asynchronously, but the
+// compiler sees them as written by the load itself and may schedule their
+// first use before tcgen05.wait::ld. Passing every loaded register through an
+// empty volatile asm after the wait (volatile asm statements keep their
+// order) makes each use depend on the wait.
+template <int N>
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "registers are fenced in groups of eight");
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                 "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
+// Waits for this thread's outstanding TMEM loads; the arrays they filled may
+// be used afterwards.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&a)[N]) {
+  tmem_ld_wait();
+  regs_after_wait(a);
+}
+template <int N, int M>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&a)[N], uint32_t (&b)[M]) {
+  tmem_ld_wait();
+  regs_after_wait(a);
+  regs_after_wait(b);
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   __syncwarp();
   asm volatile(
@@ -227,7 +255,9 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 // Per-thread register budget of the executing warpgroup (all four warps of
 // the warpgroup execute the same instruction). `dec` returns registers to the
-// CTA's pool; `inc` blocks until the pool can supply the new budget.
+// CTA's pool; `inc` blocks until the pool can supply the new budget. `inc`
+// may only raise and `dec` only lower the count the warps hold, so
+// regs_to<N, kLaunch>() picks the direction from the launch budget kLaunch.
 template <uint32_t N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
@@ -235,6 +265,15 @@ __device__ __forceinline__ void regs_dec() {
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N, uint32_t kLaunch>
+__device__ __forceinline__ void regs_to() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg takes 24..256 in steps of 8");
+  if constexpr (N > kLaunch) {
+    regs_inc<N>();
+  } else if constexpr (N < kLaunch) {
+    regs_dec<N>();
+  }
 }
 
 // ---------------------------------------------------------------- descriptors

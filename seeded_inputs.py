@@ -61,6 +61,9 @@ CONFIGS = {
     # a quarter of c4 (8 heads): still larger than L2, small enough for a
     # many-pass profiler capture
     "prof_d128": AttnConfig("prof_d128", 1, 8, 16384, 128, "bf16", 5),
+    # the d = 64 counterpart (the long-sequence workload's head size), with
+    # its q, k scaling; 8 heads of 32,768 tokens
+    "prof_d64": AttnConfig("prof_d64", 1, 8, 32768, 64, "bf16", 6, qk_gain=0.5),
 }
 
 
