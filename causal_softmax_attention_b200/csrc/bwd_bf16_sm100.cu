@@ -55,23 +55,36 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kComputeThreads = 256;  // warps 0-7
-constexpr int kDqWarp0 = 8;           // warps 8-11
-constexpr int kDqThreads = 128;
-constexpr int kMmaWarp = 12;
-constexpr int kTmaWarp = 13;
-constexpr int kThreads = 512;
-constexpr uint32_t kLaunchRegs = 65536 / kThreads;  // registers a thread holds at launch
-// Registers per thread after the split. Each SM sub-partition runs one warp
-// of every warpgroup and holds 16K registers = 512 per lane, so the four
-// budgets must add up to at most 512 (the launch gives 128 to each).
-// The dQ warps hold a whole row of up to 128 values.
+// Warp roles: two element-wise warpgroups (thread t of group g owns TMEM lane
+// t, key row j0 + t, and query columns [QC*g, QC*(g+1))), one dQ warpgroup
+// (thread = query row of the dQ tile; a whole row of up to 128 channels), and
+// a control warpgroup whose warp MMA_WARP issues the MMAs and warp TMA_WARP
+// the TMA loads (its other two warps idle). Four element-wise warpgroups at
+// d <= 64, with dQ read out by them, measured slower (736 vs 791 TFLOP/s on
+// 8 heads of 32K tokens): that pass is bound by its MUFU and issue slots, not
+// by latency.
 template <int D>
-struct RegSplit {
-  static constexpr uint32_t kCompute = 136;
-  static constexpr uint32_t kDq = 144;
-  static constexpr uint32_t kCtl = 96;
-  static_assert(2 * kCompute + kDq + kCtl <= 512, "register split exceeds the SM");
+struct Roles {
+  static constexpr int EG = 2;                      // element-wise warpgroups
+  static constexpr int QC = 128 / EG;               // query columns per element-wise group
+  static constexpr int E_THREADS = 128 * EG;
+  static constexpr int DQ_WARP0 = 4 * EG;
+  static constexpr int MMA_WARP = DQ_WARP0 + 4;
+  static constexpr int TMA_WARP = MMA_WARP + 1;
+  static constexpr int THREADS = (MMA_WARP + 4) * 32;
+  static constexpr int WGS = THREADS / 128;
+  // registers a thread holds at launch (the per-block 64K, in steps of 8)
+  static constexpr uint32_t LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
+  // Budgets after setmaxnreg. One warp of every warpgroup shares an SM
+  // sub-partition (16K registers = 512 per lane), and the budgets draw on
+  // the registers the block was launched with.
+  static constexpr uint32_t R_E = 136;
+  static constexpr uint32_t R_DQ = 144;
+  static constexpr uint32_t R_CTL = 96;
+  static_assert(EG * R_E + R_DQ + R_CTL <= WGS * LAUNCH_REGS,
+                "register split exceeds the launch budget");
+  static constexpr int DQ_READERS = 128;            // arrivals on B_DQREAD
+  static constexpr int E_CH = D / EG;               // dK / dV channels per group (epilogue)
 };
 // Pause after each 16-byte dQ reduction of a dQ thread (see the dQ warps).
 constexpr unsigned kRedPaceNs = 40;
@@ -107,7 +120,6 @@ struct BwdLayout {
   static constexpr int DQ_BUFS = DQ_OVER_DP ? 1 : 2;
   static constexpr uint32_t T_DQ = DQ_OVER_DP ? T_DP : 256 + 2 * D;  // buffer b at T_DQ + b*D
   static constexpr uint32_t T_COLS = 512;
-  static constexpr int HALF_D = D / 2;  // dK / dV channels per element-wise group
   static_assert(DQ_OVER_DP || T_DQ + DQ_BUFS * D <= T_COLS, "TMEM columns exceeded");
 };
 
@@ -162,18 +174,20 @@ __device__ __forceinline__ uint32_t ds_offset(int r, int g) {
   return (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4);
 }
 
-// TMEM columns of the bf16 pairs holding query q (q even) of P^T and dS^T.
-__host__ __device__ constexpr uint32_t p_col(int q) { return 64 * (q >> 6) + ((q & 63) >> 1); }
-__host__ __device__ constexpr uint32_t ds_col(int q) { return p_col(q) + 32; }
+// TMEM column of the bf16 pair holding query q (q even) of P^T or dS^T
+// within its region: each element-wise group packs its QC queries into the
+// first QC/2 of its own QC columns.
+template <int QC>
+__host__ __device__ constexpr uint32_t p_col(int q) { return QC * (q / QC) + (q % QC) / 2; }
 
-// P for this thread's key row over 64 queries: p_u = 2^(S_u * scale*log2e -
+// P for this thread's key row over QC queries: p_u = 2^(S_u * scale*log2e -
 // LSE_u*log2e), packed as bf16 pairs. Queries u < thr are masked (kMasked);
 // off the diagonal tile nothing is, and the compare-and-select is skipped.
-template <bool kMasked>
-__device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[64], const float* lse,
-                                              float scale_log2, int thr, uint32_t (&pk)[32]) {
+template <bool kMasked, int QC>
+__device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[QC], const float* lse,
+                                              float scale_log2, int thr, uint32_t (&pk)[QC / 2]) {
 #pragma unroll
-  for (int u = 0; u < 64; u += 4) {
+  for (int u = 0; u < QC; u += 4) {
     // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
     const float4 l4 = *reinterpret_cast<const float4*>(lse + u);
     float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), scale_log2, -l4.x));
@@ -192,12 +206,14 @@ __device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[64], const fl
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
                                const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   using L = BwdLayout<D>;
+  using R = Roles<D>;
+  constexpr int QC = R::QC;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = L::EXACT ? smem_raw
                            : reinterpret_cast<uint8_t*>(
@@ -240,12 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_QFULL + s], 1);
       mbar_init(&bars[B_QEMPTY + s], 1);
       mbar_init(&bars[B_DQFULL + s], 1);
-      mbar_init(&bars[B_DQREAD + s], kDqThreads);
+      mbar_init(&bars[B_DQREAD + s], R::DQ_READERS);
     }
     mbar_init(&bars[B_SFULL], 1);
     mbar_init(&bars[B_DPFULL], 1);
-    mbar_init(&bars[B_PFULL], kComputeThreads);
-    mbar_init(&bars[B_DSFULL], kComputeThreads);
+    mbar_init(&bars[B_PFULL], R::E_THREADS);
+    mbar_init(&bars[B_DSFULL], R::E_THREADS);
     mbar_init(&bars[B_DVDONE], 1);
     mbar_init(&bars[B_DKDONE], 1);
     mbar_init(&bars[B_DONE], 1);
@@ -268,12 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicExch(p.status, kStatusTimeout);
   };
 
-  // Registers move from the control warpgroup (warps 12-15) to the others;
-  // each budget is set at the head of its role's branch so that the compiler
-  // allocates that branch's code against it.
-  if (warp >= kMmaWarp) {
-    regs_to<RegSplit<D>::kCtl, kLaunchRegs>();
-  if (warp == kTmaWarp) {
+  // Registers move from the control warpgroup to the others; each budget is
+  // set at the head of its role's branch so that the compiler allocates that
+  // branch's code against it.
+  if (warp >= R::MMA_WARP) {
+    regs_to<R::R_CTL, R::LAUNCH_REGS>();
+  if (warp == R::TMA_WARP) {
     // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
       prefetch_tensormap(&tm_q);
@@ -314,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars[B_QFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == R::MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     // Issue order per query tile i: dV(i), S(i+1), dK(i), dQ(i), dP(i+1); S(0)
     // and dP(0) before the loop. Each wait guards one TMEM or shared-memory
@@ -359,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col(16 * kk), desc_mnmajor<D>(stage_do(it), kk),
+          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col<QC>(16 * kk), desc_mnmajor<D>(stage_do(it), kk),
                  ID_KV, (it > 0 || kk > 0));
         mma_commit(&bars[B_DVDONE]);
         if (more) {
@@ -374,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col(16 * kk), desc_mnmajor<D>(stage_q(it), kk),
+          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk), desc_mnmajor<D>(stage_q(it), kk),
                  ID_KV, (it > 0 || kk > 0));
         mma_commit(&bars[B_DKDONE]);
         // dQ_i = dS K_j (dS from shared memory)
@@ -413,9 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  } else if (warp >= kDqWarp0) {
-    regs_to<RegSplit<D>::kDq, kLaunchRegs>();
-    // ------------------------------------------------ dQ warpgroup (warps 8-11)
+  } else if (warp >= R::DQ_WARP0) {
+    regs_to<R::R_DQ, R::LAUNCH_REGS>();
+    // ------------------------------------------------ dQ warpgroup
     const int t = ((warp & 3) << 5) | (threadIdx.x & 31);  // TMEM lane = query row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     auto wait_w = [&](int b, uint32_t parity) {
@@ -451,13 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) fail();
   } else {
-    regs_to<RegSplit<D>::kCompute, kLaunchRegs>();
-    // ------------------------------------------------ element-wise warps 0-7
+    regs_to<R::R_E, R::LAUNCH_REGS>();
+    // ------------------------------------------------ element-wise warpgroups
     const int t = threadIdx.x & 127;  // TMEM lane: key row
-    const int g = threadIdx.x >> 7;   // query columns [64g, 64g+64), channels [g*D/2, ...)
+    const int g = threadIdx.x >> 7;   // query columns [QC*g, QC*(g+1)), channels [g*E_CH, ...)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int key = j0 + t;
-    const int qb = 64 * g;
+    const int qb = QC * g;
     // Outcome of a wait, made uniform across the warp: the TMEM accesses that
     // follow are warp-collective, so a warp must never split on a timeout.
     auto wait_w = [&](int b, uint32_t parity) {
@@ -476,21 +492,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e) -> bf16 into region A
       if (!(ok = wait_w(B_SFULL, it & 1))) break;
       tc_fence_after();
-      uint32_t pk[32];  // this thread's 64 P values as bf16 pairs, kept for the dS pass
+      uint32_t pk[QC / 2];  // this thread's QC P values as bf16 pairs, kept for the dS pass
       {
-        uint32_t sr[64];
-        tmem_ld32(lane_base + L::T_S + qb, *reinterpret_cast<uint32_t(*)[32]>(sr));
-        tmem_ld32(lane_base + L::T_S + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        uint32_t sr[QC];
+        tmem_ld<QC>(lane_base + L::T_S + qb, sr);
         tmem_ld_wait(sr);
         // Only the diagonal tile and the key tile past N mask anything.
         if (__any_sync(0xffffffffu, thr > qb))
-          p_from_scores<true>(sr, lse_s + qb, p.scale_log2, thr - qb, pk);
+          p_from_scores<true, QC>(sr, lse_s + qb, p.scale_log2, thr - qb, pk);
         else
-          p_from_scores<false>(sr, lse_s + qb, p.scale_log2, 0, pk);
+          p_from_scores<false, QC>(sr, lse_s + qb, p.scale_log2, 0, pk);
       }
-      // both S^T chunks were read above, so the packed P may overwrite them
-      tmem_st16(lane_base + L::T_S + p_col(qb), *reinterpret_cast<uint32_t(*)[16]>(pk));
-      tmem_st16(lane_base + L::T_S + p_col(qb + 32), *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+      // all of this group's S^T columns were read above, so the packed P may
+      // overwrite the first half of them
+#pragma unroll
+      for (int c = 0; c < QC / 2; c += 16)
+        tmem_st16(lane_base + L::T_S + p_col<QC>(qb) + c,
+                  *reinterpret_cast<uint32_t(*)[16]>(pk + c));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[B_PFULL]);
@@ -498,14 +516,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- dS^T = P^T o (dP^T - D) -> bf16 into region B and shared memory
       if (!(ok = wait_w(B_DPFULL, it & 1))) break;
       tc_fence_after();
-      uint32_t dk[32];
+      uint32_t dk[QC / 2];
       {
-        uint32_t dr[64];
-        tmem_ld32(lane_base + L::T_DP + qb, *reinterpret_cast<uint32_t(*)[32]>(dr));
-        tmem_ld32(lane_base + L::T_DP + qb + 32, *reinterpret_cast<uint32_t(*)[32]>(dr + 32));
+        uint32_t dr[QC];
+        tmem_ld<QC>(lane_base + L::T_DP + qb, dr);
         tmem_ld_wait(dr);
 #pragma unroll
-        for (int u = 0; u < 64; u += 4) {
+        for (int u = 0; u < QC; u += 4) {
           const int q0 = qb + u;
           const float4 d4 = *reinterpret_cast<const float4*>(d_s + q0);
           const float2 pa = unpack_bf16x2(pk[u / 2]);
@@ -516,14 +533,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       pb.y * (__uint_as_float(dr[u + 3]) - d4.w));
         }
       }
-      // dS^T for dK (TMEM A operand); both dP^T chunks were read above
-      tmem_st16(lane_base + L::T_DP + p_col(qb), *reinterpret_cast<uint32_t(*)[16]>(dk));
-      tmem_st16(lane_base + L::T_DP + p_col(qb + 32), *reinterpret_cast<uint32_t(*)[16]>(dk + 16));
+      // dS^T for dK (TMEM A operand); all dP^T columns of the group were read above
+#pragma unroll
+      for (int c = 0; c < QC / 2; c += 16)
+        tmem_st16(lane_base + L::T_DP + p_col<QC>(qb) + c,
+                  *reinterpret_cast<uint32_t(*)[16]>(dk + c));
       // dS for dQ (shared memory, read transposed by the MMA). dQ(it-1) has
       // finished reading the previous tile: dP^T(it) was issued after it.
       uint8_t* sdS = smem + L::DS_OFF;
 #pragma unroll
-      for (int v = 0; v < 8; ++v)
+      for (int v = 0; v < QC / 8; ++v)
         st_shared_v4(smem_u32(sdS) + ds_offset(t, qb / 8 + v), dk[4 * v], dk[4 * v + 1],
                      dk[4 * v + 2], dk[4 * v + 3]);
       tmem_st_wait();
@@ -537,22 +556,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       tc_fence_after();
       // Epilogue: dV_j and scale * dK_j rows -> bf16, group g writing channels
-      // [g*D/2, (g+1)*D/2). All lanes load; only the stores are predicated.
+      // [g*E_CH, (g+1)*E_CH). All lanes load; only the stores are predicated.
       const bool key_ok = key < p.N;
       __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
       __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
-      constexpr int W = L::HALF_D >= 32 ? 32 : 16;
+      constexpr int W = R::E_CH >= 32 ? 32 : R::E_CH;
 #pragma unroll 1
-      for (int c = 0; c < L::HALF_D / W; ++c) {
-        const int ch = g * L::HALF_D + W * c;
+      for (int c = 0; c < R::E_CH / W; ++c) {
+        const int ch = g * R::E_CH + W * c;
         uint32_t rv[W], rk[W];
-        if constexpr (W == 32) {
-          tmem_ld32(lane_base + L::T_DV + ch, rv);
-          tmem_ld32(lane_base + L::T_DK + ch, rk);
-        } else {
-          tmem_ld16(lane_base + L::T_DV + ch, rv);
-          tmem_ld16(lane_base + L::T_DK + ch, rk);
-        }
+        tmem_ld<W>(lane_base + L::T_DV + ch, rv);
+        tmem_ld<W>(lane_base + L::T_DK + ch, rk);
         tmem_ld_wait(rv, rk);
 #pragma unroll
         for (int v = 0; v < W / 8 && key_ok; ++v) {
@@ -598,7 +612,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
     cudaFuncAttributes fa;
     const cudaError_t r = cudaFuncGetAttributes(&fa, kern);
     if (r != cudaSuccess) return r;
-    return fa.numRegs == static_cast<int>(kLaunchRegs) ? cudaSuccess
+    return fa.numRegs == static_cast<int>(Roles<D>::LAUNCH_REGS) ? cudaSuccess
                                                        : cudaErrorInvalidConfiguration;
   }();
   if (regs_ok != cudaSuccess) return regs_ok;
@@ -627,7 +641,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.wait_cycles = wait_cycles;
   p.inject_fault = inject;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
-  kern<<<grid, kThreads, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
+  kern<<<grid, Roles<D>::THREADS, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
   return cudaGetLastError();
 }
 
