@@ -1,21 +1,33 @@
 // Forward of causal softmax attention on the sm_100a tensor cores (tcgen05).
 //
-// One CTA per (query tile i of 128 rows, head bh). For each key tile j that
-// the causal filter lets tile i see (j <= i):
+// One CTA per (query tile i of 128 rows, head bh), walking the key tiles j
+// that the causal filter lets tile i see (j <= i):
 //
-//   S   = Q_i K_j^T                    (tcgen05 MMA -> TMEM, lane = query row)
-//   m   = max(m, rowmax S * scale*log2e);  P = exp2(S * scale*log2e - m)
-//   z   = z * exp2(m_old - m) + rowsum P   (one thread per row, CUDA cores)
-//   O_j = P V_j                        (tcgen05 MMA -> TMEM), O = O*alpha + O_j
+//   S_j = Q_i K_j^T                    (tcgen05 MMA -> TMEM, lane = query row)
+//   m   = running row maximum of S * scale*log2e
+//   P_j = exp2(S_j * scale*log2e - m)  -> bf16, in place in S_j's columns
+//   O  += P_j V_j                      (tcgen05, A = P_j read from TMEM; O
+//                                       accumulates in TMEM across tiles)
+//   z  += rowsum P_j
 //
-// and writes O = O / z (bf16) and LSE = (m + log2 z) * ln 2, the one saved
-// number per row of ddx issue #243 (item 2). The max-shifted softmax is the
+// and writes O / z (bf16) and LSE = (m + log2 z) ln 2, the one saved number
+// per row of ddx issue #243 (item 2). The max-shifted softmax is the
 // `weights` / `norm` steps of ddx issue #217's repro; the key filter is its
-// `WHERE q.pos >= k.pos` (diagonal kept).
+// `WHERE q.pos >= k.pos` (diagonal kept). m is only raised when the row
+// maximum exceeds it by more than 8 (P stays below 2^8, exact in fp32 and
+// well inside bf16's range); O and z are then scaled by 2^(m_old - m_new)
+// before the next P V accumulates, which after the first tiles is rare.
 //
-// Warp roles as in the backward: warps 0-3 own one query row each (TMEM lane
-// = row), warp 4 issues TMA loads and MMAs from one elected lane.
+// Warps (384 threads): 0-7 two softmax warpgroups (thread t of group g owns
+// query row i0 + t = TMEM lane t, key columns [64g, 64g+64) of every S tile
+// and O channels [g*d/2, (g+1)*d/2)); the two halves of a row exchange their
+// maxima through shared memory. Warp 8 issues the MMAs, warp 9 loads K tiles
+// and warp 10 V tiles by TMA; warp 11 idles. TMEM: three S buffers
+// [0,384), O [384, 384+d): S_{j+2} is computed while the softmax works on
+// S_{j+1} and P_j V_j accumulates.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -34,6 +46,13 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kFwdThreads = 384;
+constexpr int kSoftmaxThreads = 256;  // warps 0-7
+constexpr int kFwdMmaWarp = 8;
+constexpr int kFwdKWarp = 9;
+constexpr int kFwdVWarp = 10;
+constexpr float kRescaleMargin = 8.f;  // log2 units: m is raised when the max exceeds it by this
+
 template <int D>
 struct FwdLayout {
   static constexpr int CH = D >= 64 ? 64 : D;
@@ -42,27 +61,33 @@ struct FwdLayout {
   static constexpr int CHUNK = kTile * ROWB;
   static constexpr int TILE = NCH * CHUNK;
   static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128B : kSwizzle64B;
-  static constexpr int STAGES = 2;
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;                 // [STAGES] tiles
-  static constexpr int V_OFF = K_OFF + STAGES * TILE;        // [STAGES] tiles
-  static constexpr int P_OFF = V_OFF + STAGES * TILE;        // [128 q][128 k] bf16
-  static constexpr int BAR_OFF = P_OFF + 32768;
-  static constexpr int MISC_OFF = BAR_OFF + 16 * 8;
+  static constexpr int K_OFF = Q_OFF + TILE;        // [2] tiles
+  static constexpr int V_OFF = K_OFF + 2 * TILE;    // [2] tiles
+  static constexpr int XM_OFF = V_OFF + 2 * TILE;   // [2][2][128] f32: row maxima / sums exchanged
+  static constexpr int BAR_OFF = XM_OFF + 2048;
+  static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
   static constexpr int BYTES = MISC_OFF + 64;
   static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
-  static constexpr uint32_t T_S = 0, T_O = 128;
-  static constexpr uint32_t T_COLS = 256;
+  static constexpr int SBUF = 3;                    // S buffers in TMEM
+  static constexpr uint32_t T_S = 0, T_O = 128 * SBUF;
+  static constexpr uint32_t T_COLS = 512;
+  static constexpr int HALF_D = D / 2;              // O channels per softmax group
+  static_assert(T_O + D <= T_COLS, "TMEM columns exceeded");
 };
 
-enum FBar { F_Q = 0, F_KVFULL = 1, F_KVEMPTY = 3, F_SFULL = 5, F_PFULL, F_OFULL, F_OREAD,
-            F_FINAL, F_COUNT };
+enum FBar {
+  F_Q = 0, F_KFULL = 1, F_KEMPTY = 3, F_VFULL = 5, F_VEMPTY = 7, F_SFULL = 9,
+  F_PFULL = F_SFULL + 3, F_PVDONE, F_XCHG = F_PVDONE + 2, F_FINAL, F_COUNT
+};
+static_assert(F_COUNT <= 32, "barrier slots");
 
 struct FwdParams {
   __nv_bfloat16* o;  // [BH][N][D]
   float* lse;        // [BH][N]
   int* status;
   int N, T, BH;
+  int G;             // heads per scheduling group (see the CTA order)
   int causal;
   float scale_log2;
   uint64_t wait_cycles;
@@ -79,16 +104,12 @@ __device__ __forceinline__ uint64_t fdesc_mnmajor(uint32_t tile, int kk) {
   using L = FwdLayout<D>;
   return smem_desc(tile + kk * 16 * L::ROWB, L::CHUNK, 8 * L::ROWB, L::SWZ);
 }
-__device__ __forceinline__ uint64_t fdesc_p_kmajor(uint32_t tile, int kk) {
-  const int e = kk * 16;
-  return smem_desc(tile + (e / 64) * 16384 + (e % 64) * 2, 16, 1024, kSwizzle128B);
-}
-__device__ __forceinline__ uint32_t fp_offset(int r, int g) {
-  return (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4);
-}
+// TMEM column of the bf16 pair holding key k (k even) of P_j in its S buffer:
+// each softmax group packs its 64 keys into the first 32 of its own columns.
+__host__ __device__ constexpr uint32_t fp_col(int k) { return 64 * (k >> 6) + ((k & 63) >> 1); }
 
 template <int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -101,25 +122,32 @@ __global__ void __launch_bounds__(160, 1)
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const volatile int* never = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+  float* xm = reinterpret_cast<float*>(smem + L::XM_OFF);  // [2 uses][2 groups][128 rows]
 
   const int warp = threadIdx.x >> 5;
-  // longest-first: the last query tiles see the most key tiles
-  const int it_q = p.causal ? (p.T - 1 - static_cast<int>(blockIdx.x) / p.BH)
-                            : static_cast<int>(blockIdx.x) / p.BH;
-  const int bh = blockIdx.x % p.BH;
+  // CTA order: heads in groups of G (their K and V stay in L2 while all of
+  // their query tiles pass), longest query tile first inside a group.
+  const int per_group = p.T * p.G;
+  const int g0 = (blockIdx.x / per_group) * p.G;
+  const int r = blockIdx.x % per_group;
+  const int gs = min(p.G, p.BH - g0);
+  const int it_q = p.causal ? p.T - 1 - r / gs : r / gs;
+  const int bh = g0 + r % gs;
   const int i0 = it_q * kTile;
   const int n_kv = p.causal ? it_q + 1 : p.T;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[F_Q], 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[F_KVFULL + s], 1);
-      mbar_init(&bars[F_KVEMPTY + s], 1);
+      mbar_init(&bars[F_KFULL + s], 1);
+      mbar_init(&bars[F_KEMPTY + s], 1);
+      mbar_init(&bars[F_VFULL + s], 1);
+      mbar_init(&bars[F_VEMPTY + s], 1);
+      mbar_init(&bars[F_PVDONE + s], 1);
     }
-    mbar_init(&bars[F_SFULL], 1);
-    mbar_init(&bars[F_PFULL], 128);
-    mbar_init(&bars[F_OFULL], 1);
-    mbar_init(&bars[F_OREAD], 128);
+    for (int s = 0; s < 3; ++s) mbar_init(&bars[F_SFULL + s], 1);
+    mbar_init(&bars[F_PFULL], kSoftmaxThreads);
+    mbar_init(&bars[F_XCHG], kSoftmaxThreads);
     mbar_init(&bars[F_FINAL], 1);
     *abort_flag = 0;
     *const_cast<volatile int*>(never) = 0;
@@ -138,161 +166,211 @@ __global__ void __launch_bounds__(160, 1)
     atomicExch(p.status, kStatusTimeout);
   };
 
-  if (warp == 4) {
+  if (warp == kFwdKWarp || warp == kFwdVWarp) {
+    // ------------------------------------------------ TMA: Q and K (warp 9), V (warp 10)
     if (elect_one_sync()) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(&bars[F_Q], L::TILE);
-      for (int c = 0; c < L::NCH; ++c)
-        tma_load_3d(smem + L::Q_OFF + c * L::CHUNK, &tm_q, &bars[F_Q], c * L::CH, i0, bh);
-      auto load_kv = [&](int jt) {
+      const bool is_k = warp == kFwdKWarp;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      const int full = is_k ? F_KFULL : F_VFULL, empty = is_k ? F_KEMPTY : F_VEMPTY;
+      const int off = is_k ? L::K_OFF : L::V_OFF;
+      prefetch_tensormap(map);
+      if (is_k) {
+        prefetch_tensormap(&tm_q);
+        mbar_arrive_expect_tx(&bars[F_Q], L::TILE);
+        for (int c = 0; c < L::NCH; ++c)
+          tma_load_3d(smem + L::Q_OFF + c * L::CHUNK, &tm_q, &bars[F_Q], c * L::CH, i0, bh);
+      }
+      bool ok = true;
+      int issued = 0;
+      for (int jt = 0; jt < n_kv; ++jt) {
         const int s = jt & 1;
-        uint64_t* bar = &bars[F_KVFULL + s];
-        mbar_arrive_expect_tx(bar, 2 * L::TILE);
-        for (int c = 0; c < L::NCH; ++c) {
-          tma_load_3d(smem + L::K_OFF + s * L::TILE + c * L::CHUNK, &tm_k, bar, c * L::CH,
+        // K_j is free once S_j has been computed, V_j once P_j V_j has.
+        if (jt >= 2 &&
+            !(ok = mbar_wait(&bars[empty + s], ((jt - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
+          break;
+        mbar_arrive_expect_tx(&bars[full + s], L::TILE);
+        for (int c = 0; c < L::NCH; ++c)
+          tma_load_3d(smem + off + s * L::TILE + c * L::CHUNK, map, &bars[full + s], c * L::CH,
                       jt * kTile, bh);
-          tma_load_3d(smem + L::V_OFF + s * L::TILE + c * L::CHUNK, &tm_v, bar, c * L::CH,
-                      jt * kTile, bh);
-        }
-      };
-      int loaded = 0, waited = 0;
-      for (int jt = 0; jt < n_kv && jt < 2; ++jt, ++loaded) load_kv(jt);
+        ++issued;
+      }
+      if (!ok) fail();
+      // Every load issued has landed before the CTA can exit (bounded).
+      if (is_k) mbar_wait(&bars[F_Q], 0, p.wait_cycles, never);
+      for (int w = issued > 2 ? issued - 2 : 0; w < issued; ++w)
+        mbar_wait(&bars[full + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
+    }
+    __syncwarp();
+  } else if (warp == kFwdMmaWarp) {
+    // ------------------------------------------------ MMA issuer
+    // Order: S_0, S_1, then per key tile j: P_j V_j, S_{j+2} (into the buffer
+    // that P_{j-1} occupied, once P_{j-1} V_{j-1} has completed).
+    if (elect_one_sync()) {
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_O = idesc_bf16(128, D, false, true);
-      const uint32_t sQ = sbase + L::Q_OFF, sP = sbase + L::P_OFF;
-      bool ok = mbar_wait(&bars[F_Q], 0, p.wait_cycles, abort_flag);
-      const bool q_waited = ok;
-      for (int jt = 0; ok && jt < n_kv; ++jt) {
-        const int s = jt & 1;
-        const uint32_t ph = (jt >> 1) & 1;
-        const uint32_t sK = sbase + L::K_OFF + s * L::TILE;
-        const uint32_t sV = sbase + L::V_OFF + s * L::TILE;
-        if (!(ok = mbar_wait(&bars[F_KVFULL + s], ph, p.wait_cycles, abort_flag))) break;
-        ++waited;
-        // S may be overwritten once the row threads have read S(jt-1) (they
-        // arrive on F_PFULL after that).
-        tc_fence_after();
+      const uint32_t sQ = sbase + L::Q_OFF;
+      auto wait = [&](int b, uint32_t parity) {
+        return mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag);
+      };
+      auto issue_s = [&](int jt) {
+        const uint32_t sK = sbase + L::K_OFF + (jt & 1) * L::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::T_S, fdesc_kmajor<D>(sQ, kk), fdesc_kmajor<D>(sK, kk), ID_S, kk > 0);
-        mma_commit(&bars[F_SFULL]);
-        if (!(ok = mbar_wait(&bars[F_PFULL], jt & 1, p.wait_cycles, abort_flag))) break;
-        // O_j lands where the threads read O_(jt-1); they arrive on F_OREAD after.
-        if (jt > 0 && !(ok = mbar_wait(&bars[F_OREAD], (jt - 1) & 1, p.wait_cycles, abort_flag)))
-          break;
+          mma_ss(tmem + L::T_S + (jt % 3) * 128, fdesc_kmajor<D>(sQ, kk), fdesc_kmajor<D>(sK, kk),
+                 ID_S, kk > 0);
+        mma_commit(&bars[F_SFULL + jt % 3]);
+        mma_commit(&bars[F_KEMPTY + (jt & 1)]);
+      };
+      bool ok = wait(F_Q, 0) && wait(F_KFULL, 0);
+      if (ok) {
         tc_fence_after();
+        issue_s(0);
+        if (n_kv > 1 && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
+      }
+      for (int jt = 0; ok && jt < n_kv; ++jt) {
+        if (!(ok = wait(F_PFULL, jt & 1))) break;
+        if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t sV = sbase + L::V_OFF + (jt & 1) * L::TILE;
+        const uint32_t pbuf = tmem + L::T_S + (jt % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_O, fdesc_p_kmajor(sP, kk), fdesc_mnmajor<D>(sV, kk), ID_O, kk > 0);
-        mma_commit(&bars[F_OFULL]);
-        mma_commit(&bars[F_KVEMPTY + s]);
+          mma_ts(tmem + L::T_O, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk), ID_O,
+                 (jt > 0 || kk > 0));
+        mma_commit(&bars[F_PVDONE + (jt & 1)]);
+        mma_commit(&bars[F_VEMPTY + (jt & 1)]);
         if (jt + 2 < n_kv) {
-          if (!(ok = mbar_wait(&bars[F_KVEMPTY + s], ph, p.wait_cycles, abort_flag))) break;
-          load_kv(jt + 2);
-          ++loaded;
+          // S_{j+2} overwrites P_{j-1}, which P_{j-1} V_{j-1} reads
+          if (jt >= 1 && !(ok = wait(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
+          if (!(ok = wait(F_KFULL + (jt & 1), ((jt + 2) >> 1) & 1))) break;
+          tc_fence_after();
+          issue_s(jt + 2);
         }
       }
-      if (!ok) {
-        fail();
-        if (!q_waited) mbar_wait(&bars[F_Q], 0, p.wait_cycles, never);
-        for (int w = waited; w < loaded; ++w)
-          mbar_wait(&bars[F_KVFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
-      }
+      if (!ok) fail();
       mma_commit(&bars[F_FINAL]);
       mbar_wait(&bars[F_FINAL], 0, p.wait_cycles, never);
     }
     __syncwarp();
-  } else {
-    const int t = threadIdx.x;
+  } else if (warp < 8) {
+    // ------------------------------------------------ softmax warpgroups
+    const int t = threadIdx.x & 127;
+    const int g = threadIdx.x >> 7;
     const int qrow = i0 + t;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float o[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) o[c] = 0.f;
-    float m = -INFINITY, z = 0.f;
-    // Wait outcomes are made warp-uniform: the TMEM loads are warp-collective.
-    auto wait_w = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_cycles, abort_flag));
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    // Wait outcomes are made warp-uniform: the TMEM accesses are warp-collective.
+    auto wait_w = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
     };
+    float m = -INFINITY, z = 0.f;
     bool ok = true;
-    uint8_t* sP = smem + L::P_OFF;
     for (int jt = 0; jt < n_kv; ++jt) {
-      const int j0 = jt * kTile;
+      const int kb = jt * kTile + 64 * g;  // first key of this thread's 64 columns
       // keys with local index >= lim are excluded for this row
-      int lim = p.N - j0;
-      if (p.causal && qrow - j0 + 1 < lim) lim = qrow - j0 + 1;
-      if (!(ok = wait_w(&bars[F_SFULL], jt & 1))) break;
+      int lim = p.N - kb;
+      if (p.causal && qrow - kb + 1 < lim) lim = qrow - kb + 1;
+      const bool masked = __any_sync(0xffffffffu, lim < 64);
+      if (!(ok = wait_w(F_SFULL + jt % 3, (jt / 3) & 1))) break;
       tc_fence_after();
+      const uint32_t sbuf = lane_base + L::T_S + (jt % 3) * 128;
+      uint32_t sr[64];
+      tmem_ld32(sbuf + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(sbuf + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      tmem_ld_wait(sr);
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + L::T_S + 32 * c, r);
-        tmem_ld_wait(r);
+      if (masked) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (32 * c + u < lim) mx = fmaxf(mx, __uint_as_float(r[u]));
+        for (int u = 0; u < 64; ++u)
+          if (u < lim) mx = fmaxf(mx, __uint_as_float(sr[u]));
+      } else {
+#pragma unroll
+        for (int u = 0; u < 64; ++u) mx = fmaxf(mx, __uint_as_float(sr[u]));
       }
-      const float m_new = fmaxf(m, mx * p.scale_log2);
-      // rows that have seen no key yet keep m = -inf; guard the -inf - -inf case
-      const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m - m_new);
-      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      float zt = 0.f;
+      // row maximum over both halves of the row
+      float* xmj = xm + (jt & 1) * 256;
+      xmj[g * 128 + t] = mx;
+      mbar_arrive(&bars[F_XCHG]);
+      if (!(ok = wait_w(F_XCHG, jt & 1))) break;
+      mx = fmaxf(mx, xmj[(g ^ 1) * 128 + t]) * p.scale_log2;
+      float alpha = 1.f;
+      const bool raise = mx > m + kRescaleMargin;
+      if (raise) {
+        alpha = jt > 0 ? ex2_approx(m - mx) : 1.f;
+        m = mx;
+      }
+      if (__any_sync(0xffffffffu, raise && jt > 0)) {
+        // O holds sum_{j' < j} P_j' V_j' with the old m: scale it by alpha
+        // once the last of those products has landed.
+        if (!(ok = wait_w(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
+        tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + L::T_S + 32 * c, r);
-        tmem_ld_wait(r);
-        uint32_t pk[16];
+        for (int c = 0; c < L::HALF_D; c += 16) {
+          uint32_t ov[16];
+          tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
+          tmem_ld_wait(ov);
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[u]), p.scale_log2, -msub));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[u + 1]), p.scale_log2, -msub));
-          if (32 * c + u >= lim) p0 = 0.f;
-          if (32 * c + u + 1 >= lim) p1 = 0.f;
-          zt += p0 + p1;
-          pk[u / 2] = pack_bf16x2(p0, p1);
+          for (int u = 0; u < 16; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
+          tmem_st16(lane_base + L::T_O + g * L::HALF_D + c, ov);
         }
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          st_shared_v4(smem_u32(sP) + fp_offset(t, 4 * c + v), pk[4 * v], pk[4 * v + 1],
-                       pk[4 * v + 2], pk[4 * v + 3]);
+        z *= alpha;
       }
-      z = z * alpha + zt;
-      m = m_new;
-      fence_proxy_async_smem();
+      // P = exp2(S * scale*log2e - m) -> bf16 into the first 32 of this group's columns
+      uint32_t pk[32];
+      float zt = 0.f;
+#pragma unroll
+      for (int u = 0; u < 64; u += 2) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -m));
+        float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -m));
+        if (masked) {
+          if (u >= lim) p0 = 0.f;
+          if (u + 1 >= lim) p1 = 0.f;
+        }
+        zt += p0 + p1;
+        pk[u / 2] = pack_bf16x2(p0, p1);
+      }
+      z += zt;
+      tmem_st16(sbuf + fp_col(64 * g), *reinterpret_cast<uint32_t(*)[16]>(pk));
+      tmem_st16(sbuf + fp_col(64 * g) + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[F_PFULL]);
-      if (!(ok = wait_w(&bars[F_OFULL], jt & 1))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + L::T_O + 32 * c, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) o[32 * c + u] = fmaf(o[32 * c + u], alpha, __uint_as_float(r[u]));
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[F_OREAD]);
+    }
+    // Epilogue: the last P V has landed; combine the two halves' sums.
+    if (ok) ok = wait_w(F_PVDONE + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    if (ok) {
+      float* xmz = xm + (n_kv & 1) * 256;
+      xmz[g * 128 + t] = z;
+      mbar_arrive(&bars[F_XCHG]);
+      ok = wait_w(F_XCHG, n_kv & 1);
+      if (ok) z += xmz[(g ^ 1) * 128 + t];
     }
     if (!ok) {
       fail();
-    } else if (qrow < p.N) {
+    } else {
+      tc_fence_after();
       const float inv = 1.f / z;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + qrow) * D;
+      const bool row_ok = qrow < p.N;
+      __nv_bfloat16* orow =
+          p.o + (static_cast<size_t>(bh) * p.N + (row_ok ? qrow : 0)) * D + g * L::HALF_D;
+#pragma unroll 1
+      for (int c = 0; c < L::HALF_D; c += 16) {
+        uint32_t ov[16];
+        tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
+        tmem_ld_wait(ov);
+        if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < D; c += 8) {
-        uint4 v;
-        v.x = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
-        v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
-        v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
-        v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
-        *reinterpret_cast<uint4*>(orow + c) = v;
+          for (int v = 0; v < 2; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[8 * v]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c + 8 * v) = w;
+          }
+        }
       }
-      p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(z)) * 0.6931471805599453f;
+      if (row_ok && g == 0)
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(z)) * 0.6931471805599453f;
     }
   }
   tc_fence_before();
@@ -307,6 +385,7 @@ template <int D>
 cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int BH, int N,
                          bool causal, float scale, cudaStream_t s) {
   using L = FwdLayout<D>;
+  static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = attn_fwd_bf16_sm100_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
@@ -317,11 +396,19 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
   p.N = N;
   p.T = (N + kTile - 1) / kTile;
   p.BH = BH;
+  // Heads per group: as many as fit, with their K and V tiles, in about a
+  // third of L2.
+  int dev = 0, l2 = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
+    l2 = 126 << 20;
+  const size_t head_bytes = static_cast<size_t>(p.T) * kTile * D * 4;
+  p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = kWaitLimitCycles;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
-  kern<<<grid, 160, L::ALLOC, s>>>(m.a, m.b, m.c, p);
+  kern<<<grid, kFwdThreads, L::ALLOC, s>>>(m.a, m.b, m.c, p);
   return cudaGetLastError();
 }
 
