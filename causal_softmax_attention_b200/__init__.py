@@ -199,3 +199,68 @@ def backward(q, k, v, o, dout, lse, causal: bool = True, scale: float | None = N
     ws = new_workspace(q) if workspace is None else workspace
     attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, ws, causal, scale)
     return dq, dk, dv
+
+
+def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool = True,
+                  scale: float | None = None, chunks: int = 8, stream=None):
+    """dQ, dK, dV of inputs held in (pinned) HOST memory, results written to
+    host tensors, through attn_bwd with the transfers overlapped.
+
+    The (batch, head) pairs are split into up to `chunks` consecutive groups.
+    Group c is copied to the device on one stream, its backward runs on a
+    second once its inputs have landed, and its gradients are copied back on
+    a third, so that the host->device copy of group c+1, the backward of
+    group c and the device->host copy of group c-1 proceed together.
+
+    `dev` is a dict of device buffers of the full shapes: q, k, v, o, dout
+    ([B, H, N, d]), lse ([B, H, N]), dq, dk, dv, and `workspace` sized by
+    attn_bwd_workspace_bytes for one group (chunk_workspace_bytes). The work
+    starts after everything already queued on `stream` (default: the current
+    stream) and `stream` waits for all of it to finish, so events recorded
+    on `stream` around the call time the whole transfer and compute.
+    """
+    B, H, N, d = _shape(hq)
+    BH = B * H
+    hc = max(1, -(-BH // max(1, chunks)))  # heads per group
+    caller = torch.cuda.current_stream(dev["q"].device) if stream is None else stream
+    s_in = torch.cuda.Stream(device=dev["q"].device)
+    s_run = torch.cuda.Stream(device=dev["q"].device)
+    s_out = torch.cuda.Stream(device=dev["q"].device)
+    start = torch.cuda.Event()
+    start.record(caller)
+    for s in (s_in, s_run, s_out):
+        s.wait_event(start)
+
+    def rows(t):  # [B, H, ...] -> [B*H, ...]
+        return t.reshape(BH, *t.shape[2:])
+
+    names = ("q", "k", "v", "o", "dout", "lse")
+    hosts = dict(zip(names, (hq, hk, hv, ho, hdout, hlse)))
+    outs = (("dq", hdq), ("dk", hdk), ("dv", hdv))
+    done = None
+    for c0 in range(0, BH, hc):
+        c1 = min(BH, c0 + hc)
+        with torch.cuda.stream(s_in):
+            for n in names:
+                rows(dev[n])[c0:c1].copy_(rows(hosts[n])[c0:c1], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+        s_run.wait_event(landed)
+        view = {n: rows(dev[n])[c0:c1].unsqueeze(0) for n in names + ("dq", "dk", "dv")}
+        attn_bwd(view["q"], view["k"], view["v"], view["o"], view["dout"], view["lse"],
+                 view["dq"], view["dk"], view["dv"], dev["workspace"], causal, scale, s_run)
+        ready = torch.cuda.Event()
+        ready.record(s_run)
+        s_out.wait_event(ready)
+        with torch.cuda.stream(s_out):
+            for n, h in outs:
+                rows(h)[c0:c1].copy_(rows(dev[n])[c0:c1], non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(s_out)
+    caller.wait_event(done)
+
+
+def chunk_workspace_bytes(B: int, H: int, N: int, d: int, dtype, chunks: int = 8) -> int:
+    """Workspace bytes for one group of backward_host (the largest group)."""
+    hc = max(1, -(-(B * H) // max(1, chunks)))
+    return attn_bwd_workspace_bytes(1, hc, N, d, dtype)

@@ -89,6 +89,32 @@ def test_f32_shapes(csa, B, H, N, d, causal):
 
 
 # ------------------------------------------------------------------ properties on the GPU
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_host_pipelined_matches_device(csa, dtype):
+    # host buffers in and out, heads in groups on three streams: the same
+    # gradients as one attn_bwd call on device buffers (dK, dV bit for bit;
+    # dQ up to the order of its fp32 atomic sums)
+    B, H, N, d = 2, 5, 300, 64
+    q, k, v, do = draw(B, H, N, d, 77, dtype)
+    g = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    dev = torch.device("cuda")
+    host = {n: t.pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("dout", do))}
+    host["o"] = g["O"].cpu().pin_memory()
+    host["lse"] = g["LSE"].cpu().pin_memory()
+    outs = {n: torch.empty_like(host["q"]).pin_memory() for n in ("dq", "dk", "dv")}
+    bufs = {n: torch.empty_like(host[n], device=dev) for n in ("q", "k", "v", "o", "dout", "lse")}
+    bufs.update({n: torch.empty_like(bufs["q"]) for n in ("dq", "dk", "dv")})
+    bufs["workspace"] = torch.empty(csa.chunk_workspace_bytes(B, H, N, d, bufs["q"].dtype, 4),
+                                    dtype=torch.uint8, device=dev)
+    csa.backward_host(host["q"], host["k"], host["v"], host["o"], host["dout"], host["lse"],
+                      outs["dq"], outs["dk"], outs["dv"], bufs, True, d ** -0.5, chunks=4)
+    torch.cuda.synchronize()
+    assert torch.equal(outs["dk"], g["dK"].cpu())
+    assert torch.equal(outs["dv"], g["dV"].cpu())
+    ref = as_f64(g["dQ"].cpu())
+    assert rel(as_f64(outs["dq"]), ref, np.abs(ref).max()) <= (1e-6 if dtype == "f32" else 1e-2)
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
