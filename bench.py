@@ -248,7 +248,8 @@ def config_dict(cfg, n_gpus):
             "global_batch": cfg.B * n_gpus, "seq_len": cfg.N,
             "parallelism": f"independent replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
             "l2": "inputs larger than L2 (no flush needed)"
-            if 5 * cfg.B * cfg.H * cfg.N * cfg.d * 2 > 126e6 else "L2 flushed between steps"}
+            if 5 * cfg.B * cfg.H * cfg.N * cfg.d * 2 > 126e6
+            else "L2 flushed (256 MB write) between steps, outside the steps' events"}
 
 
 # --------------------------------------------------------------------- GPU arm
@@ -268,8 +269,6 @@ def run_gpu(args, cfg, world, rank, local):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small else None
 
     def step(ev_main=None):
-        if flush is not None:
-            flush.zero_()
         csa.attn_bwd_preprocess(o, dod, lse, ws, stream)
         if ev_main is not None:
             ev_main[0].record(stream)
@@ -279,6 +278,8 @@ def run_gpu(args, cfg, world, rank, local):
         csa.attn_bwd_dq_convert(dq, ws, cfg.scale, stream)
 
     for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
         step()
     torch.cuda.synchronize()
     if csa.attn_last_status(ws) != 0:
@@ -297,6 +298,8 @@ def run_gpu(args, cfg, world, rank, local):
         t_end = torch.cuda.Event(enable_timing=True)
         t_begin.record(stream)
         for s in range(args.steps):
+            if flush is not None:  # between steps, outside the step's own events
+                flush.zero_()
             starts[s].record(stream)
             step(mains[s])
             ends[s].record(stream)
@@ -309,13 +312,8 @@ def run_gpu(args, cfg, world, rank, local):
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     main_ms = [a.elapsed_time(b) for a, b in mains]
     if flush is not None:
-        # remove the flush from the step time: time it alone
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        flush.zero_()
-        f1.record(stream)
-        torch.cuda.synchronize()
-        total_ms -= args.steps * f0.elapsed_time(f1)
+        # the L2 flushes ran between the steps: count the steps' own events
+        total_ms = sum(step_ms)
     status = csa.attn_last_status(ws)
     ms_per_step = max_over_ranks(total_ms / args.steps, world)
     flops = cfg.bwd_flops
@@ -376,28 +374,38 @@ def run_gpu(args, cfg, world, rank, local):
     peak = float(peaks["bf16_tflops"])
     traffic = dram_traffic_per_launch(cfg)
     clk = clocks.summary(host_t0, host_t1)
+    if cfg.dtype == "bf16":
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "kernel": "attn_bwd_bf16_sm100_kernel",
+                    "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                    "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                    "algorithmic_flops_per_launch": flops, "avg_launch_ms": main_avg}
+    else:
+        # the fp32 path runs on the CUDA cores: plain FFMA arithmetic
+        ffma = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": ffma, "unit": "TFLOP/s",
+                    "frac": achieved / ffma, "traffic": None,
+                    "kernel": "bwd_dkdv_f32_kernel + bwd_dq_f32_kernel",
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x sm_max_mhz",
+                    "algorithmic_flops_per_launch": flops, "avg_launch_ms": main_avg}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
         "data": "synthetic", "config": config_dict(cfg, world),
         "pct_of_dense_bf16_peak": 100.0 * value / world / peak,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "attn_bwd_bf16_sm100_kernel",
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                     "algorithmic_flops_per_launch": flops,
-                     "avg_launch_ms": main_avg},
+        "roofline": roofline,
         "stage_ms": {"step_median": statistics.median(step_ms), "main_median": statistics.median(main_ms),
                      "pre_and_convert_median": statistics.median(step_ms) - statistics.median(main_ms)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "path": f"backward_host: pinned host buffers, {e2e_chunks} head groups, "
                         "H2D / attn_bwd / D2H overlapped on three streams"},
-        "forward": {"kernel": "attn_fwd_bf16_sm100_kernel", "ms": fwd_ms,
+        "forward": {"kernel": "attn_fwd_bf16_sm100_kernel" if cfg.dtype == "bf16"
+                    else "fwd_f32_kernel", "ms": fwd_ms,
                     "tflops": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12,
-                    "frac": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12 / peak,
+                    "frac": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12 / roofline["peak"],
                     "flops_convention": "causal forward 4*B*H*N^2*d/2",
                     "note": "measured outside the timed backward step"},
         "gpu_launches": 3 * args.steps,
