@@ -5,5 +5,5 @@ arm may import it. It shares no code with the CUDA library.
 """
 from .attention_f64 import (  # noqa: F401
     backward, backward_head, backward_head_with_shift, backward_row_block,
-    causal_pair_count, forward, forward_head, keep_mask, key_tail, query_rows,
+    block_mask_keep, causal_pair_count, forward, forward_head, keep_mask, key_tail, query_rows,
 )

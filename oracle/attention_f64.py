@@ -24,7 +24,9 @@ time, in numpy float64:
   explicitly, used only to check that the shift's gradient cancels.
 
 Masked scores are excluded with a boolean mask (P is exactly 0 there), never
-with an additive large negative number.
+with an additive large negative number. Besides the causal and full filters,
+any boolean mask can be given, and ``block_mask_keep`` expands a block mask
+(one kind per 128 x 128 tile: none, all, or causal inside the tile) into one.
 
 Pins (tests/test_oracle.py): central finite differences, softmax
 normalisation, invariance to a per-row score shift, with-shift == without-shift
@@ -52,7 +54,25 @@ def keep_mask(n_q: int, n_k: int, causal: bool, q_offset: int = 0) -> np.ndarray
     return i >= j
 
 
-def forward_head(q, k, v, scale, causal=True, row_shift=None):
+def block_mask_keep(block_mask, n: int, tile: int = 128) -> np.ndarray:
+    """Boolean [n, n] mask of the scores kept under a block mask.
+
+    ``block_mask[a, b]`` describes the tile of query rows [a*tile, (a+1)*tile)
+    and key columns [b*tile, (b+1)*tile): 0 keeps none of its scores, 1 keeps
+    all of them, 2 keeps those whose key lies at or before the query inside
+    the tile (local key index <= local query index). The causal filter is the
+    instance 1 below the diagonal, 2 on it, 0 above: the block-sparse
+    generalisation of the mask that ddx PR #162 applies as a filter on the
+    grouping keys.
+    """
+    bm = np.asarray(block_mask)
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    kind = bm[i // tile, j // tile]
+    return (kind == 1) | ((kind == 2) & (j % tile <= i % tile))
+
+
+def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None):
     """Forward of one head. q, k, v: [N, d] float64.
 
     Returns a dict with S (scores, including ``row_shift`` if given), keep,
@@ -60,7 +80,9 @@ def forward_head(q, k, v, scale, causal=True, row_shift=None):
 
     ``row_shift`` (length-N, optional) is added to row i of the scores before
     the softmax; it exists only to test the invariance of everything but LSE
-    to such a shift.
+    to such a shift. ``keep`` (boolean [N_q, N_k], optional) replaces the
+    causal / full filter; a row that keeps no score has P = 0, O = 0 and
+    LSE = -inf (the log of an empty sum).
     """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -69,25 +91,27 @@ def forward_head(q, k, v, scale, causal=True, row_shift=None):
     S = scale * (q @ k.T)
     if row_shift is not None:
         S = S + np.asarray(row_shift, np.float64)[:, None]
-    keep = keep_mask(n, k.shape[0], causal)
+    keep = keep_mask(n, k.shape[0], causal) if keep is None else np.asarray(keep, bool)
     m = np.where(keep, S, -np.inf).max(axis=1)
     w = np.zeros_like(S)
     w[keep] = np.exp((S - m[:, None])[keep])
     z = w.sum(axis=1)
-    P = w / z[:, None]
+    empty = z == 0
+    P = w / np.where(empty, 1.0, z)[:, None]
     O = P @ v
-    LSE = m + np.log(z)
+    with np.errstate(divide="ignore"):
+        LSE = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, z)))
     return {"S": S, "keep": keep, "m": m, "w": w, "z": z, "P": P, "O": O, "LSE": LSE}
 
 
-def backward_head(q, k, v, do, scale, causal=True, row_shift=None):
+def backward_head(q, k, v, do, scale, causal=True, row_shift=None, keep=None):
     """Backward of one head without the shift's gradient.
 
     Returns dict(dQ, dK, dV, D, D_rows, dS, fwd) where D = sum_c dO o O (the
     form the GPU uses) and D_rows = sum_j P o dP (the softmax-weighted sum of
     ddx issue #243 item 2); the two agree up to rounding.
     """
-    f = forward_head(q, k, v, scale, causal, row_shift)
+    f = forward_head(q, k, v, scale, causal, row_shift, keep)
     do = np.asarray(do, np.float64)
     k = np.asarray(k, np.float64)
     q = np.asarray(q, np.float64)
@@ -140,22 +164,24 @@ def backward_head_with_shift(q, k, v, do, scale, causal=True, row_shift=None,
     return {"dQ": dQ, "dK": dK, "dV": dV, "dm": dm, "dS": dS}
 
 
-def forward(q, k, v, scale, causal=True):
-    """Batched forward. q, k, v: [B, H, N, d]. Returns O [B,H,N,d], LSE [B,H,N]."""
+def forward(q, k, v, scale, causal=True, keep=None):
+    """Batched forward. q, k, v: [B, H, N, d]. Returns O [B,H,N,d], LSE [B,H,N].
+    ``keep`` (boolean [N, N], optional) is shared by every head."""
     q = np.asarray(q, np.float64)
     B, H, N, d = q.shape
     O = np.empty((B, H, N, v.shape[-1]))
     LSE = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
-            f = forward_head(q[b, h], k[b, h], v[b, h], scale, causal)
+            f = forward_head(q[b, h], k[b, h], v[b, h], scale, causal, keep=keep)
             O[b, h] = f["O"]
             LSE[b, h] = f["LSE"]
     return O, LSE
 
 
-def backward(q, k, v, do, scale, causal=True):
-    """Batched backward. Returns dQ, dK, dV [B,H,N,d], O, LSE and D [B,H,N]."""
+def backward(q, k, v, do, scale, causal=True, keep=None):
+    """Batched backward. Returns dQ, dK, dV [B,H,N,d], O, LSE and D [B,H,N].
+    ``keep`` (boolean [N, N], optional) is shared by every head."""
     q = np.asarray(q, np.float64)
     B, H, N, d = q.shape
     out = {name: np.empty(q.shape) for name in ("dQ", "dK", "dV", "O")}
@@ -163,7 +189,7 @@ def backward(q, k, v, do, scale, causal=True):
     out["D"] = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
-            r = backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal)
+            r = backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal, keep=keep)
             for name in ("dQ", "dK", "dV", "D"):
                 out[name][b, h] = r[name]
             out["O"][b, h] = r["fwd"]["O"]

@@ -311,3 +311,80 @@ def test_pair_count_catches_a_mask_without_diagonal(monkeypatch):
         return (i > np.arange(n_k)[None, :]) if causal else np.ones((n_q, n_k), bool)
     monkeypatch.setattr(A, "keep_mask", strict)
     assert A.causal_pair_count(3, 2, 8) != 216
+
+
+# --------------------------------------------------------------------------
+# general and block masks (block-sparse attention)
+# --------------------------------------------------------------------------
+def causal_block_mask(n, tile=128):
+    t = -(-n // tile)
+    a = np.arange(t)
+    return np.where(a[:, None] > a[None, :], 1, np.where(a[:, None] == a[None, :], 2, 0))
+
+
+@pytest.mark.parametrize("n", [1, 5, 128, 130, 257, 640])
+def test_block_mask_expands_causal_and_full(n):
+    assert np.array_equal(A.block_mask_keep(causal_block_mask(n), n), A.keep_mask(n, n, True))
+    t = -(-n // 128)
+    assert A.block_mask_keep(np.ones((t, t), int), n).all()
+    assert not A.block_mask_keep(np.zeros((t, t), int), n).any()
+
+
+def test_block_mask_kind_two_off_the_diagonal():
+    # kind 2 keeps local key <= local query inside any tile, not only on the diagonal
+    bm = np.array([[0, 0], [2, 0]])
+    keep = A.block_mask_keep(bm, 200)
+    assert keep[128 + 5, 5] and keep[128 + 5, 0] and not keep[128 + 5, 6]
+    assert not keep[:128].any() and not keep[:, 128:].any()
+
+
+def masked_loss(q, k, v, do, scale, keep):
+    return float((do * A.forward_head(q, k, v, scale, keep=keep)["O"]).sum())
+
+
+def test_finite_differences_under_a_mask_with_an_empty_row():
+    q, k, v, do = tiny_case(seed=40)
+    rng = np.random.default_rng(41)
+    keep = rng.random((8, 8)) < 0.5
+    keep[np.arange(8), rng.integers(0, 8, 8)] = True
+    keep[3] = False  # a row that keeps nothing
+    scale, h = 0.5, 1e-6
+    r = A.backward_head(q, k, v, do, scale, keep=keep)
+    f = r["fwd"]
+    assert np.all(f["O"][3] == 0) and f["LSE"][3] == -np.inf
+    assert np.all(r["dQ"][3] == 0)
+    for which, an in ((0, r["dQ"]), (1, r["dK"]), (2, r["dV"])):
+        args = [q, k, v]
+        g = np.zeros_like(args[which])
+        for idx in np.ndindex(g.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            g[idx] = (masked_loss(*plus, do, scale, keep) - masked_loss(*minus, do, scale, keep)) / (2 * h)
+        assert np.all(np.abs(an - g) <= 1e-7 * np.abs(g).max() + 1e-9)
+
+
+def test_torch_autograd_cross_check_block_mask():
+    # a separately written formula: softmax over the kept scores (rows with
+    # none kept give zero), through float64 autograd
+    B, H, N, d = 1, 2, 300, 16
+    q, k, v, do = (rnd(60 + t, B, H, N, d) for t in range(4))
+    bm = np.random.default_rng(65).integers(0, 3, (3, 3))
+    bm[1, :] = 0  # query tile 1 keeps nothing
+    keep = A.block_mask_keep(bm, N)
+    out = A.backward(q, k, v, do, 0.25, keep=keep)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    s = 0.25 * tq @ tk.transpose(-1, -2)
+    km = torch.tensor(keep)
+    s = s.masked_fill(~km, float("-inf"))
+    row_any = km.any(-1, keepdim=True)
+    p = torch.where(row_any, torch.softmax(torch.where(row_any, s, torch.zeros_like(s)), -1),
+                    torch.zeros_like(s))
+    p = torch.where(km, p, torch.zeros_like(p))
+    o = p @ tv
+    (o * torch.tensor(do)).sum().backward()
+    assert rel(out["O"], o.detach().numpy()) <= 1e-12
+    for name, g in (("dQ", tq.grad), ("dK", tk.grad), ("dV", tv.grad)):
+        assert rel(out[name], g.numpy()) <= 1e-12
+    assert np.all(out["LSE"][:, :, 128:256] == -np.inf)
