@@ -329,7 +329,7 @@ def run_gpu(args, cfg, world, rank, local):
     # Host buffers in, host gradients out, through the package's pipelined
     # host path: groups of heads are copied in, differentiated and copied out
     # on three streams, each backward an attn_bwd call of the C ABI.
-    e2e_chunks = 8
+    e2e_chunks = max(1, min(args.e2e_chunks, B * H))
     ws_chunk = torch.empty(csa.chunk_workspace_bytes(B, H, N, d, qd.dtype, e2e_chunks),
                            dtype=torch.uint8, device=dev)
     dev_bufs = {"q": qd, "k": kd, "v": vd, "o": o, "dout": dod, "lse": lse, "dq": dq, "dk": dk,
@@ -429,6 +429,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="head groups of the end-to-end (host-buffer) measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

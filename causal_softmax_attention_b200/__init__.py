@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
         "attn_status_string": (ctypes.c_char_p, [i]),
         "attn_test_arm_timeout": (i, [ctypes.c_ulonglong]),
         "attn_bwd_noalloc": (i, [vp] * 9 + [i, i, i, i, i, f, i, vp]),
+        "attn_fwd_masked": (i, [vp] * 5 + [i, i, i, i, vp, f, i, vp]),
+        "attn_bwd_masked": (i, [vp] * 9 + [i, i, i, i, vp, f, i, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -64,7 +66,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
-            "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc")
+            "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc", "attn_fwd_masked",
+            "attn_bwd_masked")
 
 
 def library() -> ctypes.CDLL:
@@ -264,3 +267,35 @@ def chunk_workspace_bytes(B: int, H: int, N: int, d: int, dtype, chunks: int = 8
     """Workspace bytes for one group of backward_host (the largest group)."""
     hc = max(1, -(-(B * H) // max(1, chunks)))
     return attn_bwd_workspace_bytes(1, hc, N, d, dtype)
+
+
+def block_mask_tiles(N: int) -> int:
+    """Side of the block mask for N positions: ceil(N / 128) tiles."""
+    return -(-N // 128)
+
+
+def attn_fwd_masked(q, k, v, o, lse, block_mask, scale: float | None = None, stream=None,
+                    check: bool = True) -> int:
+    """O, LSE <- block-sparse forward; `block_mask` is a CUDA uint8 [T, T]
+    tensor of tile kinds (0 none, 1 all, 2 key <= query inside the tile)."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                              _ptr(block_mask), float(scale), _DTYPES[q.dtype], _stream(stream))
+    if check:
+        _check(st, "attn_fwd_masked")
+    return st
+
+
+def attn_bwd_masked(q, k, v, o, dout, lse, dq, dk, dv, block_mask, workspace,
+                    scale: float | None = None, stream=None, check: bool = True) -> int:
+    """dQ, dK, dV <- block-sparse backward (same block mask as the forward)."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _ptr(block_mask),
+                              float(scale), _DTYPES[q.dtype], _ptr(workspace),
+                              int(workspace.numel()), _stream(stream))
+    if check:
+        _check(st, "attn_bwd_masked")
+    return st

@@ -145,8 +145,11 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
   return workspace_layout(B, H, N, d, dtype).total;
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int N, int d, int causal, float scale, int dtype, void* stream) {
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, int causal, float scale, int dtype, const uint8_t* bmask,
+             void* stream) {
   if (!all_aligned({q, k, v, o, lse})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
@@ -164,7 +167,23 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return ATTN_ERR_CUDA;
   int* status = fwd_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
-  return from_cuda(launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, s));
+  return from_cuda(launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, bmask, s));
+}
+
+}  // namespace
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, int causal, float scale, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, stream);
+}
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+                    void* stream) {
+  if (block_mask == nullptr) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_BF16) return check_shape(B, H, N, d, dtype) == ATTN_OK ? ATTN_ERR_UNSUPPORTED
+                                                                         : ATTN_ERR_INVALID;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, scale, dtype, block_mask, stream);
 }
 
 int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
@@ -178,9 +197,12 @@ int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B
                                      static_cast<cudaStream_t>(stream)));
 }
 
-int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+namespace {
+
+int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, void* dq,
                   void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
-                  int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+                  int dtype, void* workspace, size_t workspace_bytes, const uint8_t* bmask,
+                  void* stream) {
   if (!all_aligned({q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
@@ -210,7 +232,17 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
       g_fault.armed = 0;
     }
   }
-  return from_cuda(launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject, s));
+  return from_cuda(
+      launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject, bmask, s));
+}
+
+}  // namespace
+
+int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                  void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                  int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
+                       workspace_bytes, nullptr, stream);
 }
 
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
@@ -240,6 +272,26 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
   if (st != ATTN_OK) return st;
   st = attn_bwd_main(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
                      workspace_bytes, stream);
+  if (st != ATTN_OK) return st;
+  return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (block_mask == nullptr) return ATTN_ERR_INVALID;
+  if (!all_aligned({q, k, v, o, dout, lse, dq, dk, dv})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  st = attn_bwd_preprocess(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, stream);
+  if (st != ATTN_OK) return st;
+  st = bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
+                     workspace_bytes, block_mask, stream);
   if (st != ATTN_OK) return st;
   return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
 }

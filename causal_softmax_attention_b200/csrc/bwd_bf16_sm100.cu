@@ -63,7 +63,7 @@ using namespace sm100;
 // d <= 64, with dQ read out by them, measured slower (736 vs 791 TFLOP/s on
 // 8 heads of 32K tokens): that pass is bound by its MUFU and issue slots, not
 // by latency.
-template <int D>
+template <int D, bool kMask = false>
 struct Roles {
   static constexpr int EG = 2;                      // element-wise warpgroups
   static constexpr int QC = 128 / EG;               // query columns per element-wise group
@@ -79,8 +79,10 @@ struct Roles {
   // sub-partition (16K registers = 512 per lane), and the budgets draw on
   // the registers the block was launched with.
   static constexpr uint32_t R_E = 136;
-  static constexpr uint32_t R_DQ = 144;
-  static constexpr uint32_t R_CTL = 96;
+  // (the block-mask walk costs the control and dQ warps a few registers at
+  // d <= 64, where their loops are otherwise tightest)
+  static constexpr uint32_t R_DQ = (D == 128 || !kMask) ? 144 : 128;
+  static constexpr uint32_t R_CTL = (D == 128 || !kMask) ? 96 : 112;
   static_assert(EG * R_E + R_DQ + R_CTL <= WGS * LAUNCH_REGS,
                 "register split exceeds the launch budget");
   static constexpr int DQ_READERS = 128;            // arrivals on B_DQREAD
@@ -139,6 +141,7 @@ struct BwdParams {
   int N, Np, T, BH;
   int G;              // heads per scheduling group (see the CTA order in the kernel)
   int causal;
+  const uint8_t* bmask;  // [T][T] tile kinds (0 none, 1 all, 2 key <= query in the tile), or null
   float scale, scale_log2;
   uint64_t wait_cycles;
   int inject_fault;   // 1: never signal the first score tile (tests the timeout path)
@@ -205,14 +208,14 @@ __device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[QC], const fl
   }
 }
 
-template <int D>
+template <int D, bool kMask>
 __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     attn_bwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
                                const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   using L = BwdLayout<D>;
-  using R = Roles<D>;
+  using R = Roles<D, kMask>;
   constexpr int QC = R::QC;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = L::EXACT ? smem_raw
@@ -240,8 +243,26 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   const int jt = r / gs;
   const int bh = g0 + r % gs;
   const int j0 = jt * kTile;
-  const int i_begin = p.causal ? jt : 0;
-  const int n_iter = p.T - i_begin;
+  // The query tiles this key tile meets, in increasing order: i >= jt under
+  // the causal filter, all of them without it, or those a block mask marks.
+  // Every role walks them with next_tile, so all agree on tile k of the walk.
+  auto tile_kind = [&](int i) -> int {
+    if constexpr (kMask) {
+      return p.bmask[static_cast<size_t>(i) * p.T + jt];
+    } else {
+      return !p.causal ? 1 : (i > jt ? 1 : (i == jt ? 2 : 0));
+    }
+  };
+  auto next_tile = [&](int i) -> int {  // first tile after i that takes part (T if none)
+    if constexpr (kMask) {
+      for (++i; i < p.T && p.bmask[static_cast<size_t>(i) * p.T + jt] == 0; ++i) {
+      }
+      return i;
+    } else {
+      return p.causal ? max(i + 1, jt) : i + 1;
+    }
+  };
+  const int i_first = next_tile(-1);
 
   // Swizzled operands need a 1024-byte aligned window; nothing has been
   // issued yet, so a misaligned window is reported and every thread returns.
@@ -303,12 +324,12 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       }
       bool ok = true;
       int issued = 0;
-      for (int it = 0; it < n_iter; ++it) {
+      for (int it = 0, i = i_first; i < p.T; ++it, i = next_tile(i)) {
         const int s = it & 1;
         if (it >= 2 &&
             !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
           break;
-        const int i0 = (i_begin + it) * kTile;
+        const int i0 = i * kTile;
         uint64_t* bar = &bars[B_QFULL + s];
         mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
         for (int c = 0; c < L::NCH; ++c) {
@@ -361,15 +382,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
         mma_commit(&bars[B_DPFULL]);
       };
-      bool ok = wait(B_KV, 0) && wait(B_QFULL, 0);
-      if (ok) {
+      bool ok = true;
+      if (i_first < p.T && (ok = wait(B_KV, 0) && wait(B_QFULL, 0))) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
-      for (int it = 0; ok && it < n_iter; ++it) {
+      for (int it = 0, i = i_first; ok && i < p.T; ++it, i = next_tile(i)) {
         const int s = it & 1;
-        const bool more = it + 1 < n_iter;
+        const bool more = next_tile(i) < p.T;
         // dV_j += P^T dO_i, P^T read from region A (K = 128 queries, 16 per step)
         if (!(ok = wait(B_PFULL, it & 1))) break;
         tc_fence_after();
@@ -438,8 +459,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
     };
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int i = i_begin + it;
+    for (int it = 0, i = i_first; i < p.T; ++it, i = next_tile(i)) {
       const int b = it % L::DQ_BUFS;
       if (!(ok = wait_w(B_DQFULL + b, (it / L::DQ_BUFS) & 1))) break;
       tc_fence_after();
@@ -480,14 +500,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag));
     };
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
+    int it = 0;
+    for (int i = i_first; i < p.T; ++it, i = next_tile(i)) {
       const int s = it & 1;
-      const int i = i_begin + it;
       if (!(ok = wait_w(B_QFULL + s, (it >> 1) & 1))) break;  // LSE_i, D_i in shared memory
       const float* lse_s = s_lse + s * 128;
       const float* d_s = s_dv + s * 128;
-      // queries with local index < thr are masked for this key row
-      const int thr = key >= p.N ? 128 : ((p.causal && i == jt) ? t : 0);
+      // queries with local index < thr are masked for this key row (kind 2:
+      // the key must not lie after the query inside the tile)
+      const int thr = key >= p.N ? 128 : (tile_kind(i) == 2 ? t : 0);
 
       // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e) -> bf16 into region A
       if (!(ok = wait_w(B_SFULL, it & 1))) break;
@@ -561,13 +582,19 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
       __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
       constexpr int W = R::E_CH >= 32 ? 32 : R::E_CH;
+      const bool any = it > 0;  // a key tile that meets no query tile has dK = dV = 0
 #pragma unroll 1
       for (int c = 0; c < R::E_CH / W; ++c) {
         const int ch = g * R::E_CH + W * c;
         uint32_t rv[W], rk[W];
-        tmem_ld<W>(lane_base + L::T_DV + ch, rv);
-        tmem_ld<W>(lane_base + L::T_DK + ch, rk);
-        tmem_ld_wait(rv, rk);
+        if (any) {
+          tmem_ld<W>(lane_base + L::T_DV + ch, rv);
+          tmem_ld<W>(lane_base + L::T_DK + ch, rk);
+          tmem_ld_wait(rv, rk);
+        } else {
+#pragma unroll
+          for (int u = 0; u < W; ++u) rv[u] = rk[u] = 0u;
+        }
 #pragma unroll
         for (int v = 0; v < W / 8 && key_ok; ++v) {
           uint4 ov, ok4;
@@ -600,20 +627,22 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 template <int D>
 cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, void* dv, int BH,
                               int N, bool causal, float scale, uint64_t wait_cycles, int inject,
-                              cudaStream_t s) {
+                              const uint8_t* bmask, cudaStream_t s) {
   using L = BwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
-  auto kern = attn_bwd_bf16_sm100_kernel<D>;
+  auto kern = bmask ? attn_bwd_bf16_sm100_kernel<D, true> : attn_bwd_bf16_sm100_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   // The setmaxnreg split redistributes exactly the registers the block is
   // launched with; with fewer at launch the increases could never be served.
-  static const cudaError_t regs_ok = [&]() {
-    cudaFuncAttributes fa;
-    const cudaError_t r = cudaFuncGetAttributes(&fa, kern);
-    if (r != cudaSuccess) return r;
-    return fa.numRegs == static_cast<int>(Roles<D>::LAUNCH_REGS) ? cudaSuccess
-                                                       : cudaErrorInvalidConfiguration;
+  static const cudaError_t regs_ok = []() {
+    for (auto k : {attn_bwd_bf16_sm100_kernel<D, false>, attn_bwd_bf16_sm100_kernel<D, true>}) {
+      cudaFuncAttributes fa;
+      const cudaError_t r = cudaFuncGetAttributes(&fa, k);
+      if (r != cudaSuccess) return r;
+      if (fa.numRegs != static_cast<int>(Roles<D>::LAUNCH_REGS)) return cudaErrorInvalidConfiguration;
+    }
+    return cudaSuccess;
   }();
   if (regs_ok != cudaSuccess) return regs_ok;
   BwdParams p;
@@ -636,6 +665,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   const size_t head_bytes = static_cast<size_t>(ws.Np) * D * 8;
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
+  p.bmask = bmask;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = wait_cycles;
@@ -649,17 +679,17 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
 
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
                             int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, cudaStream_t s) {
+                            int inject_fault, const uint8_t* block_mask, cudaStream_t s) {
   switch (d) {
     case 32:
       return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, s);
+                                   inject_fault, block_mask, s);
     case 64:
       return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, s);
+                                   inject_fault, block_mask, s);
     case 128:
       return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                    inject_fault, s);
+                                    inject_fault, block_mask, s);
     default:
       return cudaErrorInvalidValue;
   }

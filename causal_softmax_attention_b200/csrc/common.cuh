@@ -51,11 +51,14 @@ cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const
 struct TmaMaps {
   CUtensorMap a, b, c, d;
 };
+// block_mask: device [T][T] tile kinds (0 none, 1 all, 2 key <= query inside
+// the tile), T = ceil(N / 128), or null for the causal / full filter.
 cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
-                            int d, bool causal, float scale, cudaStream_t s);
+                            int d, bool causal, float scale, const uint8_t* block_mask,
+                            cudaStream_t s);
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
                             int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, cudaStream_t s);
+                            int inject_fault, const uint8_t* block_mask, cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 

@@ -89,6 +89,7 @@ struct FwdParams {
   int N, T, BH;
   int G;             // heads per scheduling group (see the CTA order)
   int causal;
+  const uint8_t* bmask;  // [T][T] tile kinds (0 none, 1 all, 2 key <= query in the tile), or null
   float scale_log2;
   uint64_t wait_cycles;
 };
@@ -108,7 +109,7 @@ __device__ __forceinline__ uint64_t fdesc_mnmajor(uint32_t tile, int kk) {
 // each softmax group packs its 64 keys into the first 32 of its own columns.
 __host__ __device__ constexpr uint32_t fp_col(int k) { return 64 * (k >> 6) + ((k & 63) >> 1); }
 
-template <int D>
+template <int D, bool kMask>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -134,7 +135,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int it_q = p.causal ? p.T - 1 - r / gs : r / gs;
   const int bh = g0 + r % gs;
   const int i0 = it_q * kTile;
-  const int n_kv = p.causal ? it_q + 1 : p.T;
+  // The key tiles this query tile meets, in increasing order: j <= i under
+  // the causal filter, all of them without it, or those a block mask marks.
+  // Every role walks them with next_tile, so all agree on tile k of the walk.
+  auto tile_kind = [&](int j) -> int {
+    if constexpr (kMask) {
+      return p.bmask[static_cast<size_t>(it_q) * p.T + j];
+    } else {
+      return !p.causal ? 1 : (j < it_q ? 1 : (j == it_q ? 2 : 0));
+    }
+  };
+  auto next_tile = [&](int j) -> int {  // first tile after j that takes part (T if none)
+    if constexpr (kMask) {
+      const uint8_t* row = p.bmask + static_cast<size_t>(it_q) * p.T;
+      for (++j; j < p.T && row[j] == 0; ++j) {
+      }
+      return j;
+    } else {
+      return (p.causal && j + 1 > it_q) ? p.T : j + 1;
+    }
+  };
+  const int j_first = next_tile(-1);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[F_Q], 1);
@@ -182,7 +203,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       bool ok = true;
       int issued = 0;
-      for (int jt = 0; jt < n_kv; ++jt) {
+      for (int jt = 0, j = j_first; j < p.T; ++jt, j = next_tile(j)) {
         const int s = jt & 1;
         // K_j is free once S_j has been computed, V_j once P_j V_j has.
         if (jt >= 2 &&
@@ -191,7 +212,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_arrive_expect_tx(&bars[full + s], L::TILE);
         for (int c = 0; c < L::NCH; ++c)
           tma_load_3d(smem + off + s * L::TILE + c * L::CHUNK, map, &bars[full + s], c * L::CH,
-                      jt * kTile, bh);
+                      j * kTile, bh);
         ++issued;
       }
       if (!ok) fail();
@@ -221,13 +242,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(&bars[F_SFULL + jt % 3]);
         mma_commit(&bars[F_KEMPTY + (jt & 1)]);
       };
-      bool ok = wait(F_Q, 0) && wait(F_KFULL, 0);
-      if (ok) {
+      bool ok = true;
+      if (j_first < p.T && (ok = wait(F_Q, 0) && wait(F_KFULL, 0))) {
         tc_fence_after();
         issue_s(0);
-        if (n_kv > 1 && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
+        if (next_tile(j_first) < p.T && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
       }
-      for (int jt = 0; ok && jt < n_kv; ++jt) {
+      for (int jt = 0, j = j_first; ok && j < p.T; ++jt, j = next_tile(j)) {
         if (!(ok = wait(F_PFULL, jt & 1))) break;
         if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
         tc_fence_after();
@@ -239,7 +260,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  (jt > 0 || kk > 0));
         mma_commit(&bars[F_PVDONE + (jt & 1)]);
         mma_commit(&bars[F_VEMPTY + (jt & 1)]);
-        if (jt + 2 < n_kv) {
+        if (next_tile(next_tile(j)) < p.T) {
           // S_{j+2} overwrites P_{j-1}, which P_{j-1} V_{j-1} reads
           if (jt >= 1 && !(ok = wait(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
           if (!(ok = wait(F_KFULL + (jt & 1), ((jt + 2) >> 1) & 1))) break;
@@ -264,11 +285,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     };
     float m = -INFINITY, z = 0.f;
     bool ok = true;
-    for (int jt = 0; jt < n_kv; ++jt) {
-      const int kb = jt * kTile + 64 * g;  // first key of this thread's 64 columns
-      // keys with local index >= lim are excluded for this row
+    int jt = 0;
+    for (int j = j_first; j < p.T; ++jt, j = next_tile(j)) {
+      const int kb = j * kTile + 64 * g;  // first key of this thread's 64 columns
+      // keys with local index >= lim are excluded for this row: keys past N,
+      // and in a kind-2 tile keys after the query inside the tile
       int lim = p.N - kb;
-      if (p.causal && qrow - kb + 1 < lim) lim = qrow - kb + 1;
+      if (tile_kind(j) == 2 && t - 64 * g + 1 < lim) lim = t - 64 * g + 1;
       const bool masked = __any_sync(0xffffffffu, lim < 64);
       if (!(ok = wait_w(F_SFULL + jt % 3, (jt / 3) & 1))) break;
       tc_fence_after();
@@ -335,9 +358,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[F_PFULL]);
     }
-    // Epilogue: the last P V has landed; combine the two halves' sums.
-    if (ok) ok = wait_w(F_PVDONE + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
-    if (ok) {
+    // Epilogue: the last P V has landed; combine the two halves' sums. A
+    // query tile that meets no key tile has O = 0 and LSE = -inf (the log of
+    // an empty sum).
+    const int n_kv = jt;
+    if (ok && n_kv > 0) ok = wait_w(F_PVDONE + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    if (ok && n_kv > 0) {
       float* xmz = xm + (n_kv & 1) * 256;
       xmz[g * 128 + t] = z;
       mbar_arrive(&bars[F_XCHG]);
@@ -348,15 +374,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       fail();
     } else {
       tc_fence_after();
-      const float inv = 1.f / z;
+      const float inv = z > 0.f ? 1.f / z : 0.f;
       const bool row_ok = qrow < p.N;
       __nv_bfloat16* orow =
           p.o + (static_cast<size_t>(bh) * p.N + (row_ok ? qrow : 0)) * D + g * L::HALF_D;
 #pragma unroll 1
       for (int c = 0; c < L::HALF_D; c += 16) {
         uint32_t ov[16];
-        tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
-        tmem_ld_wait(ov);
+        if (n_kv > 0) {
+          tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
+          tmem_ld_wait(ov);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) ov[u] = 0u;
+        }
         if (row_ok) {
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
@@ -370,7 +401,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       if (row_ok && g == 0)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(z)) * 0.6931471805599453f;
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] =
+            z > 0.f ? (m + __log2f(z)) * 0.6931471805599453f : -INFINITY;
     }
   }
   tc_fence_before();
@@ -383,10 +415,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 template <int D>
 cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int BH, int N,
-                         bool causal, float scale, cudaStream_t s) {
+                         bool causal, float scale, const uint8_t* bmask, cudaStream_t s) {
   using L = FwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
-  auto kern = attn_fwd_bf16_sm100_kernel<D>;
+  auto kern = bmask ? attn_fwd_bf16_sm100_kernel<D, true> : attn_fwd_bf16_sm100_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   FwdParams p;
@@ -405,6 +437,7 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
   const size_t head_bytes = static_cast<size_t>(p.T) * kTile * D * 4;
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
+  p.bmask = bmask;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = kWaitLimitCycles;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
@@ -415,11 +448,12 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
-                            int d, bool causal, float scale, cudaStream_t s) {
+                            int d, bool causal, float scale, const uint8_t* block_mask,
+                            cudaStream_t s) {
   switch (d) {
-    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, N, causal, scale, s);
-    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, N, causal, scale, s);
-    case 128: return launch_fwd_d<128>(maps, o, lse, status, BH, N, causal, scale, s);
+    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
+    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
+    case 128: return launch_fwd_d<128>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
     default: return cudaErrorInvalidValue;
   }
 }

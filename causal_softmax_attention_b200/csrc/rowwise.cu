@@ -56,7 +56,9 @@ __global__ void __launch_bounds__(256)
     for (int off = 1; off < G; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (active && sub == 0) {
       d_pad[r] = acc;
-      lse_pad[r] = i < N ? lse[static_cast<size_t>(bh) * N + i] * kLog2e : INFINITY;
+      // a row with no kept key (LSE = -inf) must give P = 0, like a padded row
+      const float l = i < N ? lse[static_cast<size_t>(bh) * N + i] : INFINITY;
+      lse_pad[r] = l == -INFINITY ? INFINITY : l * kLog2e;
     }
   }
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -85,7 +87,8 @@ __global__ void __launch_bounds__(256)
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
       d_pad[r] = acc;
-      lse_pad[r] = i < N ? lse[static_cast<size_t>(bh) * N + i] : INFINITY;
+      const float l = i < N ? lse[static_cast<size_t>(bh) * N + i] : INFINITY;
+      lse_pad[r] = l == -INFINITY ? INFINITY : l;
     }
   }
 }

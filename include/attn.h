@@ -97,6 +97,37 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              void* stream);
 
 /*
+ * Block-sparse attention: the causal / full filter replaced by a block mask
+ * over 128 x 128 tiles of (query, key) positions -- the generalisation of the
+ * mask that ddx PR #162 ("perf(ddx-ad): transpose causal attention's
+ * contractions without their joins", "What changed") applies as a filter on
+ * the grouping keys, and of its tile skipping. bf16 only.
+ *   block_mask : in, DEVICE [T][T] bytes, T = ceil(N / 128), row-major by
+ *                query tile: block_mask[a * T + b] describes query rows
+ *                [128a, 128a+128) against key columns [128b, 128b+128):
+ *                  0  no score of the tile takes part (the tile is skipped),
+ *                  1  every score takes part,
+ *                  2  a score takes part when its key's index inside the tile
+ *                     is at most its query's (the causal filter's diagonal
+ *                     tile; causal attention is 1 below the diagonal, 2 on
+ *                     it, 0 above). Other values act as 1.
+ *                Shared by every (batch, head). Read, not written; owned by
+ *                the caller and must stay valid until the kernels finish.
+ * Rows whose query keeps no score (a query tile with only 0 entries) get
+ * O = 0 and LSE = -inf (the log of an empty sum), and zero gradients; keys
+ * that no query keeps get dK = dV = 0.
+ * Other arguments, layouts, ownership and checks as attn_fwd / attn_bwd;
+ * block_mask == NULL -> ATTN_ERR_INVALID, dtype f32 -> ATTN_ERR_UNSUPPORTED.
+ */
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+                    void* stream);
+int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The three stages attn_bwd runs, exposed so a caller can time or overlap them
  * separately. Same arguments and checks as attn_bwd; they must be enqueued in
  * this order on one stream with the same workspace.

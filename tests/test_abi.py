@@ -119,3 +119,17 @@ def test_stage_entry_points_reject_bad_arguments():
     assert L.attn_bwd_dq_convert(A, 1, 1, 64, 40, 0.1, 1, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
     assert L.attn_last_status(None) == csa.ATTN_ERR_INVALID
     assert L.attn_test_arm_timeout(0) == csa.ATTN_ERR_INVALID
+
+
+def test_masked_entry_points_reject_bad_arguments():
+    # every call returns during argument checking (no CUDA call)
+    f, b = L.attn_fwd_masked, L.attn_bwd_masked
+    assert f(A, A, A, A, A, 1, 1, 300, 64, None, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 300, 64, A, 0.125, 0, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(A, A, A, A, A + 4, 1, 1, 300, 64, A, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 300, 96, A, 0.125, 1, None) == csa.ATTN_ERR_UNSUPPORTED
+    args = [A] * 9 + [1, 1, 300, 64]
+    assert b(*args, None, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+    assert b(*args, A, 0.125, 0, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert b(*args, A, math.nan, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+    assert b(*args, A, 0.125, 1, A, 16, None) == csa.ATTN_ERR_INVALID

@@ -144,6 +144,76 @@ def test_running_max_raised_every_key_tile(csa, d):
     assert np.abs(as_f64(gr["LSE"].cpu()) - ref["LSE"]).max() <= 1e-3 * max(1.0, np.abs(ref["LSE"]).max())
 
 
+def run_masked(csa, q, k, v, do, bm, scale):
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
+    B, H, N, d = q.shape
+    mask = torch.tensor(bm, dtype=torch.uint8, device=dev).contiguous()
+    o = torch.empty_like(qd)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    csa.attn_fwd_masked(qd, kd, vd, o, lse, mask, scale)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    csa.attn_bwd_masked(qd, kd, vd, o, dod, lse, dq, dk, dv, mask, csa.new_workspace(qd), scale)
+    torch.cuda.synchronize()
+    assert csa.attn_fwd_last_status() == 0
+    return {"O": o, "LSE": lse, "dQ": dq, "dK": dk, "dV": dv}
+
+
+def compare_masked(csa, B, H, N, d, bm, seed):
+    q, k, v, do = draw(B, H, N, d, seed, "bf16")
+    scale = d ** -0.5
+    g = run_masked(csa, q, k, v, do, bm, scale)
+    keep = oracle.block_mask_keep(bm, N)
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), scale, keep=keep)
+    gscale = max(np.abs(ref[n]).max() for n in ("dQ", "dK", "dV"))
+    for name in ("O", "dQ", "dK", "dV"):
+        e = rel(as_f64(g[name].cpu()), ref[name], gscale if name != "O" else None)
+        assert e <= TOL["bf16"], (name, e)
+    lse = as_f64(g["LSE"].cpu())
+    empty = np.isneginf(ref["LSE"])
+    assert np.array_equal(np.isneginf(lse), empty)
+    assert np.abs(lse[~empty] - ref["LSE"][~empty]).max() <= 1e-3
+    return g, ref
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_parity(csa, d):
+    # kinds 0 / 1 / 2 anywhere, an empty query tile (O = 0, LSE = -inf), a
+    # key tile no query meets (dK = dV = 0), kind 2 off the diagonal
+    N = 5 * 128 + 23
+    bm = np.random.default_rng(d).integers(0, 3, (6, 6))
+    bm[2, :] = 0
+    bm[:, 4] = 0
+    bm[5, 1] = 2
+    g, ref = compare_masked(csa, 1, 2, N, d, bm, 300 + d)
+    assert torch.all(g["O"][:, :, 256:384] == 0)
+    assert torch.all(g["dQ"][:, :, 256:384] == 0)
+    assert torch.all(g["dK"][:, :, 512:640] == 0) and torch.all(g["dV"][:, :, 512:640] == 0)
+
+
+def test_block_sparse_sliding_window(csa):
+    # local attention: each query tile sees its own tile (causally) and the
+    # two before it
+    N, w = 8 * 128, 2
+    t = np.arange(8)
+    bm = np.where(t[:, None] == t[None, :], 2,
+                  np.where((t[None, :] < t[:, None]) & (t[None, :] >= t[:, None] - w), 1, 0))
+    compare_masked(csa, 2, 2, N, 64, bm, 321)
+
+
+def test_causal_block_mask_matches_the_causal_path(csa):
+    B, H, N, d = 1, 3, 3 * 128 + 50, 128
+    q, k, v, do = draw(B, H, N, d, 333, "bf16")
+    t = np.arange(-(-N // 128))
+    bm = np.where(t[:, None] > t[None, :], 1, np.where(t[:, None] == t[None, :], 2, 0))
+    gm = run_masked(csa, q, k, v, do, bm, d ** -0.5)
+    gc = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    for name in ("O", "LSE", "dK", "dV"):
+        assert torch.equal(gm[name], gc[name]), name
+    ref = as_f64(gc["dQ"].cpu())
+    assert rel(as_f64(gm["dQ"].cpu()), ref, np.abs(ref).max()) <= 1e-2
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
