@@ -14,6 +14,12 @@ all ranks' FLOPs / max-over-ranks device time.
 
 `--impl reference` times the float64 CPU oracle instead (rank 0 only), on a
 bounded sample of the same workload per step.
+
+`--block-mask SPEC` (causal, full, window:W, random:P:SEED over 128 x 128
+tiles; bf16) times the block-sparse backward instead: the same three stages
+with the masked main kernel, FLOPs counted over the kept tiles (a kind-1 tile
+as 128 x 128 score pairs, a kind-2 tile as half), so the causal mask gives
+the causal count.
 """
 from __future__ import annotations
 
@@ -34,7 +40,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from seeded_inputs import CONFIGS, draw  # noqa: E402
+from seeded_inputs import CONFIGS, block_mask, block_mask_pairs, draw  # noqa: E402
 
 METRIC = "causal attention backward TFLOP/s (bf16, 1×B200) and % of dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -200,6 +206,29 @@ def oracle_sample(cfg, budget_s: float, rows_per_block: int = 256):
     return flops / elapsed / 1e12, desc, elapsed
 
 
+def oracle_sample_masked(cfg, spec: str, budget_s: float, n_sample: int = 2048):
+    """Time the float64 oracle's block-masked backward on whole heads of
+    n_sample tokens with the same mask recipe until `budget_s` seconds of CPU
+    work; FLOPs counted over the kept tiles, as on the GPU."""
+    import oracle
+    from seeded_inputs import as_f64
+    n = min(cfg.N, n_sample)
+    bm = block_mask(spec, n)
+    keep = oracle.block_mask_keep(bm, n)
+    q, k, v, do = draw(1, 1, n, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)
+    qh, kh, vh, doh = (as_f64(t[0, 0]) for t in (q, k, v, do))
+    flops, elapsed, heads = 0.0, 0.0, 0
+    while elapsed < budget_s:
+        t0 = time.perf_counter()
+        oracle.backward_head(qh, kh, vh, doh, cfg.scale, keep=keep)
+        elapsed += time.perf_counter() - t0
+        flops += 10.0 * cfg.d * block_mask_pairs(bm)
+        heads += 1
+    desc = (f"oracle backward_head (numpy float64, materialised {n}x{n}) with block mask {spec} "
+            f"on {heads} heads of {n} tokens, d={cfg.d}, in {elapsed:.1f} s")
+    return flops / elapsed / 1e12, desc, elapsed
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -215,11 +244,16 @@ def run_reference(args, cfg, world, rank):
     if rank != 0:
         return
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    def sample(b):
+        if args.block_mask:
+            return oracle_sample_masked(cfg, args.block_mask, b)
+        return oracle_sample(cfg, b)
+
     for _ in range(args.warmup):
-        oracle_sample(cfg, budget / 4)
+        sample(budget / 4)
     vals, descs, times = [], [], []
     for _ in range(args.steps):
-        v, d, t = oracle_sample(cfg, budget)
+        v, d, t = sample(budget)
         vals.append(v)
         descs.append(d)
         times.append(t)
@@ -230,7 +264,7 @@ def run_reference(args, cfg, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(cfg, args.gpus),
+        "config": config_dict(cfg, args.gpus, args.block_mask),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": descs[-1]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -239,17 +273,23 @@ def run_reference(args, cfg, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(cfg, n_gpus):
-    return {"workload": f"{cfg.name}: causal attention backward B={cfg.B} H={cfg.H} "
+def config_dict(cfg, n_gpus, mask_spec=None):
+    kind = "causal" if mask_spec is None else f"block-sparse ({mask_spec} over 128x128 tiles)"
+    out = {"workload": f"{cfg.name}: {kind} attention backward B={cfg.B} H={cfg.H} "
                         f"N={cfg.N} d={cfg.d} {cfg.dtype}, q,k,v,dO ~ N(0,1)"
                         + (f" (q,k x{cfg.qk_gain})" if cfg.qk_gain != 1.0 else "")
                         + f", seed {cfg.seed}, scale 1/sqrt(d)",
-            "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "causal": True,
+            "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "causal": mask_spec is None,
             "global_batch": cfg.B * n_gpus, "seq_len": cfg.N,
             "parallelism": f"independent replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
             "l2": "inputs larger than L2 (no flush needed)"
             if 5 * cfg.B * cfg.H * cfg.N * cfg.d * 2 > 126e6
             else "L2 flushed (256 MB write) between steps, outside the steps' events"}
+    if mask_spec is not None:
+        bm = block_mask(mask_spec, cfg.N)
+        out["block_mask"] = mask_spec
+        out["kept_fraction_of_causal"] = block_mask_pairs(bm) / (cfg.N * cfg.N / 2)
+    return out
 
 
 # --------------------------------------------------------------------- GPU arm
@@ -261,7 +301,18 @@ def run_gpu(args, cfg, world, rank, local):
     B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
     q, k, v, do = draw(B, H, N, d, cfg.seed + 1000 * rank, cfg.dtype, cfg.qk_gain)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o, lse = csa.forward(qd, kd, vd, True, cfg.scale)
+    mask = None
+    if args.block_mask:
+        bm = block_mask(args.block_mask, N)
+        mask = torch.from_numpy(bm).to(dev)
+        flops = 10.0 * d * block_mask_pairs(bm) * B * H
+        fwd_flops = 0.4 * flops
+        o = torch.empty_like(qd)
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+        csa.attn_fwd_masked(qd, kd, vd, o, lse, mask, cfg.scale)
+    else:
+        flops, fwd_flops = cfg.bwd_flops, cfg.fwd_flops
+        o, lse = csa.forward(qd, kd, vd, True, cfg.scale)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     ws = csa.new_workspace(qd)
     stream = torch.cuda.current_stream(dev)
@@ -272,7 +323,10 @@ def run_gpu(args, cfg, world, rank, local):
         csa.attn_bwd_preprocess(o, dod, lse, ws, stream)
         if ev_main is not None:
             ev_main[0].record(stream)
-        csa.attn_bwd_main(qd, kd, vd, dod, dq, dk, dv, ws, True, cfg.scale, stream)
+        if mask is None:
+            csa.attn_bwd_main(qd, kd, vd, dod, dq, dk, dv, ws, True, cfg.scale, stream)
+        else:
+            csa.attn_bwd_main_masked(qd, kd, vd, dod, dq, dk, dv, mask, ws, cfg.scale, stream)
         if ev_main is not None:
             ev_main[1].record(stream)
         csa.attn_bwd_dq_convert(dq, ws, cfg.scale, stream)
@@ -316,7 +370,6 @@ def run_gpu(args, cfg, world, rank, local):
         total_ms = sum(step_ms)
     status = csa.attn_last_status(ws)
     ms_per_step = max_over_ranks(total_ms / args.steps, world)
-    flops = cfg.bwd_flops
     value = whole_job_tflops(flops, world, ms_per_step)
 
     # ---- e2e through the public API with pinned host buffers
@@ -337,7 +390,7 @@ def run_gpu(args, cfg, world, rank, local):
 
     def e2e_step():
         csa.backward_host(hq, hk, hv, ho, hdo, hlse, hdq, hdk, hdv, dev_bufs, True, cfg.scale,
-                          e2e_chunks, stream)
+                          e2e_chunks, stream, block_mask=mask)
 
     e2e_steps = max(1, min(args.steps, 5))
     for _ in range(2):
@@ -356,12 +409,19 @@ def run_gpu(args, cfg, world, rank, local):
     # ---- the forward that produces O and LSE (not part of the timed step):
     # its own CUDA-event time on the same stream, same inputs, outputs reused.
     fwd_iters = 5
+
+    def fwd():
+        if mask is None:
+            csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
+        else:
+            csa.attn_fwd_masked(qd, kd, vd, o, lse, mask, cfg.scale, stream)
+
     for _ in range(2):
-        csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
+        fwd()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(fwd_iters):
-        csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
+        fwd()
     f1.record(stream)
     torch.cuda.synchronize()
     fwd_ms = max_over_ranks(f0.elapsed_time(f1) / fwd_iters, world)
@@ -372,7 +432,7 @@ def run_gpu(args, cfg, world, rank, local):
     main_avg = statistics.mean(main_ms)
     achieved = flops / (main_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = dram_traffic_per_launch(cfg)
+    traffic = dram_traffic_per_launch(cfg) if mask is None else None
     clk = clocks.summary(host_t0, host_t1)
     if cfg.dtype == "bf16":
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -393,7 +453,7 @@ def run_gpu(args, cfg, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-        "data": "synthetic", "config": config_dict(cfg, world),
+        "data": "synthetic", "config": config_dict(cfg, world, args.block_mask),
         "pct_of_dense_bf16_peak": 100.0 * value / world / peak,
         "roofline": roofline,
         "stage_ms": {"step_median": statistics.median(step_ms), "main_median": statistics.median(main_ms),
@@ -404,9 +464,10 @@ def run_gpu(args, cfg, world, rank, local):
                         "H2D / attn_bwd / D2H overlapped on three streams"},
         "forward": {"kernel": "attn_fwd_bf16_sm100_kernel" if cfg.dtype == "bf16"
                     else "fwd_f32_kernel", "ms": fwd_ms,
-                    "tflops": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12,
-                    "frac": cfg.fwd_flops / (fwd_ms * 1e-3) / 1e12 / roofline["peak"],
-                    "flops_convention": "causal forward 4*B*H*N^2*d/2",
+                    "tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
+                    "frac": fwd_flops / (fwd_ms * 1e-3) / 1e12 / roofline["peak"],
+                    "flops_convention": "causal forward 4*B*H*N^2*d/2" if mask is None
+                    else "4*d per kept score pair (kind-2 tiles count half)",
                     "note": "measured outside the timed backward step"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
@@ -414,7 +475,10 @@ def run_gpu(args, cfg, world, rank, local):
         "peak_memory_bytes": torch.cuda.max_memory_allocated(dev),
     }
     if world == 1 and not args.no_cpu_baseline:
-        v_cpu, desc, _ = oracle_sample(cfg, args.cpu_seconds)
+        if mask is None:
+            v_cpu, desc, _ = oracle_sample(cfg, args.cpu_seconds)
+        else:
+            v_cpu, desc, _ = oracle_sample_masked(cfg, args.block_mask, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": blas_threads(),
                                 "kind": "oracle", "sample": desc}
     print(json.dumps(line), flush=True)
@@ -431,10 +495,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head groups of the end-to-end (host-buffer) measurement")
+    ap.add_argument("--block-mask", default=None, metavar="SPEC",
+                    help="time the block-sparse backward: causal, full, window:W or "
+                         "random:P:SEED over 128x128 tiles (bf16 configs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = CONFIGS[args.config]
+    if args.block_mask:
+        if cfg.dtype != "bf16":
+            ap.error("--block-mask needs a bf16 config")
+        block_mask(args.block_mask, 128)  # rejects a malformed spec before any GPU work
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, cfg, world, rank)

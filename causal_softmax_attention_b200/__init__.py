@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "attn_bwd_noalloc": (i, [vp] * 9 + [i, i, i, i, i, f, i, vp]),
         "attn_fwd_masked": (i, [vp] * 5 + [i, i, i, i, vp, f, i, vp]),
         "attn_bwd_masked": (i, [vp] * 9 + [i, i, i, i, vp, f, i, vp, sz, vp]),
+        "attn_bwd_main_masked": (i, [vp] * 7 + [i, i, i, i, vp, f, i, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -67,7 +68,7 @@ _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
             "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc", "attn_fwd_masked",
-            "attn_bwd_masked")
+            "attn_bwd_masked", "attn_bwd_main_masked")
 
 
 def library() -> ctypes.CDLL:
@@ -156,6 +157,20 @@ def attn_bwd_main(q, k, v, dout, dq, dk, dv, workspace, causal: bool = True,
     return st
 
 
+def attn_bwd_main_masked(q, k, v, dout, dq, dk, dv, block_mask, workspace,
+                         scale: float | None = None, stream=None) -> int:
+    """The main stage of attn_bwd_masked (between attn_bwd_preprocess and
+    attn_bwd_dq_convert); `block_mask` as in attn_fwd_masked."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_bwd_main_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, H, N, d, _ptr(block_mask), float(scale),
+                                   _DTYPES[q.dtype], _ptr(workspace), int(workspace.numel()),
+                                   _stream(stream))
+    _check(st, "attn_bwd_main_masked")
+    return st
+
+
 def attn_bwd_dq_convert(dq, workspace, scale: float | None = None, stream=None) -> int:
     B, H, N, d = _shape(dq)
     scale = d ** -0.5 if scale is None else scale
@@ -205,7 +220,7 @@ def backward(q, k, v, o, dout, lse, causal: bool = True, scale: float | None = N
 
 
 def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool = True,
-                  scale: float | None = None, chunks: int = 8, stream=None):
+                  scale: float | None = None, chunks: int = 8, stream=None, block_mask=None):
     """dQ, dK, dV of inputs held in (pinned) HOST memory, results written to
     host tensors, through attn_bwd with the transfers overlapped.
 
@@ -220,7 +235,9 @@ def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool 
     attn_bwd_workspace_bytes for one group (chunk_workspace_bytes). The work
     starts after everything already queued on `stream` (default: the current
     stream) and `stream` waits for all of it to finish, so events recorded
-    on `stream` around the call time the whole transfer and compute.
+    on `stream` around the call time the whole transfer and compute. With a
+    `block_mask` (a device uint8 [T, T] tensor, as in attn_bwd_masked) each
+    group runs attn_bwd_masked instead and `causal` is ignored.
     """
     B, H, N, d = _shape(hq)
     BH = B * H
@@ -250,8 +267,13 @@ def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool 
             landed.record(s_in)
         s_run.wait_event(landed)
         view = {n: rows(dev[n])[c0:c1].unsqueeze(0) for n in names + ("dq", "dk", "dv")}
-        attn_bwd(view["q"], view["k"], view["v"], view["o"], view["dout"], view["lse"],
-                 view["dq"], view["dk"], view["dv"], dev["workspace"], causal, scale, s_run)
+        if block_mask is None:
+            attn_bwd(view["q"], view["k"], view["v"], view["o"], view["dout"], view["lse"],
+                     view["dq"], view["dk"], view["dv"], dev["workspace"], causal, scale, s_run)
+        else:
+            attn_bwd_masked(view["q"], view["k"], view["v"], view["o"], view["dout"], view["lse"],
+                            view["dq"], view["dk"], view["dv"], block_mask, dev["workspace"],
+                            scale, s_run)
         ready = torch.cuda.Event()
         ready.record(s_run)
         s_out.wait_event(ready)

@@ -245,6 +245,18 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
                        workspace_bytes, nullptr, stream);
 }
 
+int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                         void* dk, void* dv, int B, int H, int N, int d,
+                         const unsigned char* block_mask, float scale, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (block_mask == nullptr || !all_aligned({q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
+  const int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
+                       workspace_bytes, block_mask, stream);
+}
+
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!all_aligned({dq})) return ATTN_ERR_INVALID;
@@ -290,8 +302,8 @@ int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
   if ((st = check_device_sm100()) != ATTN_OK) return st;
   st = attn_bwd_preprocess(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, stream);
   if (st != ATTN_OK) return st;
-  st = bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
-                     workspace_bytes, block_mask, stream);
+  st = attn_bwd_main_masked(q, k, v, dout, dq, dk, dv, B, H, N, d, block_mask, scale, dtype,
+                            workspace, workspace_bytes, stream);
   if (st != ATTN_OK) return st;
   return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
 }

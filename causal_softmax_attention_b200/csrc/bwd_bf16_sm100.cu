@@ -49,6 +49,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tile_walk.cuh"
 
 namespace csa {
 namespace {
@@ -109,7 +110,12 @@ struct BwdLayout {
   static constexpr int DV_OFF = LSE_OFF + STAGES * 512;   // [STAGES][128] f32
   static constexpr int BAR_OFF = DV_OFF + STAGES * 512;
   static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
-  static constexpr int BYTES = MISC_OFF + 64;
+  // block-mask bitmaps of the key tile's column (active tiles, kind-2 tiles):
+  // 80 words fill what d = 128 leaves of the window (T <= 2,560 tiles); a
+  // longer column is walked in global memory instead
+  static constexpr int MASK_WORDS = D == 128 ? 80 : 2048;
+  static constexpr int MASK_OFF = MISC_OFF + 64;
+  static constexpr int BYTES = MASK_OFF + 2 * 4 * MASK_WORDS;
   // d = 128 fills the 227 KB window, so the window itself must be 1024-byte
   // aligned (checked at run time); smaller d keep 1 KB of alignment slack and
   // at least ~118 KB so that one CTA owns an SM's tensor memory.
@@ -246,8 +252,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   // The query tiles this key tile meets, in increasing order: i >= jt under
   // the causal filter, all of them without it, or those a block mask marks.
   // Every role walks them with next_tile, so all agree on tile k of the walk.
+  // A block mask's column is read into shared-memory bitmaps once (below)
+  // when it fits, else walked byte by byte in global memory.
+  uint32_t* s_act = reinterpret_cast<uint32_t*>(smem + L::MASK_OFF);
+  uint32_t* s_kind2 = s_act + L::MASK_WORDS;
+  const bool mask_bits =
+      kMask && (p.T + R::THREADS - 1) / R::THREADS * (R::THREADS / 32) <= L::MASK_WORDS;
   auto tile_kind = [&](int i) -> int {
     if constexpr (kMask) {
+      if (mask_bits) return bit_set(s_kind2, i) ? 2 : 1;
       return p.bmask[static_cast<size_t>(i) * p.T + jt];
     } else {
       return !p.causal ? 1 : (i > jt ? 1 : (i == jt ? 2 : 0));
@@ -255,6 +268,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   };
   auto next_tile = [&](int i) -> int {  // first tile after i that takes part (T if none)
     if constexpr (kMask) {
+      if (mask_bits) return next_set_bit(s_act, p.T, i);
       for (++i; i < p.T && p.bmask[static_cast<size_t>(i) * p.T + jt] == 0; ++i) {
       }
       return i;
@@ -262,7 +276,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       return p.causal ? max(i + 1, jt) : i + 1;
     }
   };
-  const int i_first = next_tile(-1);
+  int i_first = kMask ? p.T : next_tile(-1);
 
   // Swizzled operands need a 1024-byte aligned window; nothing has been
   // issued yet, so a misaligned window is reported and every thread returns.
@@ -295,10 +309,14 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     tmem_alloc(tmem_base_slot, L::T_COLS);
     tmem_relinquish();
   }
+  if constexpr (kMask) {
+    if (mask_bits) build_tile_bits<R::THREADS>(p.bmask + jt, p.T, p.T, s_act, s_kind2);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
+  if constexpr (kMask) i_first = next_tile(-1);  // the bitmaps are in place now
 
   auto fail = [&]() {
     *abort_flag = 1;

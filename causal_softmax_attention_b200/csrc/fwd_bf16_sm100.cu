@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tile_walk.cuh"
 
 namespace csa {
 
@@ -67,7 +68,11 @@ struct FwdLayout {
   static constexpr int XM_OFF = V_OFF + 2 * TILE;   // [2][2][128] f32: row maxima / sums exchanged
   static constexpr int BAR_OFF = XM_OFF + 2048;
   static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
-  static constexpr int BYTES = MISC_OFF + 64;
+  // block-mask bitmaps of the query tile's row (active tiles, kind-2 tiles),
+  // T <= 65,280 tiles; a longer row is walked in global memory instead
+  static constexpr int MASK_WORDS = 2040;
+  static constexpr int MASK_OFF = MISC_OFF + 64;
+  static constexpr int BYTES = MASK_OFF + 2 * 4 * MASK_WORDS;
   static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
   static constexpr int SBUF = 3;                    // S buffers in TMEM
   static constexpr uint32_t T_S = 0, T_O = 128 * SBUF;
@@ -132,30 +137,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int g0 = (blockIdx.x / per_group) * p.G;
   const int r = blockIdx.x % per_group;
   const int gs = min(p.G, p.BH - g0);
-  const int it_q = p.causal ? p.T - 1 - r / gs : r / gs;
+  // (a block mask is taken to be causal-like: later query tiles first too)
+  const int it_q = (p.causal || kMask) ? p.T - 1 - r / gs : r / gs;
   const int bh = g0 + r % gs;
   const int i0 = it_q * kTile;
   // The key tiles this query tile meets, in increasing order: j <= i under
   // the causal filter, all of them without it, or those a block mask marks.
   // Every role walks them with next_tile, so all agree on tile k of the walk.
+  // A block mask's row is read into shared-memory bitmaps once (below) when
+  // it fits, else walked byte by byte in global memory.
+  uint32_t* s_act = reinterpret_cast<uint32_t*>(smem + L::MASK_OFF);
+  uint32_t* s_kind2 = s_act + L::MASK_WORDS;
+  const uint8_t* mask_row = kMask ? p.bmask + static_cast<size_t>(it_q) * p.T : nullptr;
+  const bool mask_bits =
+      kMask && (p.T + kFwdThreads - 1) / kFwdThreads * (kFwdThreads / 32) <= L::MASK_WORDS;
   auto tile_kind = [&](int j) -> int {
     if constexpr (kMask) {
-      return p.bmask[static_cast<size_t>(it_q) * p.T + j];
+      if (mask_bits) return bit_set(s_kind2, j) ? 2 : 1;
+      return mask_row[j];
     } else {
       return !p.causal ? 1 : (j < it_q ? 1 : (j == it_q ? 2 : 0));
     }
   };
   auto next_tile = [&](int j) -> int {  // first tile after j that takes part (T if none)
     if constexpr (kMask) {
-      const uint8_t* row = p.bmask + static_cast<size_t>(it_q) * p.T;
-      for (++j; j < p.T && row[j] == 0; ++j) {
+      if (mask_bits) return next_set_bit(s_act, p.T, j);
+      for (++j; j < p.T && mask_row[j] == 0; ++j) {
       }
       return j;
     } else {
       return (p.causal && j + 1 > it_q) ? p.T : j + 1;
     }
   };
-  const int j_first = next_tile(-1);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[F_Q], 1);
@@ -178,10 +191,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tmem_alloc(tmem_base_slot, L::T_COLS);
     tmem_relinquish();
   }
+  if constexpr (kMask) {
+    if (mask_bits) build_tile_bits<kFwdThreads>(mask_row, 1, p.T, s_act, s_kind2);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
+  const int j_first = next_tile(-1);
   auto fail = [&]() {
     *abort_flag = 1;
     atomicExch(p.status, kStatusTimeout);

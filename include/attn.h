@@ -137,6 +137,8 @@ int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
  *                partial sums). For f32 it also writes dq.
  *   dq_convert : dq = scale * accumulator, rounded to bf16 (bf16 only; a
  *                no-op returning ATTN_OK for f32)
+ *   main_masked: the main stage of attn_bwd_masked (block_mask as there; bf16
+ *                only), between the same preprocess and dq_convert
  */
 int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
                         int d, int dtype, void* workspace, size_t workspace_bytes, void* stream);
@@ -145,6 +147,10 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
                   int dtype, void* workspace, size_t workspace_bytes, void* stream);
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
+int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                         void* dk, void* dv, int B, int H, int N, int d,
+                         const unsigned char* block_mask, float scale, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /*
  * Reads the backward's device status word from `workspace` (synchronises the

@@ -102,3 +102,50 @@ def ddx_issue217_input(S: int = 3, T: int = 8, H: int = 2, C: int = 4):
         x = np.sin(n * 0.37 + phase).reshape(S, T, H, C)
         outs.append(np.ascontiguousarray(x.transpose(0, 2, 1, 3)))
     return tuple(outs)
+
+
+# ----------------------------------------------------------------- block masks
+# Tile kinds of a block mask over 128 x 128 tiles: 0 the tile takes no part,
+# 1 every score of the tile takes part, 2 a score takes part when its key's
+# index inside the tile is at most its query's.
+TILE = 128
+
+
+def block_mask(spec: str, N: int) -> np.ndarray:
+    """A [T, T] uint8 block mask (T = ceil(N / 128)) named by `spec`:
+
+    * ``causal``: kind 2 on the diagonal, 1 below it (the causal mask, tile by tile);
+    * ``full``: every tile kind 1;
+    * ``window:W``: local causal attention over W tiles: query tile i sees key
+      tiles i-W+1 .. i-1 in full and its own tile causally;
+    * ``random:P:SEED``: the causal mask with each below-diagonal tile kept
+      with probability P (seeded numpy draw), the diagonal always kept.
+    """
+    T = -(-N // TILE)
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    name, *rest = spec.split(":")
+    if name == "causal":
+        m = np.where(j < i, 1, np.where(j == i, 2, 0))
+    elif name == "full":
+        m = np.ones((T, T), dtype=np.int64)
+    elif name == "window":
+        w = int(rest[0])
+        if w < 1:
+            raise ValueError("window needs W >= 1")
+        m = np.where(j == i, 2, np.where((j < i) & (j > i - w), 1, 0))
+    elif name == "random":
+        p, seed = float(rest[0]), int(rest[1]) if len(rest) > 1 else 0
+        keep = np.random.default_rng(seed).random((T, T)) < p
+        m = np.where(j == i, 2, np.where((j < i) & keep, 1, 0))
+    else:
+        raise ValueError(f"unknown block mask {spec!r}")
+    return np.ascontiguousarray(m.astype(np.uint8))
+
+
+def block_mask_pairs(mask: np.ndarray) -> float:
+    """Score pairs a block mask keeps, counted the causal way: a kind-1 tile
+    as 128 * 128 pairs, a kind-2 tile as half of that (so the causal mask of
+    N = 128 T positions counts N^2 / 2)."""
+    m = np.asarray(mask)
+    return float(TILE * TILE * (np.count_nonzero(m == 1) + 0.5 * np.count_nonzero(m == 2)))

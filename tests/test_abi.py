@@ -133,3 +133,10 @@ def test_masked_entry_points_reject_bad_arguments():
     assert b(*args, A, 0.125, 0, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
     assert b(*args, A, math.nan, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
     assert b(*args, A, 0.125, 1, A, 16, None) == csa.ATTN_ERR_INVALID
+    m = L.attn_bwd_main_masked
+    args = [A] * 7 + [1, 1, 300, 64]
+    assert m(*args, None, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+    assert m(*args, A, 0.125, 0, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert m(*args, A, math.nan, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+    assert m(*args, A, 0.125, 1, A, 16, None) == csa.ATTN_ERR_INVALID
+    assert m(*([A] * 6 + [A + 8, 1, 1, 300, 64]), A, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from seeded_inputs import CONFIGS, as_f64, draw
+from seeded_inputs import CONFIGS, as_f64, block_mask, draw
 
 pytestmark = pytest.mark.gpu
 
@@ -212,6 +212,56 @@ def test_causal_block_mask_matches_the_causal_path(csa):
         assert torch.equal(gm[name], gc[name]), name
     ref = as_f64(gc["dQ"].cpu())
     assert rel(as_f64(gm["dQ"].cpu()), ref, np.abs(ref).max()) <= 1e-2
+
+
+def test_block_mask_longer_than_the_shared_bitmaps(csa):
+    # d = 128 keeps a key tile's column in shared memory only up to 2,560
+    # tiles; past that the kernels walk the mask in global memory. Under a
+    # two-tile window, query tile t sees key tiles t-1 and t, so the three
+    # tiles t-1 .. t+1 hold every score that O, LSE, dQ of query tile t and
+    # dK, dV of key tile t depend on: the oracle runs on those 384 positions.
+    B, H, d = 1, 1, 128
+    T = 2600
+    N = T * 128 - 77
+    q, k, v, do = draw(B, H, N, d, 351, "bf16")
+    bm = block_mask("window:2", N)
+    g = run_masked(csa, q, k, v, do, bm, d ** -0.5)
+    local_bm = block_mask("window:2", 3 * 128)
+    for t in (1, 1300, T - 2):
+        lo, hi = 128 * (t - 1), min(N, 128 * (t + 2))
+        sl = [as_f64(x[0, 0, lo:hi]) for x in (q, k, v, do)]
+        keep = oracle.block_mask_keep(local_bm[: -(-(hi - lo) // 128), : -(-(hi - lo) // 128)], hi - lo)
+        ref = oracle.backward(*(x[None, None] for x in sl), d ** -0.5, keep=keep)
+        a, b = 128, min(256, hi - lo)
+        gscale = max(np.abs(ref[n][0, 0, a:b]).max() for n in ("dQ", "dK", "dV"))
+        for name in ("O", "dQ", "dK", "dV"):
+            got = as_f64(g[name][0, 0, lo + a:lo + b].cpu())
+            e = rel(got, ref[name][0, 0, a:b], gscale if name != "O" else None)
+            assert e <= TOL["bf16"], (t, name, e)
+        lse = as_f64(g["LSE"][0, 0, lo + a:lo + b].cpu())
+        assert np.abs(lse - ref["LSE"][0, 0, a:b]).max() <= 1e-3, t
+
+
+def test_staged_masked_backward_matches_the_single_call(csa):
+    # attn_bwd_preprocess + attn_bwd_main_masked + attn_bwd_dq_convert is
+    # attn_bwd_masked; the window mask comes from the bench's mask recipe
+    B, H, N, d = 1, 2, 6 * 128 + 40, 64
+    q, k, v, do = draw(B, H, N, d, 341, "bf16")
+    bm = block_mask("window:3", N)
+    g = run_masked(csa, q, k, v, do, bm, d ** -0.5)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    mask = torch.from_numpy(bm).to(dev)
+    ws = csa.new_workspace(qd)
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    csa.attn_bwd_preprocess(g["O"], dod, g["LSE"], ws)
+    csa.attn_bwd_main_masked(qd, kd, vd, dod, dq, dk, dv, mask, ws)
+    csa.attn_bwd_dq_convert(dq, ws)
+    torch.cuda.synchronize()
+    assert csa.attn_last_status(ws) == 0
+    assert torch.equal(dk, g["dK"]) and torch.equal(dv, g["dV"])
+    ref = as_f64(g["dQ"].cpu())
+    assert rel(as_f64(dq.cpu()), ref, np.abs(ref).max()) <= 1e-2
 
 
 def test_linearity_and_causality(csa):
