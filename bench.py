@@ -114,16 +114,28 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    def __del__(self):
+        if self.file is not None and os.path.exists(self.file.name):
+            os.unlink(self.file.name)
+
     def summary(self, t0=None, t1=None):
         """Median SM clock and active throttle reasons of the samples taken
-        between host times t0 and t1 (the timed region), or of all samples."""
+        between host times t0 and t1 (the timed region), or of all samples.
+        A timed region shorter than the sampling interval holds no sample:
+        then the samples within 0.3 s of it are used, and the result says so."""
+        out = self._summary(t0, t1)
+        if out.get("samples") == 0 and t0 is not None:
+            out = self._summary(t0 - 0.3, t1 + 0.3)
+            out["window"] = "timed region +- 0.3 s (the region is shorter than the sampling interval)"
+        return out
+
+    def _summary(self, t0=None, t1=None):
         import datetime
         if self.proc is None or self.file is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.file.flush()
         with open(self.file.name) as fh:
             rows = [r.strip().split(", ") for r in fh if r.strip()]
-        os.unlink(self.file.name)
         sm, smax, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
