@@ -56,6 +56,8 @@ def _load() -> ctypes.CDLL:
         "attn_fwd_masked": (i, [vp] * 5 + [i, i, i, i, vp, f, i, vp]),
         "attn_bwd_masked": (i, [vp] * 9 + [i, i, i, i, vp, f, i, vp, sz, vp]),
         "attn_bwd_main_masked": (i, [vp] * 7 + [i, i, i, i, vp, f, i, vp, sz, vp]),
+        "attn_fwd_strided": (i, [vp] * 5 + [i, i, i, i, vp, vp, i, f, i, vp]),
+        "attn_bwd_strided": (i, [vp] * 9 + [i, i, i, i, vp, vp, i, f, i, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -68,7 +70,7 @@ _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
             "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc", "attn_fwd_masked",
-            "attn_bwd_masked", "attn_bwd_main_masked")
+            "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided")
 
 
 def library() -> ctypes.CDLL:
@@ -199,6 +201,54 @@ def new_workspace(q: torch.Tensor) -> torch.Tensor:
     if nbytes == 0:
         raise AttnError(ATTN_ERR_INVALID, "attn_bwd_workspace_bytes")
     return torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+
+
+def row_strides(t: torch.Tensor) -> tuple:
+    """Element strides (b, h, n) of a [B, H, N, d] view whose channels are
+    contiguous, e.g. x.permute(0, 2, 1, 3) of a [B, N, H, d] tensor."""
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [B, H, N, d] view with unit channel stride")
+    return tuple(int(x) for x in t.stride()[:3])
+
+
+def _strides_arg(tensors, what: str):
+    st = {row_strides(t) for t in tensors}
+    if len(st) != 1:
+        raise ValueError(f"{what} must share one stride set, got {sorted(st)}")
+    return (ctypes.c_longlong * 3)(*st.pop())
+
+
+def attn_fwd_strided(q, k, v, o, lse, causal: bool = True, scale: float | None = None,
+                     stream=None, check: bool = True) -> int:
+    """attn_fwd on [B, H, N, d] views of any row strides: q, k, v share one
+    stride set (e.g. slices of a packed projection), o may have its own."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    qs, os_ = _strides_arg((q, k, v), "q, k, v"), _strides_arg((o,), "o")
+    st = _lib.attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                               ctypes.addressof(qs), ctypes.addressof(os_), int(causal),
+                               float(scale), _DTYPES[q.dtype], _stream(stream))
+    if check:
+        _check(st, "attn_fwd_strided")
+    return st
+
+
+def attn_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal: bool = True,
+                     scale: float | None = None, stream=None, check: bool = True) -> int:
+    """attn_bwd on strided views: q, k, v, dq, dk, dv share one stride set,
+    o and dout another."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    qs = _strides_arg((q, k, v, dq, dk, dv), "q, k, v, dq, dk, dv")
+    os_ = _strides_arg((o, dout), "o, dout")
+    st = _lib.attn_bwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, ctypes.addressof(qs),
+                               ctypes.addressof(os_), int(causal), float(scale),
+                               _DTYPES[q.dtype], _ptr(workspace), int(workspace.numel()),
+                               _stream(stream))
+    if check:
+        _check(st, "attn_bwd_strided")
+    return st
 
 
 def forward(q, k, v, causal: bool = True, scale: float | None = None):

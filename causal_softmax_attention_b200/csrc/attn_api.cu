@@ -61,6 +61,15 @@ bool all_aligned(std::initializer_list<const void*> ps) {
   return true;
 }
 
+// Tensor pointers: 16-byte aligned for bf16 (tensor maps, vector access),
+// 4-byte aligned for fp32 (the FFMA kernels read single elements).
+bool tensors_aligned(int dtype, std::initializer_list<const void*> ps) {
+  const uintptr_t mask = dtype == ATTN_BF16 ? 15u : 3u;
+  for (const void* p : ps)
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & mask) != 0) return false;
+  return true;
+}
+
 // The tensor-core kernels are built for sm_100a only.
 int check_device_sm100() {
   int dev = 0, major = 0, minor = 0;
@@ -91,23 +100,40 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a [BH][N][d] bf16 array: box = 128 rows x min(d, 64) channels,
-// swizzled to match the UMMA canonical layout. Rows past N read as zero.
-bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+// 4-D map {d, N, H, B} over a bf16 array whose rows `rs` lays out: box =
+// 128 rows x min(d, 64) channels of one (b, h), swizzled to match the UMMA
+// canonical layout. Rows past N read as zero.
+bool make_map(CUtensorMap* m, const void* base, int B, int N, int d, const RowStrides& rs) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const int ch = d >= 64 ? 64 : d;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(ch), static_cast<cuuint32_t>(kTile), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(rs.H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(rs.sn) * 2, static_cast<cuuint64_t>(rs.sh) * 2,
+                           static_cast<cuuint64_t>(rs.sb) * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(ch), static_cast<cuuint32_t>(kTile), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapSwizzle swz =
       ch * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Strides from the caller: positive, rows of one head at least d apart, and
+// for bf16 whole 16-byte units (the tensor maps and the vector stores need
+// it); below the tensor maps' 2^40-byte stride limit.
+int check_strides(const long long* st, int H, int d, int dtype, RowStrides* out) {
+  if (st == nullptr) return ATTN_ERR_INVALID;
+  const long long lim = 1LL << 36;
+  for (int i = 0; i < 3; ++i)
+    if (st[i] <= 0 || st[i] >= lim) return ATTN_ERR_INVALID;
+  if (st[2] < d) return ATTN_ERR_INVALID;
+  if (dtype == ATTN_BF16)
+    for (int i = 0; i < 3; ++i)
+      if (st[i] % 8 != 0) return ATTN_ERR_INVALID;
+  *out = {st[0], st[1], st[2], H};
+  return ATTN_OK;
 }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
@@ -147,10 +173,12 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
 
 namespace {
 
+// Every implementation takes the row strides of q, k, v (and of dq, dk, dv:
+// qs) and of o, dout (os); the plain entry points pass the contiguous layout.
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int N, int d, int causal, float scale, int dtype, const uint8_t* bmask,
-             void* stream) {
-  if (!all_aligned({q, k, v, o, lse})) return ATTN_ERR_INVALID;
+             const RowStrides& qs, const RowStrides& os, void* stream) {
+  if (!tensors_aligned(dtype, {q, k, v, o}) || !all_aligned({lse})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
@@ -159,51 +187,35 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (dtype == ATTN_F32)
     return from_cuda(launch_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                     static_cast<const float*>(v), static_cast<float*>(o), lse, BH,
-                                    N, d, causal != 0, scale, s));
+                                    N, d, causal != 0, scale, qs, os, s));
   if ((st = check_device_sm100()) != ATTN_OK) return st;
   TmaMaps m;
-  if (!make_map(&m.a, q, BH, N, d) || !make_map(&m.b, k, BH, N, d) ||
-      !make_map(&m.c, v, BH, N, d))
+  if (!make_map(&m.a, q, B, N, d, qs) || !make_map(&m.b, k, B, N, d, qs) ||
+      !make_map(&m.c, v, B, N, d, qs))
     return ATTN_ERR_CUDA;
   int* status = fwd_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
-  return from_cuda(launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, bmask, s));
+  return from_cuda(
+      launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, bmask, os, s));
 }
 
-}  // namespace
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int N, int d, int causal, float scale, int dtype, void* stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, stream);
-}
-
-int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+int preprocess_impl(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
+                    int dtype, void* workspace, size_t workspace_bytes, const RowStrides& os,
                     void* stream) {
-  if (block_mask == nullptr) return ATTN_ERR_INVALID;
-  if (dtype != ATTN_BF16) return check_shape(B, H, N, d, dtype) == ATTN_OK ? ATTN_ERR_UNSUPPORTED
-                                                                         : ATTN_ERR_INVALID;
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, scale, dtype, block_mask, stream);
-}
-
-int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
-                        int d, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!all_aligned({o, dout, lse})) return ATTN_ERR_INVALID;
+  if (!tensors_aligned(dtype, {o, dout}) || !all_aligned({lse})) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
   if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
   const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
-  return from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, dtype == ATTN_BF16, ws,
+  return from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, dtype == ATTN_BF16, os, ws,
                                      static_cast<cudaStream_t>(stream)));
 }
-
-namespace {
 
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, void* dq,
                   void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                   int dtype, void* workspace, size_t workspace_bytes, const uint8_t* bmask,
-                  void* stream) {
-  if (!all_aligned({q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
+                  const RowStrides& qs, const RowStrides& os, void* stream) {
+  if (!tensors_aligned(dtype, {q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
@@ -216,11 +228,11 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout,
                                     static_cast<const float*>(v),
                                     static_cast<const float*>(dout), static_cast<float*>(dq),
                                     static_cast<float*>(dk), static_cast<float*>(dv), BH, N, d,
-                                    causal != 0, scale, ws, s));
+                                    causal != 0, scale, qs, os, ws, s));
   if ((st = check_device_sm100()) != ATTN_OK) return st;
   TmaMaps m;
-  if (!make_map(&m.a, q, BH, N, d) || !make_map(&m.b, k, BH, N, d) ||
-      !make_map(&m.c, v, BH, N, d) || !make_map(&m.d, dout, BH, N, d))
+  if (!make_map(&m.a, q, B, N, d, qs) || !make_map(&m.b, k, B, N, d, qs) ||
+      !make_map(&m.c, v, B, N, d, qs) || !make_map(&m.d, dout, B, N, d, os))
     return ATTN_ERR_CUDA;
   int inject = 0;
   unsigned long long limit = kWaitLimitCycles;
@@ -232,17 +244,88 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout,
       g_fault.armed = 0;
     }
   }
-  return from_cuda(
-      launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject, bmask, s));
+  return from_cuda(launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject,
+                                   bmask, qs, s));
 }
 
+int dq_convert_impl(void* dq, int B, int H, int N, int d, float scale, int dtype,
+                    void* workspace, size_t workspace_bytes, const RowStrides& qs, void* stream) {
+  if (!tensors_aligned(dtype, {dq})) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if (dtype == ATTN_F32) return ATTN_OK;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  return from_cuda(
+      launch_dq_convert(dq, B * H, N, d, scale, qs, ws, static_cast<cudaStream_t>(stream)));
+}
+
+// The whole backward: every argument is checked before the first launch, so
+// a bad call enqueues nothing.
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+             int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+             const uint8_t* bmask, const RowStrides& qs, const RowStrides& os, void* stream) {
+  if (!tensors_aligned(dtype, {q, k, v, o, dout, dq, dk, dv}) || !all_aligned({lse}))
+    return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (bmask != nullptr && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
+  st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, os, stream);
+  if (st != ATTN_OK) return st;
+  st = bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
+                     workspace_bytes, bmask, qs, os, stream);
+  if (st != ATTN_OK) return st;
+  return dq_convert_impl(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, qs, stream);
+}
+
+RowStrides dense(int H, int N, int d) { return contiguous_strides(H, N, d); }
+
 }  // namespace
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, int causal, float scale, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, dense(H, N, d),
+                  dense(H, N, d), stream);
+}
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
+                    void* stream) {
+  if (block_mask == nullptr) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_BF16) return check_shape(B, H, N, d, dtype) == ATTN_OK ? ATTN_ERR_UNSUPPORTED
+                                                                         : ATTN_ERR_INVALID;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, scale, dtype, block_mask, dense(H, N, d),
+                  dense(H, N, d), stream);
+}
+
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, const long long* qkv_strides,
+                     const long long* o_strides, int causal, float scale, int dtype,
+                     void* stream) {
+  RowStrides qs{}, os{};
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_strides(qkv_strides, H, d, dtype, &qs)) != ATTN_OK) return st;
+  if ((st = check_strides(o_strides, H, d, dtype, &os)) != ATTN_OK) return st;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, qs, os, stream);
+}
+
+int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
+                        int d, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes,
+                         dense(H, N, d), stream);
+}
 
 int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
                   void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                   int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                       workspace_bytes, nullptr, stream);
+                       workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream);
 }
 
 int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void* dout, void* dq,
@@ -254,38 +337,21 @@ int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void
   if (st != ATTN_OK) return st;
   if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
-                       workspace_bytes, block_mask, stream);
+                       workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream);
 }
 
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  if (!all_aligned({dq})) return ATTN_ERR_INVALID;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-  int st = check_shape(B, H, N, d, dtype);
-  if (st != ATTN_OK) return st;
-  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
-  if (dtype == ATTN_F32) return ATTN_OK;
-  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
-  return from_cuda(launch_dq_convert(dq, B * H, N, d, scale, ws, static_cast<cudaStream_t>(stream)));
+  return dq_convert_impl(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, dense(H, N, d),
+                         stream);
 }
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
              int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
              void* stream) {
-  // Validate everything before the first launch so a bad call enqueues nothing.
-  if (!all_aligned({q, k, v, o, dout, lse, dq, dk, dv})) return ATTN_ERR_INVALID;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-  int st = check_shape(B, H, N, d, dtype);
-  if (st != ATTN_OK) return st;
-  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
-  if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
-  st = attn_bwd_preprocess(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, stream);
-  if (st != ATTN_OK) return st;
-  st = attn_bwd_main(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                     workspace_bytes, stream);
-  if (st != ATTN_OK) return st;
-  return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
+                  workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream);
 }
 
 int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
@@ -293,19 +359,22 @@ int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
                     int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
                     void* workspace, size_t workspace_bytes, void* stream) {
   if (block_mask == nullptr) return ATTN_ERR_INVALID;
-  if (!all_aligned({q, k, v, o, dout, lse, dq, dk, dv})) return ATTN_ERR_INVALID;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
+                  workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream);
+}
+
+int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                     int H, int N, int d, const long long* qkv_strides,
+                     const long long* o_strides, int causal, float scale, int dtype,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  RowStrides qs{}, os{};
   int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
-  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
-  if ((st = check_device_sm100()) != ATTN_OK) return st;
-  st = attn_bwd_preprocess(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, stream);
-  if (st != ATTN_OK) return st;
-  st = attn_bwd_main_masked(q, k, v, dout, dq, dk, dv, B, H, N, d, block_mask, scale, dtype,
-                            workspace, workspace_bytes, stream);
-  if (st != ATTN_OK) return st;
-  return attn_bwd_dq_convert(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, stream);
+  if ((st = check_strides(qkv_strides, H, d, dtype, &qs)) != ATTN_OK) return st;
+  if ((st = check_strides(o_strides, H, d, dtype, &os)) != ATTN_OK) return st;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
+                  workspace_bytes, nullptr, qs, os, stream);
 }
 
 int attn_last_status(const void* workspace) {

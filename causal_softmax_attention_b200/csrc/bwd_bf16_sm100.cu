@@ -141,8 +141,9 @@ struct BwdParams {
   const float* lse2;  // [BH][Np], LSE * log2(e), +inf past N
   const float* dvec;  // [BH][Np], D, 0 past N
   float* dq_acc;      // [BH][T][D/4][128][4]
-  __nv_bfloat16* dk;  // [BH][N][D]
+  __nv_bfloat16* dk;  // rows at qs.row(bh, key), D channels each
   __nv_bfloat16* dv;
+  RowStrides qs;      // strides of dk and dv (those of q, k, v)
   int* status;
   int N, Np, T, BH;
   int G;              // heads per scheduling group (see the CTA order in the kernel)
@@ -331,14 +332,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   if (warp == R::TMA_WARP) {
     // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
+      const int hh = bh % p.qs.H, hb = bh / p.qs.H;  // head and batch: TMA coordinates
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       prefetch_tensormap(&tm_do);
       mbar_arrive_expect_tx(&bars[B_KV], 2 * L::TILE);
       for (int c = 0; c < L::NCH; ++c) {
-        tma_load_3d(smem + L::K_OFF + c * L::CHUNK, &tm_k, &bars[B_KV], c * L::CH, j0, bh);
-        tma_load_3d(smem + L::V_OFF + c * L::CHUNK, &tm_v, &bars[B_KV], c * L::CH, j0, bh);
+        tma_load_4d(smem + L::K_OFF + c * L::CHUNK, &tm_k, &bars[B_KV], c * L::CH, j0, hh, hb);
+        tma_load_4d(smem + L::V_OFF + c * L::CHUNK, &tm_v, &bars[B_KV], c * L::CH, j0, hh, hb);
       }
       bool ok = true;
       int issued = 0;
@@ -351,10 +353,10 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
         uint64_t* bar = &bars[B_QFULL + s];
         mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
         for (int c = 0; c < L::NCH; ++c) {
-          tma_load_3d(smem + L::Q_OFF + s * L::TILE + c * L::CHUNK, &tm_q, bar, c * L::CH, i0,
-                      bh);
-          tma_load_3d(smem + L::DO_OFF + s * L::TILE + c * L::CHUNK, &tm_do, bar, c * L::CH,
-                      i0, bh);
+          tma_load_4d(smem + L::Q_OFF + s * L::TILE + c * L::CHUNK, &tm_q, bar, c * L::CH, i0,
+                      hh, hb);
+          tma_load_4d(smem + L::DO_OFF + s * L::TILE + c * L::CHUNK, &tm_do, bar, c * L::CH,
+                      i0, hh, hb);
         }
         bulk_load(smem + L::LSE_OFF + s * 512, p.lse2 + static_cast<size_t>(bh) * p.Np + i0, 512,
                   bar);
@@ -597,8 +599,8 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       // Epilogue: dV_j and scale * dK_j rows -> bf16, group g writing channels
       // [g*E_CH, (g+1)*E_CH). All lanes load; only the stores are predicated.
       const bool key_ok = key < p.N;
-      __nv_bfloat16* dv_row = p.dv + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
-      __nv_bfloat16* dk_row = p.dk + (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
+      __nv_bfloat16* dv_row = p.dv + p.qs.row(bh, key_ok ? key : 0);
+      __nv_bfloat16* dk_row = p.dk + p.qs.row(bh, key_ok ? key : 0);
       constexpr int W = R::E_CH >= 32 ? 32 : R::E_CH;
       const bool any = it > 0;  // a key tile that meets no query tile has dK = dV = 0
 #pragma unroll 1
@@ -645,7 +647,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 template <int D>
 cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, void* dv, int BH,
                               int N, bool causal, float scale, uint64_t wait_cycles, int inject,
-                              const uint8_t* bmask, cudaStream_t s) {
+                              const uint8_t* bmask, const RowStrides& qs, cudaStream_t s) {
   using L = BwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = bmask ? attn_bwd_bf16_sm100_kernel<D, true> : attn_bwd_bf16_sm100_kernel<D, false>;
@@ -684,6 +686,7 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.bmask = bmask;
+  p.qs = qs;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = wait_cycles;
@@ -697,17 +700,18 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
 
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
                             int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, const uint8_t* block_mask, cudaStream_t s) {
+                            int inject_fault, const uint8_t* block_mask, const RowStrides& qs,
+                            cudaStream_t s) {
   switch (d) {
     case 32:
       return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, block_mask, s);
+                                   inject_fault, block_mask, qs, s);
     case 64:
       return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, block_mask, s);
+                                   inject_fault, block_mask, qs, s);
     case 128:
       return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                    inject_fault, block_mask, s);
+                                    inject_fault, block_mask, qs, s);
     default:
       return cudaErrorInvalidValue;
   }

@@ -15,6 +15,25 @@ constexpr int kStatusTimeout = -4;
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// Element strides of a [B][H][N][d] view whose channel stride is 1: row i of
+// head (b, h) starts at element b*sb + h*sh + i*sn. H splits a flat head
+// index bh = b*H + h. The contiguous layout is {H*N*d, N*d, d}; the
+// (sequence, position, head, channel) tables of ddx issue #217 are
+// {N*H*d, d, H*d}.
+struct RowStrides {
+  long long sb, sh, sn;
+  int H;
+  __host__ __device__ __forceinline__ long long head(int bh) const {
+    return static_cast<long long>(bh / H) * sb + static_cast<long long>(bh % H) * sh;
+  }
+  __host__ __device__ __forceinline__ long long row(int bh, int i) const {
+    return head(bh) + static_cast<long long>(i) * sn;
+  }
+};
+inline RowStrides contiguous_strides(int H, int N, int d) {
+  return {static_cast<long long>(H) * N * d, static_cast<long long>(N) * d, d, H};
+}
+
 // Workspace carved out of the caller's buffer for one backward call.
 struct Workspace {
   int* status;     // device status word
@@ -37,17 +56,23 @@ Workspace carve_workspace(void* base, const WorkspaceLayout& L);
 constexpr uint64_t kWaitLimitCycles = 1ull << 31;
 
 // ---- launchers (return cudaError_t from the launch) ----
+// qs: strides of q, k, v and of dq, dk, dv; os: strides of o and dout.
 cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse, int BH, int N,
-                              int d, bool bf16, const Workspace& ws, cudaStream_t s);
-cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const Workspace& ws,
+                              int d, bool bf16, const RowStrides& os, const Workspace& ws,
                               cudaStream_t s);
+cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const RowStrides& qs,
+                              const Workspace& ws, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
-                           int BH, int N, int d, bool causal, float scale, cudaStream_t s);
+                           int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
+                           const RowStrides& os, cudaStream_t s);
 cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
                            float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                           float scale, const Workspace& ws, cudaStream_t s);
+                           float scale, const RowStrides& qs, const RowStrides& os,
+                           const Workspace& ws, cudaStream_t s);
 
-// Tensor-core (tcgen05) path; tensor maps are encoded by the caller.
+// Tensor-core (tcgen05) path; tensor maps are encoded by the caller, each a
+// 4-D map {d, N, H, B} with a box of {min(d, 64), 128, 1, 1}, loaded at
+// coordinates {channel, row, h, b}.
 struct TmaMaps {
   CUtensorMap a, b, c, d;
 };
@@ -55,10 +80,11 @@ struct TmaMaps {
 // the tile), T = ceil(N / 128), or null for the causal / full filter.
 cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
                             int d, bool causal, float scale, const uint8_t* block_mask,
-                            cudaStream_t s);
+                            const RowStrides& os, cudaStream_t s);
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
                             int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, const uint8_t* block_mask, cudaStream_t s);
+                            int inject_fault, const uint8_t* block_mask, const RowStrides& qs,
+                            cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 

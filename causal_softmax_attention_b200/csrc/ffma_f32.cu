@@ -29,14 +29,15 @@ __device__ __forceinline__ float group_sum(float x) {
   return x;
 }
 
-// Loads rows [r0, r0 + 32) x channels [0, DP) of a [N][d] fp32 matrix into
-// shared memory, zero-filling rows >= N and channels >= d.
+// Loads rows [r0, r0 + 32) x channels [0, DP) of an [N][d] fp32 matrix whose
+// rows are `sn` elements apart into shared memory, zero-filling rows >= N and
+// channels >= d.
 template <int DP>
 __device__ __forceinline__ void load_tile(float (*dst)[DP], const float* src, int r0, int N,
-                                          int d) {
+                                          int d, long long sn) {
   for (int idx = threadIdx.x; idx < kRowsTile * DP; idx += blockDim.x) {
     const int r = idx / DP, c = idx % DP;
-    dst[r][c] = (r0 + r < N && c < d) ? src[static_cast<size_t>(r0 + r) * d + c] : 0.f;
+    dst[r][c] = (r0 + r < N && c < d) ? src[(r0 + r) * sn + c] : 0.f;
   }
 }
 
@@ -44,7 +45,7 @@ template <int DP>
 __global__ void __launch_bounds__(128)
     fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                    const float* __restrict__ v, float* __restrict__ o, float* __restrict__ lse,
-                   int N, int d, int causal, float scale) {
+                   int N, int d, int causal, float scale, RowStrides qs, RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;  // rows per block
   __shared__ float sK[kRowsTile][DP];
@@ -52,15 +53,15 @@ __global__ void __launch_bounds__(128)
   const int bh = blockIdx.y;
   const int row = blockIdx.x * R + threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
-  const float* qh = q + static_cast<size_t>(bh) * N * d;
-  const float* kh = k + static_cast<size_t>(bh) * N * d;
-  const float* vh = v + static_cast<size_t>(bh) * N * d;
+  const float* qh = q + qs.head(bh);
+  const float* kh = k + qs.head(bh);
+  const float* vh = v + qs.head(bh);
 
   float qr[32], acc[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
-    qr[c] = (row < N && ch < d) ? qh[static_cast<size_t>(row) * d + ch] : 0.f;
+    qr[c] = (row < N && ch < d) ? qh[row * qs.sn + ch] : 0.f;
     acc[c] = 0.f;
   }
   float m = -INFINITY, z = 0.f;
@@ -68,8 +69,8 @@ __global__ void __launch_bounds__(128)
   const int key_end = causal ? last_row + 1 : N;
   for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sK, kh, k0, N, d);
-    load_tile<DP>(sV, vh, k0, N, d);
+    load_tile<DP>(sK, kh, k0, N, d, qs.sn);
+    load_tile<DP>(sV, vh, k0, N, d, qs.sn);
     __syncthreads();
     float s[kRowsTile];
     float mx = -INFINITY;
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(128)
   }
   if (row < N) {
     const float inv = 1.f / z;
-    float* orow = o + (static_cast<size_t>(bh) * N + row) * d;
+    float* orow = o + os.row(bh, row);
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       const int ch = 32 * part + c;
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(128)
                         const float* __restrict__ v, const float* __restrict__ dout,
                         const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
                         float* __restrict__ dk, float* __restrict__ dv, int N, int Np, int d,
-                        int causal, float scale) {
+                        int causal, float scale, RowStrides qs, RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;
   __shared__ float sQ[kRowsTile][DP];
@@ -128,22 +129,22 @@ __global__ void __launch_bounds__(128)
   const int bh = blockIdx.y;
   const int key = blockIdx.x * R + threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
-  const size_t off = static_cast<size_t>(bh) * N * d;
+  const long long off = qs.head(bh), ooff = os.head(bh);
   float kr[32], vr[32], gk[32], gv[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
     const bool in = key < N && ch < d;
-    kr[c] = in ? k[off + static_cast<size_t>(key) * d + ch] : 0.f;
-    vr[c] = in ? v[off + static_cast<size_t>(key) * d + ch] : 0.f;
+    kr[c] = in ? k[off + key * qs.sn + ch] : 0.f;
+    vr[c] = in ? v[off + key * qs.sn + ch] : 0.f;
     gk[c] = gv[c] = 0.f;
   }
   const int first_key = blockIdx.x * R;
   const int q_begin = causal ? (first_key / kRowsTile) * kRowsTile : 0;
   for (int q0 = q_begin; q0 < N; q0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sQ, q + off, q0, N, d);
-    load_tile<DP>(sdO, dout + off, q0, N, d);
+    load_tile<DP>(sQ, q + off, q0, N, d, qs.sn);
+    load_tile<DP>(sdO, dout + ooff, q0, N, d, os.sn);
     if (threadIdx.x < kRowsTile) {
       sL[threadIdx.x] = lse_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
       sD[threadIdx.x] = d_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
@@ -175,8 +176,8 @@ __global__ void __launch_bounds__(128)
     for (int c = 0; c < 32; ++c) {
       const int ch = 32 * part + c;
       if (ch < d) {
-        dk[off + static_cast<size_t>(key) * d + ch] = gk[c] * scale;
-        dv[off + static_cast<size_t>(key) * d + ch] = gv[c];
+        dk[off + key * qs.sn + ch] = gk[c] * scale;
+        dv[off + key * qs.sn + ch] = gv[c];
       }
     }
   }
@@ -188,7 +189,8 @@ __global__ void __launch_bounds__(128)
     bwd_dq_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                       const float* __restrict__ v, const float* __restrict__ dout,
                       const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
-                      float* __restrict__ dq, int N, int Np, int d, int causal, float scale) {
+                      float* __restrict__ dq, int N, int Np, int d, int causal, float scale,
+                      RowStrides qs, RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;
   __shared__ float sK[kRowsTile][DP];
@@ -196,14 +198,14 @@ __global__ void __launch_bounds__(128)
   const int bh = blockIdx.y;
   const int row = blockIdx.x * R + threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
-  const size_t off = static_cast<size_t>(bh) * N * d;
+  const long long off = qs.head(bh), ooff = os.head(bh);
   float qr[32], dor[32], g[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
     const bool in = row < N && ch < d;
-    qr[c] = in ? q[off + static_cast<size_t>(row) * d + ch] : 0.f;
-    dor[c] = in ? dout[off + static_cast<size_t>(row) * d + ch] : 0.f;
+    qr[c] = in ? q[off + row * qs.sn + ch] : 0.f;
+    dor[c] = in ? dout[ooff + row * os.sn + ch] : 0.f;
     g[c] = 0.f;
   }
   const float Li = lse_pad[static_cast<size_t>(bh) * Np + min(row, Np - 1)];
@@ -212,8 +214,8 @@ __global__ void __launch_bounds__(128)
   const int key_end = causal ? last_row + 1 : N;
   for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sK, k + off, k0, N, d);
-    load_tile<DP>(sV, v + off, k0, N, d);
+    load_tile<DP>(sK, k + off, k0, N, d, qs.sn);
+    load_tile<DP>(sV, v + off, k0, N, d, qs.sn);
     __syncthreads();
 #pragma unroll 4
     for (int u = 0; u < kRowsTile; ++u) {
@@ -237,50 +239,56 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       const int ch = 32 * part + c;
-      if (ch < d) dq[off + static_cast<size_t>(row) * d + ch] = g[c] * scale;
+      if (ch < d) dq[off + row * qs.sn + ch] = g[c] * scale;
     }
   }
 }
 
 template <int DP>
 cudaError_t fwd_f32_dp(const float* q, const float* k, const float* v, float* o, float* lse,
-                       int BH, int N, int d, bool causal, float scale, cudaStream_t s) {
+                       int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
+                       const RowStrides& os, cudaStream_t s) {
   constexpr int R = 128 / (DP / 32);
   dim3 grid((N + R - 1) / R, BH);
-  fwd_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, o, lse, N, d, causal, scale);
+  fwd_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, o, lse, N, d, causal, scale, qs, os);
   return cudaGetLastError();
 }
 
 template <int DP>
 cudaError_t bwd_f32_dp(const float* q, const float* k, const float* v, const float* dout,
                        float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                       float scale, const Workspace& ws, cudaStream_t s) {
+                       float scale, const RowStrides& qs, const RowStrides& os,
+                       const Workspace& ws, cudaStream_t s) {
   constexpr int R = 128 / (DP / 32);
   dim3 grid((N + R - 1) / R, BH);
   bwd_dkdv_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dk, dv, N,
-                                               ws.Np, d, causal, scale);
+                                               ws.Np, d, causal, scale, qs, os);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dq_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dq, N, ws.Np,
-                                             d, causal, scale);
+                                             d, causal, scale, qs, os);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
-                           int BH, int N, int d, bool causal, float scale, cudaStream_t s) {
-  if (d <= 32) return fwd_f32_dp<32>(q, k, v, o, lse, BH, N, d, causal, scale, s);
-  if (d <= 64) return fwd_f32_dp<64>(q, k, v, o, lse, BH, N, d, causal, scale, s);
-  return fwd_f32_dp<128>(q, k, v, o, lse, BH, N, d, causal, scale, s);
+                           int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
+                           const RowStrides& os, cudaStream_t s) {
+  if (d <= 32) return fwd_f32_dp<32>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
+  if (d <= 64) return fwd_f32_dp<64>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
+  return fwd_f32_dp<128>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
 }
 
 cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
                            float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                           float scale, const Workspace& ws, cudaStream_t s) {
-  if (d <= 32) return bwd_f32_dp<32>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
-  if (d <= 64) return bwd_f32_dp<64>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
-  return bwd_f32_dp<128>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, ws, s);
+                           float scale, const RowStrides& qs, const RowStrides& os,
+                           const Workspace& ws, cudaStream_t s) {
+  if (d <= 32)
+    return bwd_f32_dp<32>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
+  if (d <= 64)
+    return bwd_f32_dp<64>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
+  return bwd_f32_dp<128>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
 }
 
 }  // namespace csa

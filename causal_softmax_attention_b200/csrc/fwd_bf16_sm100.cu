@@ -88,7 +88,8 @@ enum FBar {
 static_assert(F_COUNT <= 32, "barrier slots");
 
 struct FwdParams {
-  __nv_bfloat16* o;  // [BH][N][D]
+  __nv_bfloat16* o;  // rows at os.row(bh, i), D channels each
+  RowStrides os;     // strides of o
   float* lse;        // [BH][N]
   int* status;
   int N, T, BH;
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // (a block mask is taken to be causal-like: later query tiles first too)
   const int it_q = (p.causal || kMask) ? p.T - 1 - r / gs : r / gs;
   const int bh = g0 + r % gs;
+  const int hh = bh % p.os.H, hb = bh / p.os.H;  // head and batch: TMA coordinates
   const int i0 = it_q * kTile;
   // The key tiles this query tile meets, in increasing order: j <= i under
   // the causal filter, all of them without it, or those a block mask marks.
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         prefetch_tensormap(&tm_q);
         mbar_arrive_expect_tx(&bars[F_Q], L::TILE);
         for (int c = 0; c < L::NCH; ++c)
-          tma_load_3d(smem + L::Q_OFF + c * L::CHUNK, &tm_q, &bars[F_Q], c * L::CH, i0, bh);
+          tma_load_4d(smem + L::Q_OFF + c * L::CHUNK, &tm_q, &bars[F_Q], c * L::CH, i0, hh, hb);
       }
       bool ok = true;
       int issued = 0;
@@ -228,8 +230,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           break;
         mbar_arrive_expect_tx(&bars[full + s], L::TILE);
         for (int c = 0; c < L::NCH; ++c)
-          tma_load_3d(smem + off + s * L::TILE + c * L::CHUNK, map, &bars[full + s], c * L::CH,
-                      j * kTile, bh);
+          tma_load_4d(smem + off + s * L::TILE + c * L::CHUNK, map, &bars[full + s], c * L::CH,
+                      j * kTile, hh, hb);
         ++issued;
       }
       if (!ok) fail();
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float inv = z > 0.f ? 1.f / z : 0.f;
       const bool row_ok = qrow < p.N;
       __nv_bfloat16* orow =
-          p.o + (static_cast<size_t>(bh) * p.N + (row_ok ? qrow : 0)) * D + g * L::HALF_D;
+          p.o + p.os.row(bh, row_ok ? qrow : 0) + g * L::HALF_D;
 #pragma unroll 1
       for (int c = 0; c < L::HALF_D; c += 16) {
         uint32_t ov[16];
@@ -432,7 +434,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 template <int D>
 cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int BH, int N,
-                         bool causal, float scale, const uint8_t* bmask, cudaStream_t s) {
+                         bool causal, float scale, const uint8_t* bmask, const RowStrides& os,
+                         cudaStream_t s) {
   using L = FwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = bmask ? attn_fwd_bf16_sm100_kernel<D, true> : attn_fwd_bf16_sm100_kernel<D, false>;
@@ -455,6 +458,7 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.bmask = bmask;
+  p.os = os;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = kWaitLimitCycles;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
@@ -466,11 +470,12 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
 
 cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
                             int d, bool causal, float scale, const uint8_t* block_mask,
-                            cudaStream_t s) {
+                            const RowStrides& os, cudaStream_t s) {
   switch (d) {
-    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
-    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
-    case 128: return launch_fwd_d<128>(maps, o, lse, status, BH, N, causal, scale, block_mask, s);
+    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
+    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
+    case 128:
+      return launch_fwd_d<128>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
     default: return cudaErrorInvalidValue;
   }
 }

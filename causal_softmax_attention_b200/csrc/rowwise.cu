@@ -24,7 +24,8 @@ __global__ void __launch_bounds__(256)
     preprocess_bf16_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                            const float* __restrict__ lse, float* __restrict__ lse_pad,
                            float* __restrict__ d_pad, float4* __restrict__ dq_acc,
-                           size_t acc_vecs, int* status, int BH, int N, int Np) {
+                           size_t acc_vecs, int* status, int BH, int N, int Np,
+                           RowStrides os) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = kStatusOk;
   const size_t total_rows = static_cast<size_t>(BH) * Np;
   const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -40,7 +41,7 @@ __global__ void __launch_bounds__(256)
     const int i = static_cast<int>(r % Np);
     float acc = 0.f;
     if (active && i < N) {
-      const size_t idx = (static_cast<size_t>(bh) * N + i) * G + sub;
+      const size_t idx = static_cast<size_t>(os.row(bh, i) / 8) + sub;  // 16-byte vectors
       const uint4 a = o[idx], b = dout[idx];
       const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
       const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
@@ -69,7 +70,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     preprocess_f32_kernel(const float* __restrict__ o, const float* __restrict__ dout,
                           const float* __restrict__ lse, float* __restrict__ lse_pad,
-                          float* __restrict__ d_pad, int* status, int BH, int N, int Np, int d) {
+                          float* __restrict__ d_pad, int* status, int BH, int N, int Np, int d,
+                          RowStrides os) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = kStatusOk;
   const size_t total_rows = static_cast<size_t>(BH) * Np;
   const size_t warp0 = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
@@ -80,7 +82,7 @@ __global__ void __launch_bounds__(256)
     const int i = static_cast<int>(r % Np);
     float acc = 0.f;
     if (i < N) {
-      const size_t row = (static_cast<size_t>(bh) * N + i) * d;
+      const size_t row = static_cast<size_t>(os.row(bh, i));
       for (int c = lane; c < d; c += 32) acc = fmaf(o[row + c], dout[row + c], acc);
     }
 #pragma unroll
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(256)
 // 4*c4 + e). Each thread converts 8 consecutive columns of one row.
 __global__ void __launch_bounds__(256)
     dq_convert_kernel(const float4* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int BH,
-                      int N, int T, int d, float scale) {
+                      int N, int T, int d, float scale, RowStrides qs) {
   const int g8 = d / 8;
   const size_t total = static_cast<size_t>(BH) * T * g8 * kTile;
   const size_t nthreads = static_cast<size_t>(gridDim.x) * blockDim.x;
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(256)
     h[1] = __floats2bfloat162_rn(x.z * scale, x.w * scale);
     h[2] = __floats2bfloat162_rn(y.x * scale, y.y * scale);
     h[3] = __floats2bfloat162_rn(y.z * scale, y.w * scale);
-    *reinterpret_cast<uint4*>(dq + (static_cast<size_t>(bh) * N + i) * d + 8 * g) =
+    *reinterpret_cast<uint4*>(dq + qs.row(bh, i) + 8 * g) =
         *reinterpret_cast<const uint4*>(h);
   }
 }
@@ -145,12 +147,13 @@ unsigned grid_for(size_t threads_needed) {
 }  // namespace
 
 cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse, int BH, int N,
-                              int d, bool bf16, const Workspace& ws, cudaStream_t s) {
+                              int d, bool bf16, const RowStrides& os, const Workspace& ws,
+                              cudaStream_t s) {
   const size_t rows = static_cast<size_t>(BH) * ws.Np;
   if (!bf16) {
     preprocess_f32_kernel<<<grid_for(rows * 32), 256, 0, s>>>(
         static_cast<const float*>(o), static_cast<const float*>(dout), lse, ws.lse_pad,
-        ws.d_pad, ws.status, BH, N, ws.Np, d);
+        ws.d_pad, ws.status, BH, N, ws.Np, d, os);
     return cudaGetLastError();
   }
   const size_t acc_vecs = rows * d / 4;
@@ -162,15 +165,15 @@ cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse,
   switch (G) {
     case 4:
       preprocess_bf16_kernel<4><<<grid, 256, 0, s>>>(po, pd, lse, ws.lse_pad, ws.d_pad, acc,
-                                                     acc_vecs, ws.status, BH, N, ws.Np);
+                                                     acc_vecs, ws.status, BH, N, ws.Np, os);
       break;
     case 8:
       preprocess_bf16_kernel<8><<<grid, 256, 0, s>>>(po, pd, lse, ws.lse_pad, ws.d_pad, acc,
-                                                     acc_vecs, ws.status, BH, N, ws.Np);
+                                                     acc_vecs, ws.status, BH, N, ws.Np, os);
       break;
     case 16:
       preprocess_bf16_kernel<16><<<grid, 256, 0, s>>>(po, pd, lse, ws.lse_pad, ws.d_pad, acc,
-                                                      acc_vecs, ws.status, BH, N, ws.Np);
+                                                      acc_vecs, ws.status, BH, N, ws.Np, os);
       break;
     default:
       return cudaErrorInvalidValue;
@@ -178,13 +181,13 @@ cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse,
   return cudaGetLastError();
 }
 
-cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const Workspace& ws,
-                              cudaStream_t s) {
+cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const RowStrides& qs,
+                              const Workspace& ws, cudaStream_t s) {
   const int T = ws.Np / kTile;
   const size_t total = static_cast<size_t>(BH) * T * (d / 8) * kTile;
   dq_convert_kernel<<<grid_for(total), 256, 0, s>>>(reinterpret_cast<const float4*>(ws.dq_acc),
                                                     static_cast<__nv_bfloat16*>(dq), BH, N, T, d,
-                                                    scale);
+                                                    scale, qs);
   return cudaGetLastError();
 }
 

@@ -27,9 +27,10 @@
  * the legacy default stream).
  *
  * Errors. Arguments are checked before anything is launched:
- *   null pointers, B, H, N <= 0, d <= 0, non-finite scale, pointers that are
- *   not 16-byte aligned, a workspace smaller than attn_bwd_workspace_bytes
- *     -> ATTN_ERR_INVALID
+ *   null pointers, B, H, N <= 0, d <= 0, non-finite scale, tensor pointers
+ *   not 16-byte aligned (bf16) or 4-byte aligned (f32), an LSE array or a
+ *   workspace not 16-byte aligned, a workspace smaller than
+ *   attn_bwd_workspace_bytes -> ATTN_ERR_INVALID
  *   (dtype, d) outside the built set: bf16 with d in {32, 64, 128}, f32 with
  *   1 <= d <= 128 -> ATTN_ERR_UNSUPPORTED
  *   a failed launch or a non-sm_100 device -> ATTN_ERR_CUDA
@@ -126,6 +127,34 @@ int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                     int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Strided layouts: q, k, v, o, dout, dq, dk, dv given as [B][H][N][d] views
+ * of arbitrary row strides (the channel stride is 1), so that the
+ * (sequence, position, head, channel) tables of ddx issue #217 ("Backward of
+ * batched attention builds a contraction over every pair of sequences and
+ * heads", the repro's `q`, `k`, `v` tables and its JAX restatement), or a
+ * packed [B][N][3][H][d] projection output, are consumed without a permute.
+ *   qkv_strides : in, HOST array {s_b, s_h, s_n} of element strides for q, k,
+ *                 v and for dq, dk, dv: row n of head (b, h) of q starts at
+ *                 q + b*s_b + h*s_h + n*s_n.
+ *   o_strides   : in, HOST array {s_b, s_h, s_n} for o and dout.
+ * Each stride must be > 0 and < 2^36 and s_n >= d; for bf16 each must be a
+ * multiple of 8 elements (16 bytes). Rows of the outputs must not overlap.
+ * Contiguous [B][H][N][d] is {H*N*d, N*d, d}; [B][N][H][d] is
+ * {N*H*d, d, H*d}. LSE stays a contiguous [B][H][N] fp32 array.
+ * Everything else (arguments, results, workspace, checks, statuses) as
+ * attn_fwd / attn_bwd; a NULL or out-of-range stride array -> ATTN_ERR_INVALID.
+ */
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, const long long* qkv_strides,
+                     const long long* o_strides, int causal, float scale, int dtype,
+                     void* stream);
+int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                     int H, int N, int d, const long long* qkv_strides,
+                     const long long* o_strides, int causal, float scale, int dtype,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The three stages attn_bwd runs, exposed so a caller can time or overlap them

@@ -140,3 +140,39 @@ def test_masked_entry_points_reject_bad_arguments():
     assert m(*args, A, math.nan, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
     assert m(*args, A, 0.125, 1, A, 16, None) == csa.ATTN_ERR_INVALID
     assert m(*([A] * 6 + [A + 8, 1, 1, 300, 64]), A, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID
+
+
+def test_strided_entry_points_reject_bad_strides():
+    # every call returns during argument checking (no CUDA call)
+    f, b = L.attn_fwd_strided, L.attn_bwd_strided
+    good = (ctypes.c_longlong * 3)(300 * 64 * 2, 64, 2 * 64)
+    bad = {
+        "null": None,
+        "zero": (ctypes.c_longlong * 3)(0, 64, 128),
+        "negative": (ctypes.c_longlong * 3)(300 * 128, -64, 128),
+        "row closer than d": (ctypes.c_longlong * 3)(300 * 64, 64, 32),
+        "bf16 not 16-byte": (ctypes.c_longlong * 3)(300 * 128, 68, 128),
+        "beyond the map limit": (ctypes.c_longlong * 3)(1 << 36, 64, 128),
+    }
+    fargs = [A] * 5 + [1, 2, 300, 64]
+    bargs = [A] * 9 + [1, 2, 300, 64]
+    for name, st in bad.items():
+        p = ctypes.addressof(st) if st is not None else None
+        g = ctypes.addressof(good)
+        assert f(*fargs, p, g, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID, name
+        assert f(*fargs, g, p, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID, name
+        assert b(*bargs, p, g, 1, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID, name
+        assert b(*bargs, g, p, 1, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_INVALID, name
+    # shape checks come first; an unsupported head size stays unsupported
+    g = ctypes.addressof(good)
+    assert f(*([A] * 5 + [1, 2, 300, 96]), g, g, 1, 0.125, 1, None) == csa.ATTN_ERR_UNSUPPORTED
+
+
+def test_row_strides_of_views():
+    import torch
+    x = torch.empty(2, 5, 3, 64)  # [B, N, H, d]
+    assert csa.row_strides(x.permute(0, 2, 1, 3)) == (5 * 3 * 64, 64, 3 * 64)
+    qkv = torch.empty(2, 5, 3, 4, 32)  # packed [B, N, 3, H, d]
+    assert csa.row_strides(qkv[:, :, 1].permute(0, 2, 1, 3)) == (5 * 3 * 4 * 32, 32, 3 * 4 * 32)
+    with pytest.raises(ValueError):
+        csa.row_strides(x.permute(0, 3, 1, 2))

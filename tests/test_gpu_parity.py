@@ -264,6 +264,83 @@ def test_staged_masked_backward_matches_the_single_call(csa):
     assert rel(as_f64(dq.cpu()), ref, np.abs(ref).max()) <= 1e-2
 
 
+def run_strided(csa, q, k, v, do, causal, scale, layout):
+    """Forward and backward through the strided entry points, the tensors
+    held in `layout`: "bnhd" ([B, N, H, d] arrays) or "packed" (q, k, v in
+    one [B, N, 3, H, d] array and dq, dk, dv in another; o, dO [B, N, H, d])."""
+    dev = torch.device("cuda")
+    B, H, N, d = q.shape
+
+    def bnhd(x):  # a [B, N, H, d] array holding x, returned as its [B, H, N, d] view
+        return x.to(dev).permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+
+    if layout == "packed":
+        qkv = torch.stack([x.to(dev).permute(0, 2, 1, 3) for x in (q, k, v)], dim=2).contiguous()
+        qv, kv, vv = (qkv[:, :, c].permute(0, 2, 1, 3) for c in range(3))
+        dqkv = torch.full_like(qkv, float("nan"))
+        dq, dk, dv = (dqkv[:, :, c].permute(0, 2, 1, 3) for c in range(3))
+    else:
+        qv, kv, vv = bnhd(q), bnhd(k), bnhd(v)
+        dq, dk, dv = (bnhd(torch.full_like(q, float("nan"))) for _ in range(3))
+    dov = bnhd(do)
+    o = bnhd(torch.full_like(q, float("nan")))
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    csa.attn_fwd_strided(qv, kv, vv, o, lse, causal, scale)
+    csa.attn_bwd_strided(qv, kv, vv, o, dov, lse, dq, dk, dv, csa.new_workspace(qv.contiguous()),
+                         causal, scale)
+    torch.cuda.synchronize()
+    assert csa.attn_fwd_last_status() == 0
+    return {"O": o, "LSE": lse, "dQ": dq, "dK": dk, "dV": dv}
+
+
+@pytest.mark.parametrize("dtype,d,layout", [("bf16", 64, "bnhd"), ("bf16", 128, "bnhd"),
+                                            ("bf16", 64, "packed"), ("bf16", 32, "packed"),
+                                            ("f32", 48, "bnhd"), ("f32", 7, "packed")])
+def test_strided_layouts_match_the_contiguous_path(csa, dtype, d, layout):
+    # the same kernels on the same values: O, LSE, dK, dV bit-identical to the
+    # contiguous path (dQ too for f32; bf16 dQ sums in atomic order)
+    B, H, N = 2, 3, 2 * 128 + 45
+    q, k, v, do = draw(B, H, N, d, 361 + d, dtype)
+    c = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    g = run_strided(csa, q, k, v, do, True, d ** -0.5, layout)
+    for name in ("O", "LSE", "dK", "dV") + (("dQ",) if dtype == "f32" else ()):
+        assert torch.equal(g[name].contiguous(), c[name]), name
+    if dtype == "bf16":
+        ref = as_f64(c["dQ"].cpu())
+        assert rel(as_f64(g["dQ"].cpu()), ref) <= 1e-2
+
+
+def test_strided_ddx_issue217_tables_against_the_oracle(csa):
+    # the repro's (seq, pos, head, channel) tables consumed in place (f32,
+    # 4 channels), against the oracle on the same values; loss 1/2 sum O^2
+    # so dO = O
+    from seeded_inputs import ddx_issue217_input
+    S, T, H, C = 3, 8, 2, 4
+    # [B, H, N, d], rounded to the fp32 values the GPU receives
+    qh, kh, vh = (x.astype(np.float32).astype(np.float64) for x in ddx_issue217_input(S, T, H, C))
+    scale = 1.0 / 2.0
+    o_ref, _ = oracle.forward(qh, kh, vh, scale, True)
+    ref = oracle.backward(qh, kh, vh, o_ref, scale, True)
+    dev = torch.device("cuda")
+
+    def table(x):  # [S, T, H, C] float32 table, viewed as [B, H, N, d]
+        return torch.from_numpy(x).float().to(dev).permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+
+    q, k, v = table(qh), table(kh), table(vh)
+    o = table(np.zeros_like(qh))
+    lse = torch.empty(S, H, T, dtype=torch.float32, device=dev)
+    csa.attn_fwd_strided(q, k, v, o, lse, True, scale)
+    dout = o.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    dq, dk, dv = (table(np.zeros_like(qh)) for _ in range(3))
+    csa.attn_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, csa.new_workspace(q.contiguous()),
+                         True, scale)
+    torch.cuda.synchronize()
+    assert rel(as_f64(o.cpu()), o_ref) <= 1e-5
+    gscale = max(np.abs(ref[n]).max() for n in ("dQ", "dK", "dV"))
+    for name, t in (("dQ", dq), ("dK", dk), ("dV", dv)):
+        assert rel(as_f64(t.cpu()), ref[name], gscale) <= 1e-5, name
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
