@@ -15,6 +15,17 @@ all ranks' FLOPs / max-over-ranks device time.
 `--impl reference` times the float64 CPU oracle instead (rank 0 only), on a
 bounded sample of the same workload per step.
 
+`--layout bnhd|packed` holds the tensors as [B, N, H, d] arrays (packed: q, k,
+v in one [B, N, 3, H, d] array, dq, dk, dv in another) and times one
+attn_bwd_strided call per step; the roofline then uses that whole call.
+
+`--layer` times one causal multi-head attention layer instead (the attention
+sublayer of the nanoGPT-shaped step of ddx issue #217, x [B, N, C] with
+C = H*d, the projections as cuBLAS GEMMs, the attention on the strided
+kernels): forward + backward per step, FLOPs = 24*B*N*C^2 for the four
+projections (forward and both backward products) + the attention's causal
+forward and backward.
+
 `--block-mask SPEC` (causal, full, window:W, random:P:SEED over 128 x 128
 tiles; bf16) times the block-sparse backward instead: the same three stages
 with the masked main kernel, FLOPs counted over the kept tiles (a kind-1 tile
@@ -285,8 +296,10 @@ def run_reference(args, cfg, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(cfg, n_gpus, mask_spec=None):
+def config_dict(cfg, n_gpus, mask_spec=None, layout="bhnd"):
     kind = "causal" if mask_spec is None else f"block-sparse ({mask_spec} over 128x128 tiles)"
+    if layout != "bhnd":
+        kind += f", {layout} layout"
     out = {"workload": f"{cfg.name}: {kind} attention backward B={cfg.B} H={cfg.H} "
                         f"N={cfg.N} d={cfg.d} {cfg.dtype}, q,k,v,dO ~ N(0,1)"
                         + (f" (q,k x{cfg.qk_gain})" if cfg.qk_gain != 1.0 else "")
@@ -297,11 +310,105 @@ def config_dict(cfg, n_gpus, mask_spec=None):
             "l2": "inputs larger than L2 (no flush needed)"
             if 5 * cfg.B * cfg.H * cfg.N * cfg.d * 2 > 126e6
             else "L2 flushed (256 MB write) between steps, outside the steps' events"}
+    out["layout"] = layout
     if mask_spec is not None:
         bm = block_mask(mask_spec, cfg.N)
         out["block_mask"] = mask_spec
         out["kept_fraction_of_causal"] = block_mask_pairs(bm) / (cfg.N * cfg.N / 2)
     return out
+
+
+# --------------------------------------------------------------------- layer arm
+def run_layer(args, cfg, world, rank, local):
+    import causal_softmax_attention_b200 as csa
+    from causal_softmax_attention_b200 import layer
+    from seeded_inputs import draw_layer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
+    C = H * d
+    hx, hwq, hwo, hdy = (t.pin_memory() for t in draw_layer(B, N, C, cfg.seed + 1000 * rank))
+    x, wq, wo, dy = (t.to(dev) for t in (hx, hwq, hwo, hdy))
+    ws = torch.empty(csa.attn_bwd_workspace_bytes(B, H, N, d, x.dtype), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    proj = 24.0 * B * N * C * C
+    flops = proj + cfg.fwd_flops + cfg.bwd_flops
+
+    def step():
+        y, saved = layer.layer_forward(x, wq, wo, H, stream)
+        return layer.layer_backward(dy, saved, wq, wo, H, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        time.sleep(1.0)
+        host_t0 = time.time()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        host_t1 = time.time()
+        time.sleep(0.25)
+    ms_per_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    value = whole_job_tflops(flops, world, ms_per_step)
+
+    # e2e: x, dy and the weights from pinned host memory, dx and the weight
+    # gradients back to pinned host memory, serialised with the step
+    outs = step()
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hwq, hwo, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for dst, src in zip((x, wq, wo, dy), (hx, hwq, hwo, hdy)):
+            dst.copy_(src, non_blocking=True)
+        for dst, src in zip(host_out, step()):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 5))
+    f0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, world)
+    if rank != 0:
+        return
+    if csa.attn_fwd_last_status() != 0:
+        raise RuntimeError("forward status after the layer steps")
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    line = {
+        "metric": "causal multi-head attention layer step TFLOP/s (bf16, forward + backward)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"attention layer B={B} N={N} C={C} H={H} (d={d}), causal, "
+                               "x, dy ~ N(0,1), weights ~ N(0,1/C), no biases",
+                   "B": B, "N": N, "C": C, "H": H, "d": d, "parallelism": "single GPU",
+                   "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "whole layer step (4 cuBLAS GEMMs x 3 + attention fwd + bwd)",
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": ms_per_step,
+                     "projection_flops": proj},
+        "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,  # attn_fwd, preprocess, main, dQ convert (GEMMs are cuBLAS)
+        "clocks": clocks.summary(host_t0, host_t1),
+    }
+    print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------------------- GPU arm
@@ -328,10 +435,31 @@ def run_gpu(args, cfg, world, rank, local):
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     ws = csa.new_workspace(qd)
     stream = torch.cuda.current_stream(dev)
+    if args.layout != "bhnd":
+        # the same values held in [B, N, H, d] arrays (packed: q, k, v in one
+        # [B, N, 3, H, d] array), as [B, H, N, d] views
+        def bnhd(x):
+            return x.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        if args.layout == "packed":
+            qkv = torch.stack([x.permute(0, 2, 1, 3) for x in (qd, kd, vd)], dim=2).contiguous()
+            dqkv = torch.empty_like(qkv)
+            sq, sk, sv = (qkv[:, :, c].permute(0, 2, 1, 3) for c in range(3))
+            gq, gk, gv = (dqkv[:, :, c].permute(0, 2, 1, 3) for c in range(3))
+        else:
+            sq, sk, sv = bnhd(qd), bnhd(kd), bnhd(vd)
+            gq, gk, gv = bnhd(dq), bnhd(dk), bnhd(dv)
+        so, sdo = bnhd(o), bnhd(dod)
     small = 5 * B * H * N * d * 2 <= 126e6
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small else None
 
     def step(ev_main=None):
+        if args.layout != "bhnd":
+            if ev_main is not None:
+                ev_main[0].record(stream)
+            csa.attn_bwd_strided(sq, sk, sv, so, sdo, lse, gq, gk, gv, ws, True, cfg.scale, stream)
+            if ev_main is not None:
+                ev_main[1].record(stream)
+            return
         csa.attn_bwd_preprocess(o, dod, lse, ws, stream)
         if ev_main is not None:
             ev_main[0].record(stream)
@@ -404,6 +532,30 @@ def run_gpu(args, cfg, world, rank, local):
         csa.backward_host(hq, hk, hv, ho, hdo, hlse, hdq, hdk, hdv, dev_bufs, True, cfg.scale,
                           e2e_chunks, stream, block_mask=mask)
 
+    e2e_path = (f"backward_host: pinned host buffers, {e2e_chunks} head groups, "
+                "H2D / attn_bwd / D2H overlapped on three streams")
+    if args.layout != "bhnd":
+        # the strided arrays themselves go host -> device -> host around one
+        # attn_bwd_strided call (copies serialised with the call)
+        dev_in = [x for x in ((qkv,) if args.layout == "packed" else (sq, sk, sv))]
+        dev_in = [x if x.is_contiguous() else x.permute(0, 2, 1, 3) for x in dev_in]
+        dev_in += [so.permute(0, 2, 1, 3), sdo.permute(0, 2, 1, 3), lse]
+        dev_out = [dqkv] if args.layout == "packed" else [x.permute(0, 2, 1, 3) for x in (gq, gk, gv)]
+        host_in = [x.cpu().pin_memory() for x in dev_in]
+        host_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in dev_out]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        e2e_path = f"{args.layout} arrays from pinned host memory, one attn_bwd_strided, back to host"
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for dsti, srci in zip(dev_in, host_in):
+                    dsti.copy_(srci, non_blocking=True)
+                csa.attn_bwd_strided(sq, sk, sv, so, sdo, lse, gq, gk, gv, ws, True, cfg.scale,
+                                     stream)
+                for dsto, srco in zip(host_out, dev_out):
+                    dsto.copy_(srco, non_blocking=True)
+
     e2e_steps = max(1, min(args.steps, 5))
     for _ in range(2):
         e2e_step()
@@ -423,7 +575,9 @@ def run_gpu(args, cfg, world, rank, local):
     fwd_iters = 5
 
     def fwd():
-        if mask is None:
+        if args.layout != "bhnd":
+            csa.attn_fwd_strided(sq, sk, sv, so, lse, True, cfg.scale, stream)
+        elif mask is None:
             csa.attn_fwd(qd, kd, vd, o, lse, True, cfg.scale, stream)
         else:
             csa.attn_fwd_masked(qd, kd, vd, o, lse, mask, cfg.scale, stream)
@@ -444,12 +598,13 @@ def run_gpu(args, cfg, world, rank, local):
     main_avg = statistics.mean(main_ms)
     achieved = flops / (main_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = dram_traffic_per_launch(cfg) if mask is None else None
+    traffic = dram_traffic_per_launch(cfg) if mask is None and args.layout == "bhnd" else None
     clk = clocks.summary(host_t0, host_t1)
     if cfg.dtype == "bf16":
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
-                    "kernel": "attn_bwd_bf16_sm100_kernel",
+                    "kernel": "attn_bwd_bf16_sm100_kernel" if args.layout == "bhnd"
+                    else "attn_bwd_strided (whole call: preprocess, main kernel, dQ convert)",
                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": main_avg}
@@ -465,15 +620,14 @@ def run_gpu(args, cfg, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-        "data": "synthetic", "config": config_dict(cfg, world, args.block_mask),
+        "data": "synthetic", "config": config_dict(cfg, world, args.block_mask, args.layout),
         "pct_of_dense_bf16_peak": 100.0 * value / world / peak,
         "roofline": roofline,
         "stage_ms": {"step_median": statistics.median(step_ms), "main_median": statistics.median(main_ms),
                      "pre_and_convert_median": statistics.median(step_ms) - statistics.median(main_ms)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "path": f"backward_host: pinned host buffers, {e2e_chunks} head groups, "
-                        "H2D / attn_bwd / D2H overlapped on three streams"},
+                "path": e2e_path},
         "forward": {"kernel": "attn_fwd_bf16_sm100_kernel" if cfg.dtype == "bf16"
                     else "fwd_f32_kernel", "ms": fwd_ms,
                     "tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
@@ -507,6 +661,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head groups of the end-to-end (host-buffer) measurement")
+    ap.add_argument("--layer", action="store_true",
+                    help="time one attention layer step (projections + attention, fwd + bwd)")
+    ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd", "packed"],
+                    help="memory layout of q, k, v, o, dO and the gradients")
     ap.add_argument("--block-mask", default=None, metavar="SPEC",
                     help="time the block-sparse backward: causal, full, window:W or "
                          "random:P:SEED over 128x128 tiles (bf16 configs)")
@@ -514,6 +672,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = CONFIGS[args.config]
+    if args.layout != "bhnd" and args.block_mask:
+        ap.error("--layout and --block-mask are separate measurements")
     if args.block_mask:
         if cfg.dtype != "bf16":
             ap.error("--block-mask needs a bf16 config")
@@ -529,7 +689,10 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, cfg, world, rank, local)
+        if args.layer:
+            run_layer(args, cfg, world, rank, local)
+        else:
+            run_gpu(args, cfg, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

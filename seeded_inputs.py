@@ -149,3 +149,17 @@ def block_mask_pairs(mask: np.ndarray) -> float:
     N = 128 T positions counts N^2 / 2)."""
     m = np.asarray(mask)
     return float(TILE * TILE * (np.count_nonzero(m == 1) + 0.5 * np.count_nonzero(m == 2)))
+
+
+def draw_layer(B: int, N: int, C: int, seed: int, dtype: str = "bf16"):
+    """Inputs of one attention layer: x, dy ~ N(0, 1) [B, N, C] and weights
+    W_qkv [C, 3C], W_o [C, C] ~ N(0, 1/C), drawn in that order from one seeded
+    CPU generator (float32, then rounded like `draw`)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    x = torch.randn(B, N, C, generator=g)
+    w_qkv = torch.randn(C, 3 * C, generator=g) / math.sqrt(C)
+    w_o = torch.randn(C, C, generator=g) / math.sqrt(C)
+    dy = torch.randn(B, N, C, generator=g)
+    if dtype == "bf16":
+        x, w_qkv, w_o, dy = (t.to(torch.bfloat16) for t in (x, w_qkv, w_o, dy))
+    return x, w_qkv, w_o, dy

@@ -341,6 +341,25 @@ def test_strided_ddx_issue217_tables_against_the_oracle(csa):
         assert rel(as_f64(t.cpu()), ref[name], gscale) <= 1e-5, name
 
 
+@pytest.mark.parametrize("B,N,C,H", [(12, 64, 128, 4), (2, 1000, 512, 4), (1, 700, 1024, 8)])
+def test_mha_layer_step_against_the_oracle(csa, B, N, C, H):
+    # the first shape is ddx issue #217's nanoGPT-shaped layer (batch 12,
+    # 64 positions, 128 channels, 4 heads); bf16 storage between the steps
+    from causal_softmax_attention_b200 import layer
+    from seeded_inputs import draw_layer
+    x, w_qkv, w_o, dy = draw_layer(B, N, C, 400 + C)
+    ref = oracle.mha_layer(as_f64(x), as_f64(w_qkv), as_f64(w_o), as_f64(dy), H)
+    dev = torch.device("cuda")
+    xd, wq, wo, dyd = (t.to(dev) for t in (x, w_qkv, w_o, dy))
+    y, saved = layer.layer_forward(xd, wq, wo, H)
+    dx, dwq, dwo = layer.layer_backward(dyd, saved, wq, wo, H)
+    torch.cuda.synchronize()
+    assert csa.attn_fwd_last_status() == 0
+    for name, got in (("y", y), ("dx", dx), ("dW_qkv", dwq), ("dW_o", dwo)):
+        e = rel(as_f64(got.cpu()), ref[name])
+        assert e <= TOL["bf16"], (name, e)
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")

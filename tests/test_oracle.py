@@ -388,3 +388,61 @@ def test_torch_autograd_cross_check_block_mask():
     for name, g in (("dQ", tq.grad), ("dK", tk.grad), ("dV", tv.grad)):
         assert rel(out[name], g.numpy()) <= 1e-12
     assert np.all(out["LSE"][:, :, 128:256] == -np.inf)
+
+
+# ---------------------------------------------------------------- MHA layer
+def _torch_layer(x, w_qkv, w_o, dy, H):
+    """The same layer through torch float64 autograd, written separately:
+    heads split with view/transpose, softmax by torch, causal mask by tril."""
+    x, w_qkv, w_o = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (x, w_qkv, w_o))
+    B, N, C = x.shape
+    d = C // H
+    qkv = x @ w_qkv
+    q, k, v = (qkv[..., c * C:(c + 1) * C].view(B, N, H, d).transpose(1, 2) for c in range(3))
+    s = (q @ k.transpose(-1, -2)) / d ** 0.5
+    s = s.masked_fill(~torch.ones(N, N, dtype=torch.bool).tril(), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    y = o.transpose(1, 2).reshape(B, N, C) @ w_o
+    (y * torch.tensor(dy)).sum().backward()
+    return y.detach().numpy(), x.grad.numpy(), w_qkv.grad.numpy(), w_o.grad.numpy()
+
+
+def test_mha_layer_against_torch_autograd():
+    r = np.random.default_rng(11)
+    B, N, H, d = 3, 10, 2, 4
+    C = H * d
+    x = r.standard_normal((B, N, C))
+    w_qkv = r.standard_normal((C, 3 * C)) / np.sqrt(C)
+    w_o = r.standard_normal((C, C)) / np.sqrt(C)
+    dy = r.standard_normal((B, N, C))
+    out = oracle.mha_layer(x, w_qkv, w_o, dy, H)
+    y, dx, dwq, dwo = _torch_layer(x, w_qkv, w_o, dy, H)
+    for name, ref in (("y", y), ("dx", dx), ("dW_qkv", dwq), ("dW_o", dwo)):
+        np.testing.assert_allclose(out[name], ref, rtol=1e-11, atol=1e-12, err_msg=name)
+
+
+def test_mha_layer_finite_differences():
+    r = np.random.default_rng(12)
+    B, N, H, d = 1, 5, 2, 3
+    C = H * d
+    x = r.standard_normal((B, N, C))
+    w_qkv = r.standard_normal((C, 3 * C)) / np.sqrt(C)
+    w_o = r.standard_normal((C, C)) / np.sqrt(C)
+    dy = r.standard_normal((B, N, C))
+    out = oracle.mha_layer(x, w_qkv, w_o, dy, H)
+
+    def loss(x_, wq_, wo_):
+        return float((oracle.mha_layer(x_, wq_, wo_, dy, H)["y"] * dy).sum())
+
+    h = 1e-6
+    for name, arr, idxs in (("dx", x, [(0, 0, 0), (0, 4, 5), (0, 2, 3)]),
+                            ("dW_qkv", w_qkv, [(0, 0), (5, 17), (3, 8)]),
+                            ("dW_o", w_o, [(0, 0), (5, 5), (2, 4)])):
+        for ix in idxs:
+            ap, am = arr.copy(), arr.copy()
+            ap[ix] += h
+            am[ix] -= h
+            args_p = {"dx": (ap, w_qkv, w_o), "dW_qkv": (x, ap, w_o), "dW_o": (x, w_qkv, ap)}[name]
+            args_m = {"dx": (am, w_qkv, w_o), "dW_qkv": (x, am, w_o), "dW_o": (x, w_qkv, am)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - out[name][ix]) <= 1e-6 * max(1.0, np.abs(out[name]).max()), (name, ix)
