@@ -26,6 +26,12 @@ kernels): forward + backward per step, FLOPs = 24*B*N*C^2 for the four
 projections (forward and both backward products) + the attention's causal
 forward and backward.
 
+`--shard-heads` splits ONE problem's (batch, head) pairs over the ranks
+(strong scaling; the long-sequence configuration by default): each rank
+runs the backward of its block of heads, value = the whole problem's FLOPs
+over the slowest rank's step time. `--gather` adds an NCCL all-gather of
+dQ, dK, dV to every rank inside the timed step.
+
 `--block-mask SPEC` (causal, full, window:W, random:P:SEED over 128 x 128
 tiles; bf16) times the block-sparse backward instead: the same three stages
 with the masked main kernel, FLOPs counted over the kept tiles (a kind-1 tile
@@ -316,6 +322,87 @@ def config_dict(cfg, n_gpus, mask_spec=None, layout="bhnd"):
         out["block_mask"] = mask_spec
         out["kept_fraction_of_causal"] = block_mask_pairs(bm) / (cfg.N * cfg.N / 2)
     return out
+
+
+# --------------------------------------------------------------------- head-sharded arm
+def run_sharded(args, cfg, world, rank, local):
+    import causal_softmax_attention_b200 as csa
+    from causal_softmax_attention_b200.shard import (backward_shard, gather_heads, head_block,
+                                                     head_range)
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
+    start, end = head_range(B * H, world, rank)
+    nh = end - start
+    # every rank draws the same problem and keeps its own heads on the device
+    full = draw(B, H, N, d, cfg.seed, cfg.dtype, cfg.qk_gain)
+    q, k, v, do = (torch.zeros(B, H, N, d, dtype=t.dtype, device=dev) for t in full)
+    for dst, src in zip((q, k, v, do), full):
+        if nh:
+            head_block(dst, start, end).copy_(head_block(src, start, end))
+    del full
+    o = torch.zeros_like(q)
+    lse = torch.zeros(B, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
+    stream = torch.cuda.current_stream(dev)
+    if nh:
+        blk = [head_block(t, start, end) for t in (q, k, v, o, lse)]
+        csa.attn_fwd(*blk, True, cfg.scale, stream)
+    ws = torch.empty(max(1, csa.attn_bwd_workspace_bytes(1, max(nh, 1), N, d, q.dtype)),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        backward_shard(q, k, v, o, do, lse, dq, dk, dv, ws, world, rank, True, cfg.scale,
+                       stream)
+        if args.gather and world > 1:
+            for t in (dq, dk, dv):
+                t.copy_(gather_heads(t, world, rank))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        time.sleep(1.0)
+        host_t0 = time.time()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        host_t1 = time.time()
+        time.sleep(0.25)
+    barrier(world)
+    ms_per_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    flops = cfg.bwd_flops  # the whole problem, shared out
+    value = flops / (ms_per_step * 1e-3) / 1e12
+    if nh and csa.attn_last_status(ws) != 0:
+        raise RuntimeError("device status after the sharded steps")
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic",
+        "config": dict(config_dict(cfg, world), parallelism=f"heads sharded over {world} ranks"
+                       + (", dQ/dK/dV all-gathered (NCCL) in the step" if args.gather else "")),
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak,
+                     "unit": "TFLOP/s", "frac": value / world / peak, "traffic": None,
+                     "kernel": "attn_bwd per rank (preprocess, main, dQ convert)"
+                               + (" + all-gather" if args.gather else ""),
+                     "peak_source": f"{peak_kind} bf16_tflops (burst), per GPU",
+                     "algorithmic_flops_per_launch": flops / world, "avg_launch_ms": ms_per_step},
+        "e2e": None,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(host_t0, host_t1),
+        "heads_per_rank": -(-(B * H) // world),
+    }
+    print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------------------- layer arm
@@ -661,6 +748,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head groups of the end-to-end (host-buffer) measurement")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="split one problem's heads over the ranks (strong scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard-heads: all-gather dQ, dK, dV inside the step")
     ap.add_argument("--layer", action="store_true",
                     help="time one attention layer step (projections + attention, fwd + bwd)")
     ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd", "packed"],
@@ -671,6 +762,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.shard_heads and "--config" not in sys.argv:
+        args.config = "c5"  # the long-sequence problem is the one worth sharding
     cfg = CONFIGS[args.config]
     if args.layout != "bhnd" and args.block_mask:
         ap.error("--layout and --block-mask are separate measurements")
@@ -691,6 +784,8 @@ def main():
     try:
         if args.layer:
             run_layer(args, cfg, world, rank, local)
+        elif args.shard_heads:
+            run_sharded(args, cfg, world, rank, local)
         else:
             run_gpu(args, cfg, world, rank, local)
     finally:

@@ -54,3 +54,71 @@ def test_single_rank_defaults(monkeypatch):
     assert bench.dist_env() == (1, 0, 0)
     assert bench.max_over_ranks(3.0, 1) == 3.0
     assert bench.whole_job_tflops(1e12, 1, 1.0) == pytest.approx(1000.0)
+
+
+def test_head_ranges_cover_every_head_once():
+    from causal_softmax_attention_b200.shard import head_range
+    for BH in (1, 3, 4, 7, 32, 33):
+        for world in (1, 2, 3, 4, 8):
+            seen = []
+            for r in range(world):
+                s, e = head_range(BH, world, r)
+                assert 0 <= s <= e <= BH
+                assert e - s <= -(-BH // world)
+                seen.extend(range(s, e))
+            assert seen == list(range(BH)), (BH, world)
+
+
+def _gather_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from causal_softmax_attention_b200.shard import gather_heads, head_block, head_range
+        B, H, N, d = 2, 3, 5, 4
+        full = torch.arange(B * H * N * d, dtype=torch.float32).reshape(B, H, N, d)
+        mine = torch.full_like(full, -1.0)
+        s, e = head_range(B * H, world, rank)
+        head_block(mine, s, e).copy_(head_block(full, s, e))  # this rank's "result"
+        got = gather_heads(mine, world, rank)
+        q.put((rank, bool(torch.equal(got, full)), (s, e)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gather_heads_reassembles_the_blocks(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok, _ in res), res
+
+
+def test_backward_shard_hands_each_rank_its_block(monkeypatch):
+    # the views passed to attn_bwd: [1, heads of the rank, N, d] starting at
+    # the rank's first head, for every tensor (no GPU: attn_bwd is recorded)
+    import causal_softmax_attention_b200 as csa
+    from causal_softmax_attention_b200 import shard
+    calls = []
+    monkeypatch.setattr(csa, "attn_bwd", lambda *a, **k: calls.append(a))
+    B, H, N, d = 2, 3, 4, 8
+    ts = [torch.randn(B, H, N, d) for _ in range(5)] + [torch.randn(B, H, N)] + \
+         [torch.zeros(B, H, N, d) for _ in range(3)]
+    for world in (1, 2, 4, 8):
+        for rank in range(world):
+            calls.clear()
+            s, e = shard.backward_shard(*ts, "ws", world, rank)
+            if e == s:
+                assert not calls
+                continue
+            (args,) = calls
+            for t, blk in zip(ts, args[:9]):
+                assert blk.shape == (1, e - s) + tuple(t.shape[2:])
+                assert blk.data_ptr() == t.reshape(B * H, *t.shape[2:])[s].data_ptr()
+            assert args[9] == "ws"
