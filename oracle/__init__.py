@@ -8,3 +8,4 @@ from .attention_f64 import (  # noqa: F401
     block_mask_keep, causal_pair_count, forward, forward_head, keep_mask, key_tail, query_rows,
 )
 from .mha_layer_f64 import layer as mha_layer  # noqa: F401,E402
+from .double_backward_f64 import double_backward, double_backward_head  # noqa: F401,E402

@@ -446,3 +446,59 @@ def test_mha_layer_finite_differences():
             args_m = {"dx": (am, w_qkv, w_o), "dW_qkv": (x, am, w_o), "dW_o": (x, w_qkv, am)}[name]
             fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
             assert abs(fd - out[name][ix]) <= 1e-6 * max(1.0, np.abs(out[name]).max()), (name, ix)
+
+
+# ------------------------------------------------- backward-over-backward
+def _bob_inputs(seed, n=7, d=3):
+    r = np.random.default_rng(seed)
+    return [r.standard_normal((n, d)) for _ in range(7)]
+
+
+def _l2(q, k, v, do, uq, uk, uv, scale, causal):
+    g = A.backward_head(q, k, v, do, scale, causal)
+    return float((uq * g["dQ"]).sum() + (uk * g["dK"]).sum() + (uv * g["dV"]).sum())
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_double_backward_finite_differences(causal):
+    q, k, v, do, uq, uk, uv = _bob_inputs(21 + causal)
+    scale = 0.6
+    out = oracle.double_backward_head(q, k, v, do, uq, uk, uv, scale, causal)
+    h = 1e-6
+    args = [q, k, v, do]
+    for idx, name in enumerate(("gQ", "gK", "gV", "gdO")):
+        fd = np.zeros_like(args[idx])
+        for ix in np.ndindex(*fd.shape):
+            ap = [a.copy() for a in args]
+            am = [a.copy() for a in args]
+            ap[idx][ix] += h
+            am[idx][ix] -= h
+            fd[ix] = (_l2(*ap, uq, uk, uv, scale, causal) - _l2(*am, uq, uk, uv, scale, causal)) / (2 * h)
+        err = np.abs(fd - out[name]).max()
+        assert err <= 1e-7 * max(1.0, np.abs(out[name]).max()), (name, err)
+
+
+def test_double_backward_against_torch_double_backward():
+    q, k, v, do, uq, uk, uv = (torch.tensor(a) for a in _bob_inputs(23, n=9, d=4))
+    scale = 0.5
+    out = oracle.double_backward_head(*(t.numpy() for t in (q, k, v, do, uq, uk, uv)), scale, True)
+    q, k, v, do = (t.clone().requires_grad_(True) for t in (q, k, v, do))
+    n = q.shape[0]
+    s = (q @ k.T) * scale
+    s = s.masked_fill(~torch.ones(n, n, dtype=torch.bool).tril(), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    dq, dk, dv = torch.autograd.grad(o, (q, k, v), do, create_graph=True)
+    l2 = (uq * dq).sum() + (uk * dk).sum() + (uv * dv).sum()
+    gq, gk, gv, gdo = torch.autograd.grad(l2, (q, k, v, do))
+    for name, t in (("gQ", gq), ("gK", gk), ("gV", gv), ("gdO", gdo)):
+        np.testing.assert_allclose(out[name], t.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+
+
+def test_double_backward_is_linear_in_the_cotangents():
+    q, k, v, do, uq, uk, uv = _bob_inputs(24)
+    a = oracle.double_backward_head(q, k, v, do, uq, uk, uv, 0.7)
+    b = oracle.double_backward_head(q, k, v, do, 2 * uq, 2 * uk, 2 * uv, 0.7)
+    z = oracle.double_backward_head(q, k, v, do, 0 * uq, 0 * uk, 0 * uv, 0.7)
+    for name in ("gQ", "gK", "gV", "gdO"):
+        np.testing.assert_allclose(b[name], 2 * a[name], rtol=1e-12, atol=1e-13)
+        assert np.abs(z[name]).max() == 0.0
