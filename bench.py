@@ -32,6 +32,11 @@ runs the backward of its block of heads, value = the whole problem's FLOPs
 over the slowest rank's step time. `--gather` adds an NCCL all-gather of
 dQ, dK, dV to every rank inside the timed step.
 
+`--bob` times the backward-over-backward (fp32 FFMA kernels; the fp32
+256-token configuration by default): FLOPs counted as its 12 matrix products
+per kept score pair (24*d per pair, 12*B*H*N^2*d causal), against the
+derived FFMA peak.
+
 `--block-mask SPEC` (causal, full, window:W, random:P:SEED over 128 x 128
 tiles; bf16) times the block-sparse backward instead: the same three stages
 with the masked main kernel, FLOPs counted over the kept tiles (a kind-1 tile
@@ -405,6 +410,113 @@ def run_sharded(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------- backward-over-backward arm
+def run_bob(args, cfg, world, rank, local):
+    import causal_softmax_attention_b200 as csa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
+    ins = draw(B, H, N, d, cfg.seed + 1000 * rank, "f32", cfg.qk_gain)
+    cots = draw(B, H, N, d, cfg.seed + 1000 * rank + 500, "f32")[:3]
+    host = [t.pin_memory() for t in ins + cots]
+    q, k, v, do, uq, uk, uv = (t.to(dev) for t in host)
+    o, lse = csa.forward(q, k, v, True, cfg.scale)
+    outs = [torch.empty_like(q) for _ in range(4)]
+    ws = torch.empty(csa.library().attn_bwd_bwd_workspace_bytes(B, H, N, d, csa.ATTN_F32),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = 12.0 * B * H * N * N * d
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        csa.attn_bwd_bwd(q, k, v, o, do, lse, uq, uk, uv, *outs, ws, True, cfg.scale, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        time.sleep(1.0)
+        host_t0 = time.time()
+        for i in range(args.steps):
+            flush.zero_()  # between steps, outside the step's events
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        host_t1 = time.time()
+        time.sleep(0.25)
+    ms_per_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps,
+                                 world)
+    value = whole_job_tflops(flops, world, ms_per_step)
+    # e2e: the seven inputs and O, LSE from pinned host memory, the four
+    # gradients back, serialised with the call
+    h_o, h_lse = o.cpu().pin_memory(), lse.cpu().pin_memory()
+    dev_in, host_in = [q, k, v, do, uq, uk, uv, o, lse], host + [h_o, h_lse]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+
+    def e2e_step():
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(host_out, outs):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, world)
+    if rank != 0:
+        return
+    if csa.attn_last_status(ws) != 0:
+        raise RuntimeError("device status after the double-backward steps")
+    peaks, _ = load_peaks()
+    ffma = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    line = {
+        "metric": "causal attention backward-over-backward TFLOP/s (fp32, 1xB200)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(config_dict(cfg, world), workload=f"{cfg.name}: causal attention "
+                       f"backward-over-backward B={B} H={H} N={N} d={d} f32, q,k,v,dO,U ~ N(0,1)"),
+        "roofline": {"bound": "alu", "achieved": value / world, "peak": ffma, "unit": "TFLOP/s",
+                     "frac": value / world / ffma, "traffic": None,
+                     "kernel": "bob_rows_f32_kernel + bob_cols_f32_kernel (+ preprocess)",
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x sm_max_mhz",
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": ms_per_step,
+                     "flops_convention": "12 matrix products per kept pair (24*d), causal N^2/2"},
+        "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(host_t0, host_t1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        from seeded_inputs import as_f64
+        a = [as_f64(t) for t in ins + cots]
+        t0 = time.perf_counter()
+        n_runs = 0
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.double_backward(*a, cfg.scale, True)
+            n_runs += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": flops * n_runs / el / 1e12, "unit": "TFLOP/s",
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"oracle double_backward (numpy float64) on the whole "
+                                          f"workload, {n_runs} runs in {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------------------- layer arm
 def run_layer(args, cfg, world, rank, local):
     import causal_softmax_attention_b200 as csa
@@ -752,6 +864,8 @@ def main():
                     help="split one problem's heads over the ranks (strong scaling)")
     ap.add_argument("--gather", action="store_true",
                     help="with --shard-heads: all-gather dQ, dK, dV inside the step")
+    ap.add_argument("--bob", action="store_true",
+                    help="time the backward-over-backward (fp32)")
     ap.add_argument("--layer", action="store_true",
                     help="time one attention layer step (projections + attention, fwd + bwd)")
     ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd", "packed"],
@@ -764,6 +878,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.shard_heads and "--config" not in sys.argv:
         args.config = "c5"  # the long-sequence problem is the one worth sharding
+    if args.bob and "--config" not in sys.argv:
+        args.config = "c1"  # the fp32 kernels' configuration
     cfg = CONFIGS[args.config]
     if args.layout != "bhnd" and args.block_mask:
         ap.error("--layout and --block-mask are separate measurements")
@@ -786,6 +902,8 @@ def main():
             run_layer(args, cfg, world, rank, local)
         elif args.shard_heads:
             run_sharded(args, cfg, world, rank, local)
+        elif args.bob:
+            run_bob(args, cfg, world, rank, local)
         else:
             run_gpu(args, cfg, world, rank, local)
     finally:

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "attn_bwd_main_masked": (i, [vp] * 7 + [i, i, i, i, vp, f, i, vp, sz, vp]),
         "attn_fwd_strided": (i, [vp] * 5 + [i, i, i, i, vp, vp, i, f, i, vp]),
         "attn_bwd_strided": (i, [vp] * 9 + [i, i, i, i, vp, vp, i, f, i, vp, sz, vp]),
+        "attn_bwd_bwd_workspace_bytes": (sz, [i, i, i, i, i]),
+        "attn_bwd_bwd": (i, [vp] * 13 + [i, i, i, i, i, f, i, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -70,7 +72,8 @@ _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
             "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc", "attn_fwd_masked",
-            "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided")
+            "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided",
+            "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd")
 
 
 def library() -> ctypes.CDLL:
@@ -249,6 +252,34 @@ def attn_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal: bool 
     if check:
         _check(st, "attn_bwd_strided")
     return st
+
+
+def attn_bwd_bwd(q, k, v, o, dout, lse, uq, uk, uv, gq, gk, gv, gdout, workspace,
+                 causal: bool = True, scale: float | None = None, stream=None,
+                 check: bool = True) -> int:
+    """Backward-over-backward: gq, gk, gv, gdout <- the gradients of
+    <uq, dQ> + <uk, dK> + <uv, dV> w.r.t. q, k, v, dout (f32)."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_bwd_bwd(*(_ptr(t) for t in (q, k, v, o, dout, lse, uq, uk, uv, gq, gk, gv,
+                                               gdout)),
+                           B, H, N, d, int(causal), float(scale), _DTYPES[q.dtype],
+                           _ptr(workspace), int(workspace.numel()), _stream(stream))
+    if check:
+        _check(st, "attn_bwd_bwd")
+    return st
+
+
+def backward_over_backward(q, k, v, o, dout, lse, uq, uk, uv, causal: bool = True,
+                           scale: float | None = None):
+    """Convenience: allocate the outputs and a workspace, run attn_bwd_bwd."""
+    B, H, N, d = _shape(q)
+    out = [torch.empty_like(q) for _ in range(4)]
+    ws = torch.empty(max(1, int(_lib.attn_bwd_bwd_workspace_bytes(B, H, N, d,
+                                                                  _DTYPES[q.dtype]))),
+                     dtype=torch.uint8, device=q.device)
+    attn_bwd_bwd(q, k, v, o, dout, lse, uq, uk, uv, *out, ws, causal, scale)
+    return tuple(out)
 
 
 def forward(q, k, v, causal: bool = True, scale: float | None = None):

@@ -377,6 +377,50 @@ int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
                   workspace_bytes, nullptr, qs, os, stream);
 }
 
+// Backward-over-backward: the f32 backward's workspace (status, padded LSE,
+// D) followed by the two row scalars r and g, [BH][Np] floats each.
+namespace {
+size_t bob_extra_off(int B, int H, int N, int d) {
+  return (workspace_layout(B, H, N, d, ATTN_F32).total + 255) / 256 * 256;
+}
+}  // namespace
+
+size_t attn_bwd_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
+  if (check_shape(B, H, N, d, dtype) != ATTN_OK || dtype != ATTN_F32) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * round_up(N, kTile);
+  return bob_extra_off(B, H, N, d) + 2 * ((rows * sizeof(float) + 255) / 256 * 256);
+}
+
+int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, const void* uq, const void* uk, const void* uv, void* gq,
+                 void* gk, void* gv, void* gdout, int B, int H, int N, int d, int causal,
+                 float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!tensors_aligned(ATTN_F32, {q, k, v, o, dout, uq, uk, uv, gq, gk, gv, gdout}) ||
+      !all_aligned({lse}))
+    return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+  int st = check_shape(B, H, N, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      workspace_bytes < attn_bwd_bwd_workspace_bytes(B, H, N, d, dtype))
+    return ATTN_ERR_INVALID;
+  st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes,
+                       dense(H, N, d), stream);
+  if (st != ATTN_OK) return st;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  const size_t rows = static_cast<size_t>(B) * H * ws.Np;
+  float* r_pad = reinterpret_cast<float*>(static_cast<char*>(workspace) + bob_extra_off(B, H, N, d));
+  float* g_pad =
+      reinterpret_cast<float*>(reinterpret_cast<char*>(r_pad) + (rows * sizeof(float) + 255) / 256 * 256);
+  return from_cuda(launch_bob_f32(
+      static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+      static_cast<const float*>(dout), static_cast<const float*>(uq),
+      static_cast<const float*>(uk), static_cast<const float*>(uv), static_cast<float*>(gq),
+      static_cast<float*>(gk), static_cast<float*>(gv), static_cast<float*>(gdout), B * H, N, d,
+      causal != 0, scale, ws, r_pad, g_pad, static_cast<cudaStream_t>(stream)));
+}
+
 int attn_last_status(const void* workspace) {
   if (workspace == nullptr) return ATTN_ERR_INVALID;
   int v = 0;

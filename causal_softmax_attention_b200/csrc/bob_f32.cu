@@ -1,0 +1,256 @@
+// Backward-over-backward of causal softmax attention on the CUDA cores
+// (fp32 FFMA): the gradient of L2 = <U_Q, dQ> + <U_K, dK> + <U_V, dV> with
+// respect to Q, K, V and dO, where (dQ, dK, dV) is attention's first
+// backward. The operation and its shape -- two row-wise scalars, then affine
+// maps of recomputed tiles, in two passes over the scores -- follow the
+// FlashBoB listing ("Approaching I/O-optimality for Approximate Attention",
+// abstract). Per score pair (i, j), recomputed from the rows alone:
+//
+//   P  = exp(s q_i.k_j - LSE_i)         dP = dO_i.v_j
+//   M  = s (u_Q,i . k_j + q_i . u_K,j)  W  = dO_i . u_V,j
+//   row scalars  r_i = sum_j P M,  g_i = sum_j P (M dP) - 2 r_i D_i + sum_j P W
+//   dS = P (dP - D_i)   E = P (M - r_i)   dS2 = P (M (dP - D_i) - r_i dP + W - g_i)
+//
+//   gQ_i  = s sum_j (dS u_K,j + dS2 k_j)     gdO_i = sum_j (E v_j + P u_V,j)
+//   gK_j  = s sum_i (dS u_Q,i + dS2 q_i)     gV_j  = sum_i E dO_i
+//
+// (D_i = sum_c dO_ic O_ic from the first backward's preprocess.) Kernel 1
+// owns query rows: a first sweep over the key tiles accumulates r and g, a
+// second accumulates gQ and gdO, and r, g go to the workspace. Kernel 2 owns
+// key rows and accumulates gK and gV over the query tiles. No atomics: the
+// results are deterministic. Each thread holds 16 channels of its row's
+// vectors; TPR = DP/16 threads share a row and finish dot products with
+// shuffles, the other side streams through shared memory 16 rows at a time.
+#include "common.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kCpt = 16;   // channels per thread
+constexpr int kRows = 16;  // rows of the streamed side per shared-memory tile
+
+template <int TPR>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int off = 1; off < TPR; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// rows [r0, r0 + kRows) x channels [0, DP) of an [N][d] fp32 head (rows d
+// apart) into shared memory; rows >= N and channels >= d read as zero
+template <int DP>
+__device__ __forceinline__ void stage(float (*dst)[DP], const float* src, int r0, int N, int d) {
+  for (int idx = threadIdx.x; idx < kRows * DP; idx += blockDim.x) {
+    const int r = idx / DP, c = idx % DP;
+    dst[r][c] = (r0 + r < N && c < d) ? src[static_cast<size_t>(r0 + r) * d + c] : 0.f;
+  }
+}
+
+template <int DP>
+__device__ __forceinline__ void load_row(float (&dst)[kCpt], const float* src, int row, int N,
+                                         int d, int part) {
+#pragma unroll
+  for (int c = 0; c < kCpt; ++c) {
+    const int ch = kCpt * part + c;
+    dst[c] = (row < N && ch < d) ? src[static_cast<size_t>(row) * d + ch] : 0.f;
+  }
+}
+
+template <int DP>
+__device__ __forceinline__ float dot(const float (&a)[kCpt], const float (*tile)[DP], int u,
+                                     int part) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < kCpt; ++c) s = fmaf(a[c], tile[u][kCpt * part + c], s);
+  return s;
+}
+
+template <int DP>
+__device__ __forceinline__ void store_row(float* dst, const float (&a)[kCpt], float mul, int row,
+                                          int N, int d, int part) {
+  if (row >= N) return;
+#pragma unroll
+  for (int c = 0; c < kCpt; ++c) {
+    const int ch = kCpt * part + c;
+    if (ch < d) dst[static_cast<size_t>(row) * d + ch] = a[c] * mul;
+  }
+}
+
+struct BobArgs {
+  const float *q, *k, *v, *dout, *uq, *uk, *uv;
+  float *gq, *gk, *gv, *gdout;
+  const float *lse_pad, *d_pad;  // [BH][Np]: LSE (+inf past N), D (0 past N)
+  float *r_pad, *g_pad;          // [BH][Np]: the two row scalars (0 past N)
+  int N, Np, d, causal;
+  float scale;
+};
+
+// ------------------------------------------------------------ query rows
+template <int DP>
+__global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
+  constexpr int TPR = DP / kCpt;
+  constexpr int R = 128 / TPR;
+  __shared__ float sK[kRows][DP], sV[kRows][DP], sUK[kRows][DP], sUV[kRows][DP];
+  const int bh = blockIdx.y;
+  const int row = blockIdx.x * R + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
+  const size_t off = static_cast<size_t>(bh) * a.N * a.d;
+  const float *kh = a.k + off, *vh = a.v + off, *ukh = a.uk + off, *uvh = a.uv + off;
+  float qr[kCpt], dor[kCpt], uqr[kCpt];
+  load_row<DP>(qr, a.q + off, row, a.N, a.d, part);
+  load_row<DP>(dor, a.dout + off, row, a.N, a.d, part);
+  load_row<DP>(uqr, a.uq + off, row, a.N, a.d, part);
+  const size_t prow = static_cast<size_t>(bh) * a.Np + min(row, a.Np - 1);
+  const float L = row < a.N ? a.lse_pad[prow] : INFINITY;
+  const float D = row < a.N ? a.d_pad[prow] : 0.f;
+  const int last_row = min(a.N - 1, static_cast<int>(blockIdx.x) * R + R - 1);
+  const int key_end = a.causal ? last_row + 1 : a.N;
+
+  // one score pair's recomputed quantities
+  auto pair = [&](int u, int key, float& p, float& dp, float& m, float& w) {
+    const float sc = group_sum<TPR>(dot<DP>(qr, sK, u, part)) * a.scale;
+    dp = group_sum<TPR>(dot<DP>(dor, sV, u, part));
+    m = group_sum<TPR>(dot<DP>(uqr, sK, u, part) + dot<DP>(qr, sUK, u, part)) * a.scale;
+    w = group_sum<TPR>(dot<DP>(dor, sUV, u, part));
+    const bool keep = row < a.N && key < a.N && (!a.causal || key <= row);
+    p = keep ? expf(sc - L) : 0.f;
+  };
+
+  // sweep 1: the row scalars
+  float r = 0.f, t1 = 0.f, t3 = 0.f;
+  for (int k0 = 0; k0 < key_end; k0 += kRows) {
+    __syncthreads();
+    stage<DP>(sK, kh, k0, a.N, a.d);
+    stage<DP>(sV, vh, k0, a.N, a.d);
+    stage<DP>(sUK, ukh, k0, a.N, a.d);
+    stage<DP>(sUV, uvh, k0, a.N, a.d);
+    __syncthreads();
+    for (int u = 0; u < kRows; ++u) {
+      float p, dp, m, w;
+      pair(u, k0 + u, p, dp, m, w);
+      r = fmaf(p, m, r);
+      t1 = fmaf(p * m, dp, t1);
+      t3 = fmaf(p, w, t3);
+    }
+  }
+  const float g = t1 - 2.f * r * D + t3;
+
+  // sweep 2: gQ and gdO
+  float gq[kCpt], gdo[kCpt];
+#pragma unroll
+  for (int c = 0; c < kCpt; ++c) gq[c] = gdo[c] = 0.f;
+  for (int k0 = 0; k0 < key_end; k0 += kRows) {
+    __syncthreads();
+    stage<DP>(sK, kh, k0, a.N, a.d);
+    stage<DP>(sV, vh, k0, a.N, a.d);
+    stage<DP>(sUK, ukh, k0, a.N, a.d);
+    stage<DP>(sUV, uvh, k0, a.N, a.d);
+    __syncthreads();
+    for (int u = 0; u < kRows; ++u) {
+      float p, dp, m, w;
+      pair(u, k0 + u, p, dp, m, w);
+      const float ds = p * (dp - D);
+      const float e = p * (m - r);
+      const float ds2 = p * (m * (dp - D) - r * dp + w - g);
+#pragma unroll
+      for (int c = 0; c < kCpt; ++c) {
+        const int ch = kCpt * part + c;
+        gq[c] = fmaf(ds, sUK[u][ch], fmaf(ds2, sK[u][ch], gq[c]));
+        gdo[c] = fmaf(e, sV[u][ch], fmaf(p, sUV[u][ch], gdo[c]));
+      }
+    }
+  }
+  store_row<DP>(a.gq + off, gq, a.scale, row, a.N, a.d, part);
+  store_row<DP>(a.gdout + off, gdo, 1.f, row, a.N, a.d, part);
+  if (part == 0 && row < a.Np) {
+    a.r_pad[prow] = row < a.N ? r : 0.f;
+    a.g_pad[prow] = row < a.N ? g : 0.f;
+  }
+}
+
+// ------------------------------------------------------------ key rows
+template <int DP>
+__global__ void __launch_bounds__(128) bob_cols_f32_kernel(const BobArgs a) {
+  constexpr int TPR = DP / kCpt;
+  constexpr int R = 128 / TPR;
+  __shared__ float sQ[kRows][DP], sdO[kRows][DP], sUQ[kRows][DP];
+  __shared__ float sL[kRows], sD[kRows], sR[kRows], sG[kRows];
+  const int bh = blockIdx.y;
+  const int key = blockIdx.x * R + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
+  const size_t off = static_cast<size_t>(bh) * a.N * a.d;
+  const size_t poff = static_cast<size_t>(bh) * a.Np;
+  float kr[kCpt], vr[kCpt], ukr[kCpt], uvr[kCpt];
+  load_row<DP>(kr, a.k + off, key, a.N, a.d, part);
+  load_row<DP>(vr, a.v + off, key, a.N, a.d, part);
+  load_row<DP>(ukr, a.uk + off, key, a.N, a.d, part);
+  load_row<DP>(uvr, a.uv + off, key, a.N, a.d, part);
+  float gk[kCpt], gv[kCpt];
+#pragma unroll
+  for (int c = 0; c < kCpt; ++c) gk[c] = gv[c] = 0.f;
+  const int first_key = blockIdx.x * R;
+  const int q_begin = a.causal ? (first_key / kRows) * kRows : 0;
+  for (int q0 = q_begin; q0 < a.N; q0 += kRows) {
+    __syncthreads();
+    stage<DP>(sQ, a.q + off, q0, a.N, a.d);
+    stage<DP>(sdO, a.dout + off, q0, a.N, a.d);
+    stage<DP>(sUQ, a.uq + off, q0, a.N, a.d);
+    if (threadIdx.x < kRows) {
+      const int qi = q0 + threadIdx.x;
+      const bool in = qi < a.N;
+      sL[threadIdx.x] = in ? a.lse_pad[poff + qi] : INFINITY;
+      sD[threadIdx.x] = in ? a.d_pad[poff + qi] : 0.f;
+      sR[threadIdx.x] = in ? a.r_pad[poff + qi] : 0.f;
+      sG[threadIdx.x] = in ? a.g_pad[poff + qi] : 0.f;
+    }
+    __syncthreads();
+    for (int u = 0; u < kRows; ++u) {
+      const int qi = q0 + u;
+      const float sc = group_sum<TPR>(dot<DP>(kr, sQ, u, part)) * a.scale;
+      const float dp = group_sum<TPR>(dot<DP>(vr, sdO, u, part));
+      const float m =
+          group_sum<TPR>(dot<DP>(kr, sUQ, u, part) + dot<DP>(ukr, sQ, u, part)) * a.scale;
+      const float w = group_sum<TPR>(dot<DP>(uvr, sdO, u, part));
+      const bool keep = qi < a.N && key < a.N && (!a.causal || qi >= key);
+      const float p = keep ? expf(sc - sL[u]) : 0.f;
+      const float ds = p * (dp - sD[u]);
+      const float e = p * (m - sR[u]);
+      const float ds2 = p * (m * (dp - sD[u]) - sR[u] * dp + w - sG[u]);
+#pragma unroll
+      for (int c = 0; c < kCpt; ++c) {
+        const int ch = kCpt * part + c;
+        gk[c] = fmaf(ds, sUQ[u][ch], fmaf(ds2, sQ[u][ch], gk[c]));
+        gv[c] = fmaf(e, sdO[u][ch], gv[c]);
+      }
+    }
+  }
+  store_row<DP>(a.gk + off, gk, a.scale, key, a.N, a.d, part);
+  store_row<DP>(a.gv + off, gv, 1.f, key, a.N, a.d, part);
+}
+
+template <int DP>
+cudaError_t bob_dp(const BobArgs& a, int BH, cudaStream_t s) {
+  constexpr int R = 128 / (DP / kCpt);
+  dim3 grid((a.N + R - 1) / R, BH);
+  bob_rows_f32_kernel<DP><<<grid, 128, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bob_cols_f32_kernel<DP><<<grid, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bob_f32(const float* q, const float* k, const float* v, const float* dout,
+                           const float* uq, const float* uk, const float* uv, float* gq,
+                           float* gk, float* gv, float* gdout, int BH, int N, int d, bool causal,
+                           float scale, const Workspace& ws, float* r_pad, float* g_pad,
+                           cudaStream_t s) {
+  BobArgs a{q, k, v, dout, uq, uk, uv, gq, gk, gv, gdout, ws.lse_pad, ws.d_pad,
+            r_pad, g_pad, N, ws.Np, d, causal ? 1 : 0, scale};
+  if (d <= 32) return bob_dp<32>(a, BH, s);
+  if (d <= 64) return bob_dp<64>(a, BH, s);
+  return bob_dp<128>(a, BH, s);
+}
+
+}  // namespace csa

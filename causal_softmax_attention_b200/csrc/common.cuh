@@ -70,6 +70,15 @@ cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const
                            float scale, const RowStrides& qs, const RowStrides& os,
                            const Workspace& ws, cudaStream_t s);
 
+// Backward-over-backward on the CUDA cores (contiguous fp32 [BH][N][d]);
+// needs the preprocess's lse_pad and d_pad in `ws`, and writes the two row
+// scalars to r_pad, g_pad ([BH][Np] each).
+cudaError_t launch_bob_f32(const float* q, const float* k, const float* v, const float* dout,
+                           const float* uq, const float* uk, const float* uv, float* gq,
+                           float* gk, float* gv, float* gdout, int BH, int N, int d, bool causal,
+                           float scale, const Workspace& ws, float* r_pad, float* g_pad,
+                           cudaStream_t s);
+
 // Tensor-core (tcgen05) path; tensor maps are encoded by the caller, each a
 // 4-D map {d, N, H, B} with a box of {min(d, 64), 128, 1, 1}, loaded at
 // coordinates {channel, row, h, b}.

@@ -157,6 +157,30 @@ int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward-over-backward (the FlashBoB listing, "Approaching I/O-optimality
+ * for Approximate Attention": exact differentiation through attention's
+ * backward pass). With (dQ, dK, dV) the first backward of (q, k, v, dout)
+ * and uq, uk, uv cotangents on them, computes the gradients of
+ *     L2 = <uq, dQ> + <uk, dK> + <uv, dV>
+ * with respect to q, k, v and dout:
+ *   gq, gk, gv, gdout : out, DEVICE [B][H][N][d], same dtype as q.
+ * o and lse are the forward's outputs for (q, k, v) (attn_fwd). The scores
+ * are recomputed tile by tile in two passes (two row-wise scalars first,
+ * then the gradients); nothing N x N is stored. f32 only for now (bf16 ->
+ * ATTN_ERR_UNSUPPORTED), 1 <= d <= 128, contiguous [B][H][N][d], pointers
+ * 4-byte aligned, lse and workspace 16-byte aligned.
+ *   workspace : DEVICE scratch of >= attn_bwd_bwd_workspace_bytes bytes
+ *               (0 for an unsupported shape or dtype).
+ * Three stream-ordered kernels: the backward's preprocess (D, padded LSE),
+ * a query-row kernel (row scalars, gq, gdout), a key-row kernel (gk, gv).
+ */
+size_t attn_bwd_bwd_workspace_bytes(int B, int H, int N, int d, int dtype);
+int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, const void* uq, const void* uk, const void* uv, void* gq,
+                 void* gk, void* gv, void* gdout, int B, int H, int N, int d, int causal,
+                 float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The three stages attn_bwd runs, exposed so a caller can time or overlap them
  * separately. Same arguments and checks as attn_bwd; they must be enqueued in
  * this order on one stream with the same workspace.

@@ -64,6 +64,8 @@ CONFIGS = {
     # the d = 64 counterpart (the long-sequence workload's head size), with
     # its q, k scaling; 8 heads of 32,768 tokens
     "prof_d64": AttnConfig("prof_d64", 1, 8, 32768, 64, "bf16", 6, qk_gain=0.5),
+    # backward-over-backward at a length where its fp32 kernels fill the GPU
+    "bob_4k": AttnConfig("bob_4k", 1, 8, 4096, 64, "f32", 7),
 }
 
 

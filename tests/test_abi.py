@@ -176,3 +176,20 @@ def test_row_strides_of_views():
     assert csa.row_strides(qkv[:, :, 1].permute(0, 2, 1, 3)) == (5 * 3 * 4 * 32, 32, 3 * 4 * 32)
     with pytest.raises(ValueError):
         csa.row_strides(x.permute(0, 3, 1, 2))
+
+
+def test_double_backward_entry_point_rejects_bad_arguments():
+    # every call returns during argument checking (no CUDA call)
+    f = L.attn_bwd_bwd
+    assert L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 64, 1) == 0  # bf16: not built
+    need = L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 64, 0)
+    assert need >= 2 * 2 * 384 * 4
+    ptrs = [A] * 13
+    assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 0, A, need - 1, None) == csa.ATTN_ERR_INVALID
+    assert f(*ptrs, 1, 2, 300, 64, 1, math.inf, 0, A, need, None) == csa.ATTN_ERR_INVALID
+    assert f(*ptrs, 1, 2, 300, 200, 1, 0.125, 0, A, need, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(*([A] * 12 + [None]), 1, 2, 300, 64, 1, 0.125, 0, A, need, None) == csa.ATTN_ERR_INVALID
+    assert f(*([A] * 5 + [A + 4] + [A] * 7), 1, 2, 300, 64, 1, 0.125, 0, A, need,
+             None) == csa.ATTN_ERR_INVALID  # lse must be 16-byte aligned
+    assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 0, A + 8, need, None) == csa.ATTN_ERR_INVALID

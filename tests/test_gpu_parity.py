@@ -360,6 +360,25 @@ def test_mha_layer_step_against_the_oracle(csa, B, N, C, H):
         assert e <= TOL["bf16"], (name, e)
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 1, 256, 64, True), (2, 3, 200, 48, True),
+                                             (2, 3, 200, 48, False), (1, 2, 130, 128, True),
+                                             (3, 1, 77, 7, True), (1, 1, 1, 32, True)])
+def test_double_backward_against_the_oracle(csa, B, H, N, d, causal):
+    q, k, v, do = draw(B, H, N, d, 500 + N, "f32")
+    uq, uk, uv, _ = draw(B, H, N, d, 600 + N, "f32")
+    scale = d ** -0.5
+    ref = oracle.double_backward(*(as_f64(t) for t in (q, k, v, do, uq, uk, uv)), scale, causal)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod, uqd, ukd, uvd = (t.to(dev) for t in (q, k, v, do, uq, uk, uv))
+    o, lse = csa.forward(qd, kd, vd, causal, scale)
+    gq, gk, gv, gdo = csa.backward_over_backward(qd, kd, vd, o, dod, lse, uqd, ukd, uvd, causal,
+                                                 scale)
+    torch.cuda.synchronize()
+    gscale = max(np.abs(ref[n]).max() for n in ("gQ", "gK", "gV", "gdO"))
+    for name, t in (("gQ", gq), ("gK", gk), ("gV", gv), ("gdO", gdo)):
+        assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["f32"], name
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
