@@ -18,15 +18,16 @@
 // owns query rows: a first sweep over the key tiles accumulates r and g, a
 // second accumulates gQ and gdO, and r, g go to the workspace. Kernel 2 owns
 // key rows and accumulates gK and gV over the query tiles. No atomics: the
-// results are deterministic. Each thread holds 16 channels of its row's
-// vectors; TPR = DP/16 threads share a row and finish dot products with
-// shuffles, the other side streams through shared memory 16 rows at a time.
+// results are deterministic. Each thread holds CPT channels of its row's
+// vectors (16, or 8 at d = 128 and for small problems, where twice the CTAs
+// and ~105 instead of ~166 registers win); TPR = DP/CPT threads share a row
+// and finish dot products with shuffles, the other side streams through
+// shared memory 16 rows at a time.
 #include "common.cuh"
 
 namespace csa {
 namespace {
 
-constexpr int kCpt = 16;   // channels per thread
 constexpr int kRows = 16;  // rows of the streamed side per shared-memory tile
 
 template <int TPR>
@@ -46,32 +47,34 @@ __device__ __forceinline__ void stage(float (*dst)[DP], const float* src, int r0
   }
 }
 
-template <int DP>
-__device__ __forceinline__ void load_row(float (&dst)[kCpt], const float* src, int row, int N,
+template <int CPT>
+__device__ __forceinline__ void load_row(float (&dst)[CPT], const float* src, int row, int N,
                                          int d, int part) {
 #pragma unroll
-  for (int c = 0; c < kCpt; ++c) {
-    const int ch = kCpt * part + c;
+  for (int c = 0; c < CPT; ++c) {
+    const int ch = CPT * part + c;
     dst[c] = (row < N && ch < d) ? src[static_cast<size_t>(row) * d + ch] : 0.f;
   }
 }
 
-template <int DP>
-__device__ __forceinline__ float dot(const float (&a)[kCpt], const float (*tile)[DP], int u,
+// four independent partial sums: the chains are a quarter as long, so the
+// latency of one dot product no longer serialises the pair
+template <int DP, int CPT>
+__device__ __forceinline__ float dot(const float (&a)[CPT], const float (*tile)[DP], int u,
                                      int part) {
-  float s = 0.f;
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int c = 0; c < kCpt; ++c) s = fmaf(a[c], tile[u][kCpt * part + c], s);
-  return s;
+  for (int c = 0; c < CPT; ++c) s[c % 4] = fmaf(a[c], tile[u][CPT * part + c], s[c % 4]);
+  return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
-template <int DP>
-__device__ __forceinline__ void store_row(float* dst, const float (&a)[kCpt], float mul, int row,
+template <int CPT>
+__device__ __forceinline__ void store_row(float* dst, const float (&a)[CPT], float mul, int row,
                                           int N, int d, int part) {
   if (row >= N) return;
 #pragma unroll
-  for (int c = 0; c < kCpt; ++c) {
-    const int ch = kCpt * part + c;
+  for (int c = 0; c < CPT; ++c) {
+    const int ch = CPT * part + c;
     if (ch < d) dst[static_cast<size_t>(row) * d + ch] = a[c] * mul;
   }
 }
@@ -86,9 +89,9 @@ struct BobArgs {
 };
 
 // ------------------------------------------------------------ query rows
-template <int DP>
+template <int DP, int CPT>
 __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
-  constexpr int TPR = DP / kCpt;
+  constexpr int TPR = DP / CPT;
   constexpr int R = 128 / TPR;
   __shared__ float sK[kRows][DP], sV[kRows][DP], sUK[kRows][DP], sUV[kRows][DP];
   const int bh = blockIdx.y;
@@ -96,10 +99,10 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
   const int part = threadIdx.x % TPR;
   const size_t off = static_cast<size_t>(bh) * a.N * a.d;
   const float *kh = a.k + off, *vh = a.v + off, *ukh = a.uk + off, *uvh = a.uv + off;
-  float qr[kCpt], dor[kCpt], uqr[kCpt];
-  load_row<DP>(qr, a.q + off, row, a.N, a.d, part);
-  load_row<DP>(dor, a.dout + off, row, a.N, a.d, part);
-  load_row<DP>(uqr, a.uq + off, row, a.N, a.d, part);
+  float qr[CPT], dor[CPT], uqr[CPT];
+  load_row<CPT>(qr, a.q + off, row, a.N, a.d, part);
+  load_row<CPT>(dor, a.dout + off, row, a.N, a.d, part);
+  load_row<CPT>(uqr, a.uq + off, row, a.N, a.d, part);
   const size_t prow = static_cast<size_t>(bh) * a.Np + min(row, a.Np - 1);
   const float L = row < a.N ? a.lse_pad[prow] : INFINITY;
   const float D = row < a.N ? a.d_pad[prow] : 0.f;
@@ -108,10 +111,10 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
 
   // one score pair's recomputed quantities
   auto pair = [&](int u, int key, float& p, float& dp, float& m, float& w) {
-    const float sc = group_sum<TPR>(dot<DP>(qr, sK, u, part)) * a.scale;
-    dp = group_sum<TPR>(dot<DP>(dor, sV, u, part));
-    m = group_sum<TPR>(dot<DP>(uqr, sK, u, part) + dot<DP>(qr, sUK, u, part)) * a.scale;
-    w = group_sum<TPR>(dot<DP>(dor, sUV, u, part));
+    const float sc = group_sum<TPR>(dot<DP, CPT>(qr, sK, u, part)) * a.scale;
+    dp = group_sum<TPR>(dot<DP, CPT>(dor, sV, u, part));
+    m = group_sum<TPR>(dot<DP, CPT>(uqr, sK, u, part) + dot<DP, CPT>(qr, sUK, u, part)) * a.scale;
+    w = group_sum<TPR>(dot<DP, CPT>(dor, sUV, u, part));
     const bool keep = row < a.N && key < a.N && (!a.causal || key <= row);
     p = keep ? expf(sc - L) : 0.f;
   };
@@ -136,9 +139,9 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
   const float g = t1 - 2.f * r * D + t3;
 
   // sweep 2: gQ and gdO
-  float gq[kCpt], gdo[kCpt];
+  float gq[CPT], gdo[CPT];
 #pragma unroll
-  for (int c = 0; c < kCpt; ++c) gq[c] = gdo[c] = 0.f;
+  for (int c = 0; c < CPT; ++c) gq[c] = gdo[c] = 0.f;
   for (int k0 = 0; k0 < key_end; k0 += kRows) {
     __syncthreads();
     stage<DP>(sK, kh, k0, a.N, a.d);
@@ -153,15 +156,15 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
       const float e = p * (m - r);
       const float ds2 = p * (m * (dp - D) - r * dp + w - g);
 #pragma unroll
-      for (int c = 0; c < kCpt; ++c) {
-        const int ch = kCpt * part + c;
+      for (int c = 0; c < CPT; ++c) {
+        const int ch = CPT * part + c;
         gq[c] = fmaf(ds, sUK[u][ch], fmaf(ds2, sK[u][ch], gq[c]));
         gdo[c] = fmaf(e, sV[u][ch], fmaf(p, sUV[u][ch], gdo[c]));
       }
     }
   }
-  store_row<DP>(a.gq + off, gq, a.scale, row, a.N, a.d, part);
-  store_row<DP>(a.gdout + off, gdo, 1.f, row, a.N, a.d, part);
+  store_row<CPT>(a.gq + off, gq, a.scale, row, a.N, a.d, part);
+  store_row<CPT>(a.gdout + off, gdo, 1.f, row, a.N, a.d, part);
   if (part == 0 && row < a.Np) {
     a.r_pad[prow] = row < a.N ? r : 0.f;
     a.g_pad[prow] = row < a.N ? g : 0.f;
@@ -169,9 +172,9 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
 }
 
 // ------------------------------------------------------------ key rows
-template <int DP>
+template <int DP, int CPT>
 __global__ void __launch_bounds__(128) bob_cols_f32_kernel(const BobArgs a) {
-  constexpr int TPR = DP / kCpt;
+  constexpr int TPR = DP / CPT;
   constexpr int R = 128 / TPR;
   __shared__ float sQ[kRows][DP], sdO[kRows][DP], sUQ[kRows][DP];
   __shared__ float sL[kRows], sD[kRows], sR[kRows], sG[kRows];
@@ -180,14 +183,14 @@ __global__ void __launch_bounds__(128) bob_cols_f32_kernel(const BobArgs a) {
   const int part = threadIdx.x % TPR;
   const size_t off = static_cast<size_t>(bh) * a.N * a.d;
   const size_t poff = static_cast<size_t>(bh) * a.Np;
-  float kr[kCpt], vr[kCpt], ukr[kCpt], uvr[kCpt];
-  load_row<DP>(kr, a.k + off, key, a.N, a.d, part);
-  load_row<DP>(vr, a.v + off, key, a.N, a.d, part);
-  load_row<DP>(ukr, a.uk + off, key, a.N, a.d, part);
-  load_row<DP>(uvr, a.uv + off, key, a.N, a.d, part);
-  float gk[kCpt], gv[kCpt];
+  float kr[CPT], vr[CPT], ukr[CPT], uvr[CPT];
+  load_row<CPT>(kr, a.k + off, key, a.N, a.d, part);
+  load_row<CPT>(vr, a.v + off, key, a.N, a.d, part);
+  load_row<CPT>(ukr, a.uk + off, key, a.N, a.d, part);
+  load_row<CPT>(uvr, a.uv + off, key, a.N, a.d, part);
+  float gk[CPT], gv[CPT];
 #pragma unroll
-  for (int c = 0; c < kCpt; ++c) gk[c] = gv[c] = 0.f;
+  for (int c = 0; c < CPT; ++c) gk[c] = gv[c] = 0.f;
   const int first_key = blockIdx.x * R;
   const int q_begin = a.causal ? (first_key / kRows) * kRows : 0;
   for (int q0 = q_begin; q0 < a.N; q0 += kRows) {
@@ -206,37 +209,49 @@ __global__ void __launch_bounds__(128) bob_cols_f32_kernel(const BobArgs a) {
     __syncthreads();
     for (int u = 0; u < kRows; ++u) {
       const int qi = q0 + u;
-      const float sc = group_sum<TPR>(dot<DP>(kr, sQ, u, part)) * a.scale;
-      const float dp = group_sum<TPR>(dot<DP>(vr, sdO, u, part));
+      const float sc = group_sum<TPR>(dot<DP, CPT>(kr, sQ, u, part)) * a.scale;
+      const float dp = group_sum<TPR>(dot<DP, CPT>(vr, sdO, u, part));
       const float m =
-          group_sum<TPR>(dot<DP>(kr, sUQ, u, part) + dot<DP>(ukr, sQ, u, part)) * a.scale;
-      const float w = group_sum<TPR>(dot<DP>(uvr, sdO, u, part));
+          group_sum<TPR>(dot<DP, CPT>(kr, sUQ, u, part) + dot<DP, CPT>(ukr, sQ, u, part)) * a.scale;
+      const float w = group_sum<TPR>(dot<DP, CPT>(uvr, sdO, u, part));
       const bool keep = qi < a.N && key < a.N && (!a.causal || qi >= key);
       const float p = keep ? expf(sc - sL[u]) : 0.f;
       const float ds = p * (dp - sD[u]);
       const float e = p * (m - sR[u]);
       const float ds2 = p * (m * (dp - sD[u]) - sR[u] * dp + w - sG[u]);
 #pragma unroll
-      for (int c = 0; c < kCpt; ++c) {
-        const int ch = kCpt * part + c;
+      for (int c = 0; c < CPT; ++c) {
+        const int ch = CPT * part + c;
         gk[c] = fmaf(ds, sUQ[u][ch], fmaf(ds2, sQ[u][ch], gk[c]));
         gv[c] = fmaf(e, sdO[u][ch], gv[c]);
       }
     }
   }
-  store_row<DP>(a.gk + off, gk, a.scale, key, a.N, a.d, part);
-  store_row<DP>(a.gv + off, gv, 1.f, key, a.N, a.d, part);
+  store_row<CPT>(a.gk + off, gk, a.scale, key, a.N, a.d, part);
+  store_row<CPT>(a.gv + off, gv, 1.f, key, a.N, a.d, part);
 }
 
-template <int DP>
+template <int DP, int CPT>
 cudaError_t bob_dp(const BobArgs& a, int BH, cudaStream_t s) {
-  constexpr int R = 128 / (DP / kCpt);
+  constexpr int R = 128 / (DP / CPT);
   dim3 grid((a.N + R - 1) / R, BH);
-  bob_rows_f32_kernel<DP><<<grid, 128, 0, s>>>(a);
+  bob_rows_f32_kernel<DP, CPT><<<grid, 128, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bob_cols_f32_kernel<DP><<<grid, 128, 0, s>>>(a);
+  bob_cols_f32_kernel<DP, CPT><<<grid, 128, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+// 16 channels per thread while that still gives two CTAs per SM, else 8
+template <int DP>
+cudaError_t bob_pick(const BobArgs& a, int BH, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  constexpr int R16 = 128 / (DP / 16);
+  const long long ctas16 = static_cast<long long>((a.N + R16 - 1) / R16) * BH;
+  if (DP == 128 || ctas16 < 2LL * sms) return bob_dp<DP, 8>(a, BH, s);
+  return bob_dp<DP, 16>(a, BH, s);
 }
 
 }  // namespace
@@ -248,9 +263,9 @@ cudaError_t launch_bob_f32(const float* q, const float* k, const float* v, const
                            cudaStream_t s) {
   BobArgs a{q, k, v, dout, uq, uk, uv, gq, gk, gv, gdout, ws.lse_pad, ws.d_pad,
             r_pad, g_pad, N, ws.Np, d, causal ? 1 : 0, scale};
-  if (d <= 32) return bob_dp<32>(a, BH, s);
-  if (d <= 64) return bob_dp<64>(a, BH, s);
-  return bob_dp<128>(a, BH, s);
+  if (d <= 32) return bob_pick<32>(a, BH, s);
+  if (d <= 64) return bob_pick<64>(a, BH, s);
+  return bob_pick<128>(a, BH, s);
 }
 
 }  // namespace csa
