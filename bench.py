@@ -712,10 +712,8 @@ def run_gpu(args, cfg, world, rank, local):
     value = whole_job_tflops(flops, world, ms_per_step)
 
     # ---- e2e through the public API with pinned host buffers
-    hq, hk, hv, ho, hdo = (t.cpu().pin_memory() for t in (qd, kd, vd, o, dod))
-    hlse = lse.cpu().pin_memory()
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (qd, kd, vd, dod))
     hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ho, hdo, hlse))
     d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
 
     # Host buffers in, host gradients out, through the package's pipelined
@@ -727,12 +725,17 @@ def run_gpu(args, cfg, world, rank, local):
     dev_bufs = {"q": qd, "k": kd, "v": vd, "o": o, "dout": dod, "lse": lse, "dq": dq, "dk": dk,
                 "dv": dv, "workspace": ws_chunk}
 
-    def e2e_step():
-        csa.backward_host(hq, hk, hv, ho, hdo, hlse, hdq, hdk, hdv, dev_bufs, True, cfg.scale,
-                          e2e_chunks, stream, block_mask=mask)
+    # q, k, v, dO cross from the host; O and LSE are recomputed on the device
+    # by each head group's forward (FLOPs still counted for the backward only)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
 
-    e2e_path = (f"backward_host: pinned host buffers, {e2e_chunks} head groups, "
-                "H2D / attn_bwd / D2H overlapped on three streams")
+    def e2e_step():
+        csa.backward_host(hq, hk, hv, None, hdo, None, hdq, hdk, hdv, dev_bufs, True, cfg.scale,
+                          e2e_chunks, stream, block_mask=mask, recompute_forward=True)
+
+    e2e_path = (f"backward_host: pinned host q, k, v, dO in, dQ, dK, dV out, {e2e_chunks} head "
+                "groups, H2D / forward + backward / D2H overlapped on three streams (O and LSE "
+                "recomputed on the device; the forward's FLOPs are not counted)")
     if args.layout != "bhnd":
         # the strided arrays themselves go host -> device -> host around one
         # attn_bwd_strided call (copies serialised with the call)

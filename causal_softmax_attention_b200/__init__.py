@@ -301,7 +301,8 @@ def backward(q, k, v, o, dout, lse, causal: bool = True, scale: float | None = N
 
 
 def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool = True,
-                  scale: float | None = None, chunks: int = 8, stream=None, block_mask=None):
+                  scale: float | None = None, chunks: int = 8, stream=None, block_mask=None,
+                  recompute_forward: bool = False):
     """dQ, dK, dV of inputs held in (pinned) HOST memory, results written to
     host tensors, through attn_bwd with the transfers overlapped.
 
@@ -318,7 +319,10 @@ def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool 
     stream) and `stream` waits for all of it to finish, so events recorded
     on `stream` around the call time the whole transfer and compute. With a
     `block_mask` (a device uint8 [T, T] tensor, as in attn_bwd_masked) each
-    group runs attn_bwd_masked instead and `causal` is ignored.
+    group runs attn_bwd_masked instead and `causal` is ignored. With
+    `recompute_forward` the host O and LSE are not used (ho, hlse may be
+    None): each group's forward runs on the device before its backward, into
+    dev["o"] and dev["lse"], so only q, k, v and dout cross to the device.
     """
     B, H, N, d = _shape(hq)
     BH = B * H
@@ -335,8 +339,8 @@ def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool 
     def rows(t):  # [B, H, ...] -> [B*H, ...]
         return t.reshape(BH, *t.shape[2:])
 
-    names = ("q", "k", "v", "o", "dout", "lse")
-    hosts = dict(zip(names, (hq, hk, hv, ho, hdout, hlse)))
+    names = ("q", "k", "v", "dout") if recompute_forward else ("q", "k", "v", "o", "dout", "lse")
+    hosts = dict(zip(("q", "k", "v", "o", "dout", "lse"), (hq, hk, hv, ho, hdout, hlse)))
     outs = (("dq", hdq), ("dk", hdk), ("dv", hdv))
     done = None
     for c0 in range(0, BH, hc):
@@ -347,7 +351,15 @@ def backward_host(hq, hk, hv, ho, hdout, hlse, hdq, hdk, hdv, dev, causal: bool 
             landed = torch.cuda.Event()
             landed.record(s_in)
         s_run.wait_event(landed)
-        view = {n: rows(dev[n])[c0:c1].unsqueeze(0) for n in names + ("dq", "dk", "dv")}
+        view = {n: rows(dev[n])[c0:c1].unsqueeze(0)
+                for n in ("q", "k", "v", "o", "dout", "lse", "dq", "dk", "dv")}
+        if recompute_forward:
+            if block_mask is None:
+                attn_fwd(view["q"], view["k"], view["v"], view["o"], view["lse"], causal, scale,
+                         s_run)
+            else:
+                attn_fwd_masked(view["q"], view["k"], view["v"], view["o"], view["lse"],
+                                block_mask, scale, s_run)
         if block_mask is None:
             attn_bwd(view["q"], view["k"], view["v"], view["o"], view["dout"], view["lse"],
                      view["dq"], view["dk"], view["dv"], dev["workspace"], causal, scale, s_run)

@@ -89,11 +89,13 @@ def test_f32_shapes(csa, B, H, N, d, causal):
 
 
 # ------------------------------------------------------------------ properties on the GPU
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_backward_host_pipelined_matches_device(csa, dtype):
+@pytest.mark.parametrize("dtype,recompute", [("bf16", False), ("f32", False), ("bf16", True),
+                                             ("f32", True)])
+def test_backward_host_pipelined_matches_device(csa, dtype, recompute):
     # host buffers in and out, heads in groups on three streams: the same
     # gradients as one attn_bwd call on device buffers (dK, dV bit for bit;
-    # dQ up to the order of its fp32 atomic sums)
+    # dQ up to the order of its fp32 atomic sums); with the forward recomputed
+    # on the device per group, O and LSE never cross from the host
     B, H, N, d = 2, 5, 300, 64
     q, k, v, do = draw(B, H, N, d, 77, dtype)
     g = run_gpu(csa, q, k, v, do, True, d ** -0.5)
@@ -106,9 +108,13 @@ def test_backward_host_pipelined_matches_device(csa, dtype):
     bufs.update({n: torch.empty_like(bufs["q"]) for n in ("dq", "dk", "dv")})
     bufs["workspace"] = torch.empty(csa.chunk_workspace_bytes(B, H, N, d, bufs["q"].dtype, 4),
                                     dtype=torch.uint8, device=dev)
-    csa.backward_host(host["q"], host["k"], host["v"], host["o"], host["dout"], host["lse"],
-                      outs["dq"], outs["dk"], outs["dv"], bufs, True, d ** -0.5, chunks=4)
+    csa.backward_host(host["q"], host["k"], host["v"], None if recompute else host["o"],
+                      host["dout"], None if recompute else host["lse"],
+                      outs["dq"], outs["dk"], outs["dv"], bufs, True, d ** -0.5, chunks=4,
+                      recompute_forward=recompute)
     torch.cuda.synchronize()
+    if recompute:
+        assert torch.equal(bufs["o"], g["O"]) and torch.equal(bufs["lse"], g["LSE"])
     assert torch.equal(outs["dk"], g["dK"].cpu())
     assert torch.equal(outs["dv"], g["dV"].cpu())
     ref = as_f64(g["dQ"].cpu())
