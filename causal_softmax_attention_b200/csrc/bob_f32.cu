@@ -15,9 +15,10 @@
 //   gK_j  = s sum_i (dS u_Q,i + dS2 q_i)     gV_j  = sum_i E dO_i
 //
 // (D_i = sum_c dO_ic O_ic from the first backward's preprocess.) Kernel 1
-// owns query rows: a first sweep over the key tiles accumulates r and g, a
-// second accumulates gQ and gdO, and r, g go to the workspace. Kernel 2 owns
-// key rows and accumulates gK and gV over the query tiles. No atomics: the
+// owns query rows: one sweep over the key tiles accumulates r, g and seven
+// vectors that gQ and gdO are affine combinations of (in r and g), and r, g
+// go to the workspace. Kernel 2 owns key rows and accumulates gK and gV over
+// the query tiles. No atomics: the
 // results are deterministic. Each thread holds CPT channels of its row's
 // vectors (16, or 8 at d = 128 and for small problems, where twice the CTAs
 // and ~105 instead of ~166 registers win); TPR = DP/CPT threads share a row
@@ -89,6 +90,12 @@ struct BobArgs {
 };
 
 // ------------------------------------------------------------ query rows
+// One sweep over the key tiles. dS2 needs the complete row scalar g, so
+// instead of a second sweep the row side is kept affine in (r, g): with
+// per-pair scalars p, dP, M, W,
+//   gQ / s = sum p (dP - D) u_K + sum p (M (dP - D) + W) k - r sum p dP k - g sum p k
+//   gdO    = sum p M v - r sum p v + sum p u_V
+// so seven vectors are accumulated and combined once r and g are known.
 template <int DP, int CPT>
 __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
   constexpr int TPR = DP / CPT;
@@ -109,17 +116,9 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
   const int last_row = min(a.N - 1, static_cast<int>(blockIdx.x) * R + R - 1);
   const int key_end = a.causal ? last_row + 1 : a.N;
 
-  // one score pair's recomputed quantities
-  auto pair = [&](int u, int key, float& p, float& dp, float& m, float& w) {
-    const float sc = group_sum<TPR>(dot<DP, CPT>(qr, sK, u, part)) * a.scale;
-    dp = group_sum<TPR>(dot<DP, CPT>(dor, sV, u, part));
-    m = group_sum<TPR>(dot<DP, CPT>(uqr, sK, u, part) + dot<DP, CPT>(qr, sUK, u, part)) * a.scale;
-    w = group_sum<TPR>(dot<DP, CPT>(dor, sUV, u, part));
-    const bool keep = row < a.N && key < a.N && (!a.causal || key <= row);
-    p = keep ? expf(sc - L) : 0.f;
-  };
-
-  // sweep 1: the row scalars
+  float x1[CPT], x2[CPT], x3[CPT], x4[CPT], y1[CPT], y2[CPT], y3[CPT];
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) x1[c] = x2[c] = x3[c] = x4[c] = y1[c] = y2[c] = y3[c] = 0.f;
   float r = 0.f, t1 = 0.f, t3 = 0.f;
   for (int k0 = 0; k0 < key_end; k0 += kRows) {
     __syncthreads();
@@ -129,42 +128,43 @@ __global__ void __launch_bounds__(128) bob_rows_f32_kernel(const BobArgs a) {
     stage<DP>(sUV, uvh, k0, a.N, a.d);
     __syncthreads();
     for (int u = 0; u < kRows; ++u) {
-      float p, dp, m, w;
-      pair(u, k0 + u, p, dp, m, w);
+      const int key = k0 + u;
+      const float sc = group_sum<TPR>(dot<DP, CPT>(qr, sK, u, part)) * a.scale;
+      const float dp = group_sum<TPR>(dot<DP, CPT>(dor, sV, u, part));
+      const float m =
+          group_sum<TPR>(dot<DP, CPT>(uqr, sK, u, part) + dot<DP, CPT>(qr, sUK, u, part)) * a.scale;
+      const float w = group_sum<TPR>(dot<DP, CPT>(dor, sUV, u, part));
+      const bool keep = row < a.N && key < a.N && (!a.causal || key <= row);
+      const float p = keep ? expf(sc - L) : 0.f;
       r = fmaf(p, m, r);
       t1 = fmaf(p * m, dp, t1);
       t3 = fmaf(p, w, t3);
-    }
-  }
-  const float g = t1 - 2.f * r * D + t3;
-
-  // sweep 2: gQ and gdO
-  float gq[CPT], gdo[CPT];
-#pragma unroll
-  for (int c = 0; c < CPT; ++c) gq[c] = gdo[c] = 0.f;
-  for (int k0 = 0; k0 < key_end; k0 += kRows) {
-    __syncthreads();
-    stage<DP>(sK, kh, k0, a.N, a.d);
-    stage<DP>(sV, vh, k0, a.N, a.d);
-    stage<DP>(sUK, ukh, k0, a.N, a.d);
-    stage<DP>(sUV, uvh, k0, a.N, a.d);
-    __syncthreads();
-    for (int u = 0; u < kRows; ++u) {
-      float p, dp, m, w;
-      pair(u, k0 + u, p, dp, m, w);
-      const float ds = p * (dp - D);
-      const float e = p * (m - r);
-      const float ds2 = p * (m * (dp - D) - r * dp + w - g);
+      const float a1 = p * (dp - D);
+      const float a2 = p * fmaf(m, dp - D, w);
+      const float a3 = p * dp;
+      const float b1 = p * m;
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
         const int ch = CPT * part + c;
-        gq[c] = fmaf(ds, sUK[u][ch], fmaf(ds2, sK[u][ch], gq[c]));
-        gdo[c] = fmaf(e, sV[u][ch], fmaf(p, sUV[u][ch], gdo[c]));
+        const float kk = sK[u][ch], vv = sV[u][ch];
+        x1[c] = fmaf(a1, sUK[u][ch], x1[c]);
+        x2[c] = fmaf(a2, kk, x2[c]);
+        x3[c] = fmaf(a3, kk, x3[c]);
+        x4[c] = fmaf(p, kk, x4[c]);
+        y1[c] = fmaf(b1, vv, y1[c]);
+        y2[c] = fmaf(p, vv, y2[c]);
+        y3[c] = fmaf(p, sUV[u][ch], y3[c]);
       }
     }
   }
-  store_row<CPT>(a.gq + off, gq, a.scale, row, a.N, a.d, part);
-  store_row<CPT>(a.gdout + off, gdo, 1.f, row, a.N, a.d, part);
+  const float g = t1 - 2.f * r * D + t3;
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    x1[c] = x1[c] + x2[c] - r * x3[c] - g * x4[c];  // gQ / s
+    y1[c] = y1[c] - r * y2[c] + y3[c];              // gdO
+  }
+  store_row<CPT>(a.gq + off, x1, a.scale, row, a.N, a.d, part);
+  store_row<CPT>(a.gdout + off, y1, 1.f, row, a.N, a.d, part);
   if (part == 0 && row < a.Np) {
     a.r_pad[prow] = row < a.N ? r : 0.f;
     a.g_pad[prow] = row < a.N ? g : 0.f;
@@ -231,14 +231,16 @@ __global__ void __launch_bounds__(128) bob_cols_f32_kernel(const BobArgs a) {
   store_row<CPT>(a.gv + off, gv, 1.f, key, a.N, a.d, part);
 }
 
+// The query-row kernel keeps seven accumulators per row, so it always holds
+// 8 channels per thread; the key-row kernel takes CPT.
 template <int DP, int CPT>
 cudaError_t bob_dp(const BobArgs& a, int BH, cudaStream_t s) {
-  constexpr int R = 128 / (DP / CPT);
-  dim3 grid((a.N + R - 1) / R, BH);
-  bob_rows_f32_kernel<DP, CPT><<<grid, 128, 0, s>>>(a);
+  constexpr int RR = 128 / (DP / 8);
+  bob_rows_f32_kernel<DP, 8><<<dim3((a.N + RR - 1) / RR, BH), 128, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bob_cols_f32_kernel<DP, CPT><<<grid, 128, 0, s>>>(a);
+  constexpr int RC = 128 / (DP / CPT);
+  bob_cols_f32_kernel<DP, CPT><<<dim3((a.N + RC - 1) / RC, BH), 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -502,3 +502,30 @@ def test_double_backward_is_linear_in_the_cotangents():
     for name in ("gQ", "gK", "gV", "gdO"):
         np.testing.assert_allclose(b[name], 2 * a[name], rtol=1e-12, atol=1e-13)
         assert np.abs(z[name]).max() == 0.0
+
+
+def test_double_backward_row_side_is_affine_in_the_two_row_scalars():
+    # gQ and gdO of a row are fixed vectors combined with r and g (the
+    # structure the FlashBoB listing states): accumulating the seven vectors
+    # below, whose per-pair weights need neither scalar, and combining them
+    # with r and g reproduces the oracle
+    q, k, v, do, uq, uk, uv = _bob_inputs(25, n=11, d=5)
+    scale, n = 0.45, 11
+    out = oracle.double_backward_head(q, k, v, do, uq, uk, uv, scale, True)
+    f = A.forward_head(q, k, v, scale, True)
+    P = f["P"]
+    dP = do @ v.T
+    D = (P * dP).sum(axis=1, keepdims=True)
+    M = scale * (uq @ k.T + q @ uk.T)
+    W = do @ uv.T
+    r = (P * M).sum(axis=1, keepdims=True)
+    g = (P * M * dP).sum(axis=1, keepdims=True) - 2 * r * D + (P * W).sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(r[:, 0], out["r"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(g[:, 0], out["g"], rtol=1e-12, atol=1e-13)
+    x1 = (P * (dP - D)) @ uk
+    x2 = (P * (M * (dP - D) + W)) @ k
+    x3 = (P * dP) @ k
+    x4 = P @ k
+    y1, y2, y3 = (P * M) @ v, P @ v, P @ uv
+    np.testing.assert_allclose(scale * (x1 + x2 - r * x3 - g * x4), out["gQ"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(y1 - r * y2 + y3, out["gdO"], rtol=1e-11, atol=1e-12)
