@@ -861,7 +861,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=8,
+    ap.add_argument("--e2e-chunks", type=int, default=16,
                     help="head groups of the end-to-end (host-buffer) measurement")
     ap.add_argument("--shard-heads", action="store_true",
                     help="split one problem's heads over the ranks (strong scaling)")
