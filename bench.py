@@ -82,7 +82,7 @@ def load_peaks():
 
 def kernel_source_digest() -> str:
     h = hashlib.sha256()
-    for name in ("bwd_bf16_sm100.cu", "sm100.cuh", "common.cuh"):
+    for name in ("bwd_bf16_sm100.cu", "sm100.cuh", "common.cuh", "tile_walk.cuh"):
         with open(os.path.join(ROOT, "causal_softmax_attention_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
