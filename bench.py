@@ -65,6 +65,8 @@ import torch  # noqa: E402
 from seeded_inputs import CONFIGS, block_mask, block_mask_pairs, draw  # noqa: E402
 
 METRIC = "causal attention backward TFLOP/s (bf16, 1×B200) and % of dense tensor peak"
+BOB_METRIC = "causal attention backward-over-backward TFLOP/s (fp32, 1xB200)"
+LAYER_METRIC = "causal multi-head attention layer step TFLOP/s (bf16, forward + backward)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 MAIN_KERNEL_SOURCE = os.path.join(ROOT, "causal_softmax_attention_b200", "csrc",
                                   "bwd_bf16_sm100.cu")
@@ -274,11 +276,74 @@ def blas_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def oracle_sample_repeat(name, fn, flops_per_run, budget_s):
+    """Run the oracle call `fn` until `budget_s` seconds of CPU work."""
+    runs, elapsed = 0, 0.0
+    while elapsed < budget_s:
+        t0 = time.perf_counter()
+        fn()
+        elapsed += time.perf_counter() - t0
+        runs += 1
+    return flops_per_run * runs / elapsed / 1e12, f"{name}: {runs} runs in {elapsed:.1f} s", elapsed
+
+
+def oracle_sample_bob(cfg, budget_s):
+    """The double-backward oracle on the whole workload (as the --bob arm)."""
+    import oracle
+    from seeded_inputs import as_f64
+    a = [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed, "f32", cfg.qk_gain)]
+    a += [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed + 500, "f32")[:3]]
+    return oracle_sample_repeat(
+        f"oracle double_backward (numpy float64) on {cfg.name}",
+        lambda: oracle.double_backward(*a, cfg.scale, True), 12.0 * cfg.B * cfg.H * cfg.N ** 2 * cfg.d,
+        budget_s)
+
+
+def oracle_sample_layer(cfg, budget_s, n_sample=256):
+    """The layer oracle on one sequence of n_sample tokens with the --layer
+    arm's widths (C = H*d); FLOPs counted as that arm counts them."""
+    import oracle
+    from seeded_inputs import as_f64, draw_layer
+    C, n = cfg.H * cfg.d, min(cfg.N, n_sample)
+    x, wq, wo, dy = (as_f64(t) for t in draw_layer(1, n, C, cfg.seed))
+    flops = 24.0 * n * C * C + 7.0 * cfg.H * n * n * cfg.d
+    return oracle_sample_repeat(
+        f"oracle mha_layer (numpy float64) on 1 x {n} tokens, C={C}, H={cfg.H}",
+        lambda: oracle.mha_layer(x, wq, wo, dy, cfg.H), flops, budget_s)
+
+
+def bob_config(cfg, n_gpus):
+    return dict(config_dict(cfg, n_gpus), workload=f"{cfg.name}: causal attention "
+                f"backward-over-backward B={cfg.B} H={cfg.H} N={cfg.N} d={cfg.d} f32, "
+                "q,k,v,dO,U ~ N(0,1)")
+
+
+def layer_config(cfg):
+    C = cfg.H * cfg.d
+    return {"workload": f"attention layer B={cfg.B} N={cfg.N} C={C} H={cfg.H} (d={cfg.d}), causal, "
+                        "x, dy ~ N(0,1), weights ~ N(0,1/C), no biases",
+            "B": cfg.B, "N": cfg.N, "C": C, "H": cfg.H, "d": cfg.d, "parallelism": "single GPU",
+            "l2": "inputs larger than L2 (no flush needed)"}
+
+
+def mode_metric_config(args, cfg, n_gpus):
+    """The metric and config of the measurement the flags select."""
+    if args.bob:
+        return BOB_METRIC, bob_config(cfg, n_gpus)
+    if args.layer:
+        return LAYER_METRIC, layer_config(cfg)
+    return METRIC, config_dict(cfg, n_gpus, args.block_mask, args.layout)
+
+
 def run_reference(args, cfg, world, rank):
     if rank != 0:
         return
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     def sample(b):
+        if args.bob:
+            return oracle_sample_bob(cfg, b)
+        if args.layer:
+            return oracle_sample_layer(cfg, b)
         if args.block_mask:
             return oracle_sample_masked(cfg, args.block_mask, b)
         return oracle_sample(cfg, b)
@@ -293,12 +358,13 @@ def run_reference(args, cfg, world, rank):
         times.append(t)
     value = statistics.median(vals)
     cores = blas_threads()
+    metric, config = mode_metric_config(args, cfg, args.gpus)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": metric, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(cfg, args.gpus, args.block_mask),
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": descs[-1]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -481,12 +547,11 @@ def run_bob(args, cfg, world, rank, local):
     peaks, _ = load_peaks()
     ffma = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
     line = {
-        "metric": "causal attention backward-over-backward TFLOP/s (fp32, 1xB200)",
+        "metric": BOB_METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(config_dict(cfg, world), workload=f"{cfg.name}: causal attention "
-                       f"backward-over-backward B={B} H={H} N={N} d={d} f32, q,k,v,dO,U ~ N(0,1)"),
+        "config": bob_config(cfg, world),
         "roofline": {"bound": "alu", "achieved": value / world, "peak": ffma, "unit": "TFLOP/s",
                      "frac": value / world / ffma, "traffic": None,
                      "kernel": "bob_rows_f32_kernel + bob_cols_f32_kernel (+ preprocess)",
@@ -588,14 +653,11 @@ def run_layer(args, cfg, world, rank, local):
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (ms_per_step * 1e-3) / 1e12
     line = {
-        "metric": "causal multi-head attention layer step TFLOP/s (bf16, forward + backward)",
+        "metric": LAYER_METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"attention layer B={B} N={N} C={C} H={H} (d={d}), causal, "
-                               "x, dy ~ N(0,1), weights ~ N(0,1/C), no biases",
-                   "B": B, "N": N, "C": C, "H": H, "d": d, "parallelism": "single GPU",
-                   "l2": "inputs larger than L2 (no flush needed)"},
+        "config": layer_config(cfg),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
                      "kernel": "whole layer step (4 cuBLAS GEMMs x 3 + attention fwd + bwd)",
