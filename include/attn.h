@@ -11,8 +11,13 @@
  * cancels in w / z (same issue, item 1); the backward uses the row term
  * D_i = sum_c dO_ic O_ic instead.
  *
- * Layout. Every matrix argument is a DEVICE pointer to a contiguous
- * [B][H][N][d] row-major array (batch, head, position, channel), of the
+ * Beyond that: block-sparse masks (attn_*_masked), arbitrary row strides
+ * (attn_*_strided) and the backward-over-backward (attn_bwd_bwd), each
+ * declared below with its own conventions.
+ *
+ * Layout. Unless an entry point says otherwise, every matrix argument is a
+ * DEVICE pointer to a contiguous [B][H][N][d] row-major array (batch, head,
+ * position, channel), of the
  * element type `dtype` (ATTN_F32: float, ATTN_BF16: bfloat16 bits). LSE is a
  * device [B][H][N] float array in natural-log units: LSE_i = m_i + ln z_i of
  * the SCALED scores s_ij = scale * q_i . k_j (the scale is applied before the
