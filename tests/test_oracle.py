@@ -529,3 +529,14 @@ def test_double_backward_row_side_is_affine_in_the_two_row_scalars():
     y1, y2, y3 = (P * M) @ v, P @ v, P @ uv
     np.testing.assert_allclose(scale * (x1 + x2 - r * x3 - g * x4), out["gQ"], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(y1 - r * y2 + y3, out["gdO"], rtol=1e-11, atol=1e-12)
+
+
+def test_double_backward_single_position_closed_form():
+    # N = 1: P = 1, so dS = E = dS2 = 0 and only dV = dO depends on dO:
+    # gQ = gK = gV = 0, gdO = U_V
+    r = np.random.default_rng(26)
+    q, k, v, do, uq, uk, uv = (r.standard_normal((1, 6)) for _ in range(7))
+    out = oracle.double_backward_head(q, k, v, do, uq, uk, uv, 0.8)
+    for name in ("gQ", "gK", "gV"):
+        assert np.abs(out[name]).max() == 0.0, name
+    np.testing.assert_array_equal(out["gdO"], uv)
