@@ -951,7 +951,10 @@ def main():
     if args.block_mask:
         if cfg.dtype != "bf16":
             ap.error("--block-mask needs a bf16 config")
-        block_mask(args.block_mask, 128)  # rejects a malformed spec before any GPU work
+        try:
+            block_mask(args.block_mask, 128)  # a malformed spec fails before any GPU work
+        except (ValueError, IndexError) as e:
+            ap.error(f"--block-mask: {e}")
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, cfg, world, rank)

@@ -122,3 +122,15 @@ def test_backward_shard_hands_each_rank_its_block(monkeypatch):
                 assert blk.shape == (1, e - s) + tuple(t.shape[2:])
                 assert blk.data_ptr() == t.reshape(B * H, *t.shape[2:])[s].data_ptr()
             assert args[9] == "ws"
+
+
+@pytest.mark.parametrize("argv", [["--layout", "bnhd", "--block-mask", "causal"],
+                                  ["--block-mask", "causal", "--config", "c1"],
+                                  ["--block-mask", "diagonal"],
+                                  ["--warmup", "2"]])
+def test_bench_rejects_contradictory_flags_before_any_gpu_work(argv):
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        *argv], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2 and "Traceback" not in r.stderr, r.stderr[-500:]
