@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "attn_status_string": (ctypes.c_char_p, [i]),
         "attn_test_arm_timeout": (i, [ctypes.c_ulonglong]),
         "attn_bwd_noalloc": (i, [vp] * 9 + [i, i, i, i, i, f, i, vp]),
+        "attn_bwd_noalloc_last_status": (i, []),
         "attn_fwd_masked": (i, [vp] * 5 + [i, i, i, i, vp, f, i, vp]),
         "attn_bwd_masked": (i, [vp] * 9 + [i, i, i, i, vp, f, i, vp, sz, vp]),
         "attn_bwd_main_masked": (i, [vp] * 7 + [i, i, i, i, vp, f, i, vp, sz, vp]),
@@ -71,7 +72,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_preprocess",
             "attn_bwd_main", "attn_bwd_dq_convert", "attn_last_status", "attn_fwd_last_status",
-            "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc", "attn_fwd_masked",
+            "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc",
+            "attn_bwd_noalloc_last_status", "attn_fwd_masked",
             "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided",
             "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd")
 
@@ -193,8 +195,10 @@ def attn_fwd_last_status() -> int:
     return int(_lib.attn_fwd_last_status())
 
 
-def attn_test_arm_timeout(wait_limit_ns: int) -> int:
-    return int(_lib.attn_test_arm_timeout(int(wait_limit_ns)))
+def attn_test_arm_timeout(wait_limit_cycles: int) -> int:
+    """Arm the one-shot timeout of the next bf16 backward; each of its device
+    waits is bounded by `wait_limit_cycles` SM clock cycles."""
+    return int(_lib.attn_test_arm_timeout(int(wait_limit_cycles)))
 
 
 def new_workspace(q: torch.Tensor) -> torch.Tensor:

@@ -32,22 +32,54 @@ namespace {
 static __device__ __align__(256) unsigned char g_bwd_scratch[ATTN_BWD_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_device_addr[kMaxDevices] = {};
+// Per device: the context the address was looked up in, and the address.
+// A device reset (or a destroyed and recreated primary context) reloads the
+// module and may move the array, so the address is only reused while the
+// current context is the one it was found in.
+struct ScratchSlot {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of g_bwd_scratch on the current device, looked up on the
-// first call made with that device current and cached afterwards.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_bwd_scratch on the current device, looked up (with
+// that device current) on the first call in each context and cached.
 int scratch_on_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) return ATTN_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_device_addr[dev] == nullptr) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (ctx == nullptr || slot.addr == nullptr || slot.ctx != ctx) {
+    // The lookup also initialises the device's primary context (and makes it
+    // current) when no context is current yet.
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr)
       return ATTN_ERR_CUDA;
-    g_scratch_device_addr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return ATTN_ERR_CUDA;
+    slot.ctx = ctx;
+    slot.addr = p;
   }
-  *out = g_scratch_device_addr[dev];
+  *out = slot.addr;
   return ATTN_OK;
 }
 
@@ -69,4 +101,11 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
   if (st != ATTN_OK) return st;
   return attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, dtype, scratch,
                   ATTN_BWD_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int attn_bwd_noalloc_last_status(void) {
+  void* scratch = nullptr;
+  const int st = scratch_on_current_device(&scratch);
+  if (st != ATTN_OK) return st;
+  return attn_last_status(scratch);
 }

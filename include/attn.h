@@ -258,14 +258,24 @@ int attn_test_arm_timeout(unsigned long long wait_limit_cycles);
  * device current) and caches it; make that first call before any stream
  * capture. All calls share the one array and it keeps the last call's
  * contents (each call re-zeroes what must start at zero), so calls that
- * overlap on the same GPU race: serialise them. Device-side timeouts are
- * recorded in the array's status word, which this entry point does not
- * expose. Returns an attn_status.
+ * overlap on the same GPU race: serialise them. The address is cached per
+ * device together with the CUDA context it was found in; a call from a new
+ * context (after a device reset, say) looks it up again. Device-side
+ * timeouts are recorded in the array's status word: read it with
+ * attn_bwd_noalloc_last_status. Returns an attn_status.
  */
 #define ATTN_BWD_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                      int H, int N, int d, int causal, float scale, int dtype, void* stream);
+
+/*
+ * The status word of the last attn_bwd_noalloc on the current device (as
+ * attn_last_status reads a workspace's): ATTN_OK, or ATTN_ERR_TIMEOUT if a
+ * bounded device wait of that call ran out. Synchronises the calling thread
+ * with the device; allocates nothing.
+ */
+int attn_bwd_noalloc_last_status(void);
 
 #ifdef __cplusplus
 }

@@ -264,6 +264,28 @@ def backward_row_block(q, k, v, do, scale, r0, r1, causal=True):
             "O": O, "LSE": m + np.log(z), "D": D}
 
 
+def backward_blocked(q, k, v, do, scale, causal=True, rows_per_block=1024):
+    """The whole backward of one head as the sum of its row blocks.
+
+    Runs ``backward_row_block`` over consecutive blocks of query rows and adds
+    up their dK, dV contributions (dK and dV are sums over query rows); dQ, O,
+    LSE and D of each block's rows are complete as they come. The result is
+    ``backward_head``'s without ever holding more than rows_per_block x N of
+    the score table. q, k, v, do: [N, d] float64.
+    """
+    n, d = np.asarray(q).shape
+    out = {"dQ": np.empty((n, d)), "dK": np.zeros((n, d)), "dV": np.zeros((n, d)),
+           "O": np.empty((n, np.asarray(v).shape[1])), "LSE": np.empty(n), "D": np.empty(n)}
+    for r0 in range(0, n, rows_per_block):
+        r1 = min(n, r0 + rows_per_block)
+        blk = backward_row_block(q, k, v, do, scale, r0, r1, causal)
+        out["dK"] += blk["dK"]
+        out["dV"] += blk["dV"]
+        for name in ("dQ", "O", "LSE", "D"):
+            out[name][r0:r1] = blk[name]
+    return out
+
+
 def key_tail(q, k, v, do, scale, j0):
     """dK and dV of keys j >= j0 of one causal head.
 

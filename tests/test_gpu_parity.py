@@ -1,9 +1,13 @@
 """GPU parity: the CUDA library (through its C ABI) against the float64 oracle.
 
-Small and medium shapes are compared element by element over every output;
-the two long-sequence workloads (16,384 x 32 heads and 262,144 tokens) are
-compared on sampled query rows and on the last key rows, which the oracle
-computes one by one, plus identities that hold at any size.
+Small and medium shapes are compared element by element over every output,
+and so are 8-head cases of 8,192 (d = 128) and 16,384 (d = 64) tokens, whose
+key tiles walk 64 and 128 query tiles, through the oracle's row-blocked pass.
+Of the 16,384-token x 32-head workload two whole heads are compared element by
+element and two more on sampled rows and the last key rows; the 262,144-token
+workload on sampled query rows and its last key rows (the only keys whose
+gradients the oracle can form without a full head), plus identities that
+hold at any size.
 
 Tolerances (max |gpu - oracle| / max |oracle| per output): 1e-5 for the fp32
 path, 2e-2 for the bf16 path (bf16 inputs and outputs, fp32 accumulation).
@@ -438,8 +442,101 @@ def test_nonfinite_inputs_propagate(csa):
     assert not torch.isnan(g["O"][0, 0, :, :3]).any()
 
 
+# ------------------------------------------------------------------ long tile walks, every element
+def full_head_parity(g, q, k, v, do, scale, heads, tol=TOL["bf16"]):
+    """Every element of O, LSE, dQ, dK, dV of the given heads against the
+    oracle's row-blocked pass over all query rows (the materialised head's
+    result, without an N x N table); per head, gradients are measured
+    against the largest of its three gradients, as in compare_full."""
+    for (b, h) in heads:
+        qh, kh, vh, doh = (as_f64(t[b, h]) for t in (q, k, v, do))
+        ref = oracle.backward_blocked(qh, kh, vh, doh, scale, True)
+        gscale = max(np.abs(ref[n]).max() for n in ("dQ", "dK", "dV"))
+        for name in ("O", "dQ", "dK", "dV"):
+            got = as_f64(g[name][b, h].cpu())
+            e = rel(got, ref[name], None if name == "O" else gscale)
+            assert e <= tol, ((b, h), name, e)
+        assert np.abs(as_f64(g["LSE"][b, h].cpu()) - ref["LSE"]).max() <= 1e-3, (b, h)
+
+
+@pytest.mark.parametrize("N,d,qk_gain", [(8192, 128, 1.0), (16384, 64, 0.5)])
+def test_long_walk_every_element(csa, N, d, qk_gain):
+    # 8 heads: key tile 0 accumulates dK, dV over 64 (d = 128) or 128 (d = 64)
+    # query tiles in tensor memory, and the CTAs run in two L2 head groups of
+    # unequal size (5 + 3 heads); every output element of every head is checked
+    B, H = 1, 8
+    q, k, v, do = draw(B, H, N, d, 700 + d, "bf16", qk_gain)
+    g = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    full_head_parity(g, q, k, v, do, d ** -0.5, [(0, h) for h in range(H)])
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_head_sharded_backward_against_the_oracle(csa, world):
+    # every rank's block through shard.backward_shard, all ranks in this one
+    # process writing into shared full-size gradients (6 heads: 3 + 3, 2 + 2
+    # + 2, and 2 + 2 + 2 + none)
+    from causal_softmax_attention_b200.shard import backward_shard, head_range
+    B, H, N, d = 2, 3, 500, 64
+    q, k, v, do = draw(B, H, N, d, 720 + world, "bf16")
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = csa.forward(qd, kd, vd, True, d ** -0.5)
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    covered = []
+    for rank in range(world):
+        start, end = head_range(B * H, world, rank)
+        ws = torch.empty(max(1, csa.attn_bwd_workspace_bytes(1, max(1, end - start), N, d,
+                                                                 qd.dtype)),
+                         dtype=torch.uint8, device=dev)
+        got = backward_shard(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, world, rank, True,
+                             d ** -0.5)
+        assert got == (start, end)
+        covered += list(range(start, end))
+    torch.cuda.synchronize()
+    assert covered == list(range(B * H))
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), d ** -0.5, True)
+    gscale = max(np.abs(ref[n]).max() for n in ("dQ", "dK", "dV"))
+    for name, t in (("dQ", dq), ("dK", dk), ("dV", dv)):
+        assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["bf16"], name
+
+
+@pytest.mark.parametrize("dtype,N,d", [("bf16", 333, 64), ("bf16", 130, 128), ("f32", 201, 48)])
+def test_outputs_stay_inside_their_buffers(csa, dtype, N, d):
+    # dQ, dK, dV (and O, LSE) written into the middle of larger buffers whose
+    # guard regions hold a canary pattern: no byte outside the outputs changes
+    B, H = 2, 2
+    q, k, v, do = draw(B, H, N, d, 730 + N, dtype)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    n = B * H * N * d
+    guard = 4096  # elements on each side (a multiple of 8: keeps 16-byte alignment)
+
+    def guarded(count, dt):
+        buf = torch.empty(count + 2 * guard, dtype=dt, device=dev)
+        buf.view(torch.uint8).fill_(0xA5)
+        return buf
+
+    bufs = {name: guarded(n, qd.dtype) for name in ("o", "dq", "dk", "dv")}
+    bufs["lse"] = guarded(B * H * N, torch.float32)
+    view = {name: b[guard:guard + n].view(B, H, N, d) for name, b in bufs.items() if name != "lse"}
+    lse = bufs["lse"][guard:guard + B * H * N].view(B, H, N)
+    csa.attn_fwd(qd, kd, vd, view["o"], lse, True, d ** -0.5)
+    csa.attn_bwd(qd, kd, vd, view["o"], dod, lse, view["dq"], view["dk"], view["dv"],
+                 csa.new_workspace(qd), True, d ** -0.5)
+    torch.cuda.synchronize()
+    for name, b in bufs.items():
+        raw = b.view(torch.uint8)
+        per = b.element_size()
+        assert bool((raw[:guard * per] == 0xA5).all()), (name, "before")
+        assert bool((raw[-guard * per:] == 0xA5).all()), (name, "after")
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), d ** -0.5, True)
+    gscale = max(np.abs(ref[n_]).max() for n_ in ("dQ", "dK", "dV"))
+    for name in ("dq", "dk", "dv"):
+        assert rel(as_f64(view[name].cpu()), ref["d" + name[1:].upper()], gscale) <= TOL[dtype]
+
+
 # ------------------------------------------------------------------ full-size workloads
-def sampled_parity(csa, name, heads, n_rows=24, tail=128):
+def sampled_parity(csa, name, heads, n_rows=24, tail=128, full_heads=()):
     c = CONFIGS[name]
     q, k, v, do = draw(c.B, c.H, c.N, c.d, c.seed, c.dtype, c.qk_gain)
     torch.cuda.reset_peak_memory_stats()
@@ -449,6 +546,8 @@ def sampled_parity(csa, name, heads, n_rows=24, tail=128):
     # memory is linear in N: inputs, outputs and workspace are O(B*H*N*d)
     elems = c.B * c.H * c.N * c.d
     assert peak <= elems * 2 * 12 + c.B * c.H * c.N * 64, peak
+    # whole heads, every element (every key tile's walk, the longest included)
+    full_head_parity(g, q, k, v, do, c.scale, full_heads)
     rng = np.random.default_rng(c.seed)
     for (b, h) in heads:
         rows = np.sort(np.concatenate([rng.choice(c.N, n_rows - 4, replace=False),
@@ -473,7 +572,9 @@ def sampled_parity(csa, name, heads, n_rows=24, tail=128):
 
 
 def test_long_sequence_16k_parity(csa):
-    sampled_parity(csa, "c4", heads=[(0, 0), (1, 15)])
+    # two whole heads element by element (their key tile 0 walks all 128
+    # query tiles), sampled rows and the key tail of two more
+    sampled_parity(csa, "c4", heads=[(0, 7), (1, 8)], full_heads=[(0, 0), (1, 15)])
 
 
 def test_long_sequence_262k_parity(csa):

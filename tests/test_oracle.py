@@ -258,6 +258,20 @@ def test_query_rows_and_row_blocks(causal):
         assert rel(tail["dV"], full["dV"][50:]) <= 1e-12
 
 
+@pytest.mark.parametrize("causal,block", [(True, 16), (True, 23), (False, 16), (True, 1000)])
+def test_blocked_backward_equals_the_materialised_head(causal, block):
+    # the sum of the row blocks, whatever the block size (ragged last block,
+    # one block for everything), is the materialised head's backward
+    n, d = 70, 8
+    q, k, v, do = tiny_case(31, n=n, d=d)
+    full = A.backward_head(q, k, v, do, 0.35, causal)
+    got = A.backward_blocked(q, k, v, do, 0.35, causal, rows_per_block=block)
+    for name in ("dQ", "dK", "dV", "D"):
+        assert rel(got[name], full[name]) <= 1e-12, name
+    assert rel(got["O"], full["fwd"]["O"]) <= 1e-12
+    assert np.allclose(got["LSE"], full["fwd"]["LSE"], rtol=1e-13)
+
+
 def test_batched_equals_per_head_and_head_permutation():
     B, H, N, d = 2, 3, 19, 4
     q, k, v, do = (rnd(40 + t, B, H, N, d) for t in range(4))
