@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "attn_bwd_main_masked": (i, [vp] * 7 + [i, i, i, i, vp, f, i, vp, sz, vp]),
         "attn_fwd_strided": (i, [vp] * 5 + [i, i, i, i, vp, vp, i, f, i, vp]),
         "attn_bwd_strided": (i, [vp] * 9 + [i, i, i, i, vp, vp, i, f, i, vp, sz, vp]),
+        "attn_fwd_rect": (i, [vp] * 5 + [i] * 7 + [f, i, vp]),
+        "attn_bwd_rect": (i, [vp] * 9 + [i] * 7 + [f, i, vp, sz, vp]),
         "attn_bwd_bwd_workspace_bytes": (sz, [i, i, i, i, i]),
         "attn_bwd_bwd": (i, [vp] * 13 + [i, i, i, i, i, f, i, vp, sz, vp]),
     }
@@ -75,7 +77,7 @@ EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_prepro
             "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc",
             "attn_bwd_noalloc_last_status", "attn_fwd_masked",
             "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided",
-            "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd")
+            "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd", "attn_fwd_rect", "attn_bwd_rect")
 
 
 def library() -> ctypes.CDLL:
@@ -256,6 +258,55 @@ def attn_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal: bool 
     if check:
         _check(st, "attn_bwd_strided")
     return st
+
+
+def attn_fwd_rect(q, k, v, o, lse, q_offset: int = 0, causal: bool = True,
+                  scale: float | None = None, stream=None, check: bool = True) -> int:
+    """O, LSE <- forward of N_q query rows ([B, H, N_q, d] q, o) over N_k keys
+    ([B, H, N_k, d] k, v); query row r is position q_offset + r."""
+    B, H, nq, d = _shape(q)
+    nk = int(k.shape[2])
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_fwd_rect(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, nq, nk, d,
+                            int(q_offset), int(causal), float(scale), _DTYPES[q.dtype],
+                            _stream(stream))
+    if check:
+        _check(st, "attn_fwd_rect")
+    return st
+
+
+def attn_bwd_rect(q, k, v, o, dout, lse, dq, dk, dv, workspace, q_offset: int = 0,
+                  causal: bool = True, scale: float | None = None, stream=None,
+                  check: bool = True) -> int:
+    """dQ, dK, dV of attn_fwd_rect; `workspace` sized by
+    attn_bwd_workspace_bytes(B, H, N_q, d, dtype)."""
+    B, H, nq, d = _shape(q)
+    nk = int(k.shape[2])
+    scale = d ** -0.5 if scale is None else scale
+    st = _lib.attn_bwd_rect(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, H, nq, nk, d, int(q_offset), int(causal),
+                            float(scale), _DTYPES[q.dtype], _ptr(workspace),
+                            int(workspace.numel()), _stream(stream))
+    if check:
+        _check(st, "attn_bwd_rect")
+    return st
+
+
+def forward_rect(q, k, v, q_offset: int = 0, causal: bool = True, scale: float | None = None):
+    """Convenience: allocate O and LSE and run attn_fwd_rect."""
+    B, H, nq, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, nq, dtype=torch.float32, device=q.device)
+    attn_fwd_rect(q, k, v, o, lse, q_offset, causal, scale)
+    return o, lse
+
+
+def backward_rect(q, k, v, o, dout, lse, q_offset: int = 0, causal: bool = True,
+                  scale: float | None = None):
+    """Convenience: allocate dQ, dK, dV and a workspace and run attn_bwd_rect."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    attn_bwd_rect(q, k, v, o, dout, lse, dq, dk, dv, new_workspace(q), q_offset, causal, scale)
+    return dq, dk, dv
 
 
 def attn_bwd_bwd(q, k, v, o, dout, lse, uq, uk, uv, gq, gk, gv, gdout, workspace,

@@ -55,6 +55,18 @@ int check_shape(int B, int H, int N, int d, int dtype) {
   return ATTN_OK;
 }
 
+// Extents of a rectangular call: at least one query row and one key, a
+// query offset in [0, 2^30], and tile counts the launch grids can hold.
+int check_extent(int B, int H, const Extent& ex, int d, int dtype) {
+  int st = check_shape(B, H, ex.nq, d, dtype);
+  if (st != ATTN_OK) return st;
+  if ((st = check_shape(B, H, ex.nk, d, dtype)) != ATTN_OK) return st;
+  if (ex.q_off < 0 || ex.q_off > (1 << 30)) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+Extent square(int N) { return {N, N, 0}; }
+
 bool all_aligned(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (p == nullptr || !aligned16(p)) return false;
@@ -176,27 +188,27 @@ namespace {
 // Every implementation takes the row strides of q, k, v (and of dq, dk, dv:
 // qs) and of o, dout (os); the plain entry points pass the contiguous layout.
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int N, int d, int causal, float scale, int dtype, const uint8_t* bmask,
-             const RowStrides& qs, const RowStrides& os, void* stream) {
+             const Extent& ex, int d, int causal, float scale, int dtype, const uint8_t* bmask,
+             const RowStrides& qs, const RowStrides& os, void* stream, const RowStrides& ks) {
   if (!tensors_aligned(dtype, {q, k, v, o}) || !all_aligned({lse})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-  int st = check_shape(B, H, N, d, dtype);
+  int st = check_extent(B, H, ex, d, dtype);
   if (st != ATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (dtype == ATTN_F32)
     return from_cuda(launch_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                     static_cast<const float*>(v), static_cast<float*>(o), lse, BH,
-                                    N, d, causal != 0, scale, qs, os, s));
+                                    ex, d, causal != 0, scale, qs, ks, os, s));
   if ((st = check_device_sm100()) != ATTN_OK) return st;
   TmaMaps m;
-  if (!make_map(&m.a, q, B, N, d, qs) || !make_map(&m.b, k, B, N, d, qs) ||
-      !make_map(&m.c, v, B, N, d, qs))
+  if (!make_map(&m.a, q, B, ex.nq, d, qs) || !make_map(&m.b, k, B, ex.nk, d, ks) ||
+      !make_map(&m.c, v, B, ex.nk, d, ks))
     return ATTN_ERR_CUDA;
   int* status = fwd_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
   return from_cuda(
-      launch_fwd_bf16(m, o, lse, status, BH, N, d, causal != 0, scale, bmask, os, s));
+      launch_fwd_bf16(m, o, lse, status, BH, ex, d, causal != 0, scale, bmask, os, s));
 }
 
 int preprocess_impl(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
@@ -212,27 +224,28 @@ int preprocess_impl(const void* o, const void* dout, const float* lse, int B, in
 }
 
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, void* dq,
-                  void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
-                  int dtype, void* workspace, size_t workspace_bytes, const uint8_t* bmask,
-                  const RowStrides& qs, const RowStrides& os, void* stream) {
+                  void* dk, void* dv, int B, int H, const Extent& ex, int d, int causal,
+                  float scale, int dtype, void* workspace, size_t workspace_bytes,
+                  const uint8_t* bmask, const RowStrides& qs, const RowStrides& os,
+                  void* stream, const RowStrides& ks) {
   if (!tensors_aligned(dtype, {q, k, v, dout, dq, dk, dv})) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-  int st = check_shape(B, H, N, d, dtype);
+  int st = check_extent(B, H, ex, d, dtype);
   if (st != ATTN_OK) return st;
-  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
-  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
+  if ((st = check_ws(B, H, ex.nq, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, ex.nq, d, dtype));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (dtype == ATTN_F32)
     return from_cuda(launch_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                     static_cast<const float*>(v),
                                     static_cast<const float*>(dout), static_cast<float*>(dq),
-                                    static_cast<float*>(dk), static_cast<float*>(dv), BH, N, d,
-                                    causal != 0, scale, qs, os, ws, s));
+                                    static_cast<float*>(dk), static_cast<float*>(dv), BH, ex, d,
+                                    causal != 0, scale, qs, ks, os, ws, s));
   if ((st = check_device_sm100()) != ATTN_OK) return st;
   TmaMaps m;
-  if (!make_map(&m.a, q, B, N, d, qs) || !make_map(&m.b, k, B, N, d, qs) ||
-      !make_map(&m.c, v, B, N, d, qs) || !make_map(&m.d, dout, B, N, d, os))
+  if (!make_map(&m.a, q, B, ex.nq, d, qs) || !make_map(&m.b, k, B, ex.nk, d, ks) ||
+      !make_map(&m.c, v, B, ex.nk, d, ks) || !make_map(&m.d, dout, B, ex.nq, d, os))
     return ATTN_ERR_CUDA;
   int inject = 0;
   unsigned long long limit = kWaitLimitCycles;
@@ -244,8 +257,8 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout,
       g_fault.armed = 0;
     }
   }
-  return from_cuda(launch_bwd_bf16(m, ws, dk, dv, BH, N, d, causal != 0, scale, limit, inject,
-                                   bmask, qs, s));
+  return from_cuda(launch_bwd_bf16(m, ws, dk, dv, BH, ex, d, causal != 0, scale, limit, inject,
+                                   bmask, ks, s));
 }
 
 int dq_convert_impl(void* dq, int B, int H, int N, int d, float scale, int dtype,
@@ -264,23 +277,26 @@ int dq_convert_impl(void* dq, int B, int H, int N, int d, float scale, int dtype
 // The whole backward: every argument is checked before the first launch, so
 // a bad call enqueues nothing.
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
-             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-             int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
-             const uint8_t* bmask, const RowStrides& qs, const RowStrides& os, void* stream) {
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, const Extent& ex,
+             int d, int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+             const uint8_t* bmask, const RowStrides& qs, const RowStrides& os, void* stream,
+             const RowStrides& ks) {
   if (!tensors_aligned(dtype, {q, k, v, o, dout, dq, dk, dv}) || !all_aligned({lse}))
     return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-  int st = check_shape(B, H, N, d, dtype);
+  int st = check_extent(B, H, ex, d, dtype);
   if (st != ATTN_OK) return st;
   if (bmask != nullptr && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  if ((st = check_ws(B, H, N, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
+  if ((st = check_ws(B, H, ex.nq, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
   if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
-  st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes, os, stream);
+  st = preprocess_impl(o, dout, lse, B, H, ex.nq, d, dtype, workspace, workspace_bytes, os,
+                       stream);
   if (st != ATTN_OK) return st;
-  st = bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                     workspace_bytes, bmask, qs, os, stream);
+  st = bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, ex, d, causal, scale, dtype, workspace,
+                     workspace_bytes, bmask, qs, os, stream, ks);
   if (st != ATTN_OK) return st;
-  return dq_convert_impl(dq, B, H, N, d, scale, dtype, workspace, workspace_bytes, qs, stream);
+  return dq_convert_impl(dq, B, H, ex.nq, d, scale, dtype, workspace, workspace_bytes, qs,
+                         stream);
 }
 
 RowStrides dense(int H, int N, int d) { return contiguous_strides(H, N, d); }
@@ -289,8 +305,8 @@ RowStrides dense(int H, int N, int d) { return contiguous_strides(H, N, d); }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int N, int d, int causal, float scale, int dtype, void* stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, dense(H, N, d),
-                  dense(H, N, d), stream);
+  return fwd_impl(q, k, v, o, lse, B, H, square(N), d, causal, scale, dtype, nullptr, dense(H, N, d),
+                  dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -299,8 +315,8 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
   if (block_mask == nullptr) return ATTN_ERR_INVALID;
   if (dtype != ATTN_BF16) return check_shape(B, H, N, d, dtype) == ATTN_OK ? ATTN_ERR_UNSUPPORTED
                                                                          : ATTN_ERR_INVALID;
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, scale, dtype, block_mask, dense(H, N, d),
-                  dense(H, N, d), stream);
+  return fwd_impl(q, k, v, o, lse, B, H, square(N), d, 0, scale, dtype, block_mask, dense(H, N, d),
+                  dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -312,7 +328,7 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
   if (st != ATTN_OK) return st;
   if ((st = check_strides(qkv_strides, H, d, dtype, &qs)) != ATTN_OK) return st;
   if ((st = check_strides(o_strides, H, d, dtype, &os)) != ATTN_OK) return st;
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, nullptr, qs, os, stream);
+  return fwd_impl(q, k, v, o, lse, B, H, square(N), d, causal, scale, dtype, nullptr, qs, os, stream, qs);
 }
 
 int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N,
@@ -324,8 +340,8 @@ int attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B
 int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
                   void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                   int dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                       workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream);
+  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, square(N), d, causal, scale, dtype, workspace,
+                       workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void* dout, void* dq,
@@ -336,8 +352,8 @@ int attn_bwd_main_masked(const void* q, const void* k, const void* v, const void
   const int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
   if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
-                       workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream);
+  return bwd_main_impl(q, k, v, dout, dq, dk, dv, B, H, square(N), d, 0, scale, dtype, workspace,
+                       workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, int dtype,
@@ -350,8 +366,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
              int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
              void* stream) {
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                  workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, square(N), d, causal, scale, dtype, workspace,
+                  workspace_bytes, nullptr, dense(H, N, d), dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
@@ -359,8 +375,8 @@ int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
                     int H, int N, int d, const unsigned char* block_mask, float scale, int dtype,
                     void* workspace, size_t workspace_bytes, void* stream) {
   if (block_mask == nullptr) return ATTN_ERR_INVALID;
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, 0, scale, dtype, workspace,
-                  workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, square(N), d, 0, scale, dtype, workspace,
+                  workspace_bytes, block_mask, dense(H, N, d), dense(H, N, d), stream, dense(H, N, d));
 }
 
 int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
@@ -373,8 +389,24 @@ int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
   if (st != ATTN_OK) return st;
   if ((st = check_strides(qkv_strides, H, d, dtype, &qs)) != ATTN_OK) return st;
   if ((st = check_strides(o_strides, H, d, dtype, &os)) != ATTN_OK) return st;
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, dtype, workspace,
-                  workspace_bytes, nullptr, qs, os, stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, square(N), d, causal, scale, dtype, workspace,
+                  workspace_bytes, nullptr, qs, os, stream, qs);
+}
+
+int attn_fwd_rect(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int n_q, int n_k, int d, int q_offset, int causal, float scale,
+                  int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, Extent{n_q, n_k, q_offset}, d, causal, scale, dtype,
+                  nullptr, dense(H, n_q, d), dense(H, n_q, d), stream, dense(H, n_k, d));
+}
+
+int attn_bwd_rect(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int n_q, int n_k,
+                  int d, int q_offset, int causal, float scale, int dtype, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, Extent{n_q, n_k, q_offset}, d, causal,
+                  scale, dtype, workspace, workspace_bytes, nullptr, dense(H, n_q, d),
+                  dense(H, n_q, d), stream, dense(H, n_k, d));
 }
 
 // Backward-over-backward: the f32 backward's workspace (status, padded LSE,

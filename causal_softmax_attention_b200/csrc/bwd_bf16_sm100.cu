@@ -33,15 +33,21 @@
 //               red.global.add while the next tiles are computed.
 //   warp 12     MMA issuer (one elected lane).
 //   warp 13     TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
-//               the tile's LSE / D rows per query tile, two stages.
+//               the tile's LSE / D rows per query tile, three stages deep at
+//               d <= 64, two at d = 128.
 //   warps 14-15 idle (they complete the fourth warpgroup, which setmaxnreg
 //               needs to move registers to the dQ and element-wise warps).
-// TMEM (512 columns): region A [0,128) holds S^T, then P^T as bf16 (query q
-// at column 64*(q/64) + (q%64)/2); region B [128,256) holds dP^T, then dS^T as
-// bf16 in the same packing; dV [256,256+d), dK [256+d,256+2d). dQ takes
-// region B at d = 128 (after dK has read dS^T) and two buffers of its own at
-// smaller d. Because P^T and dS^T live in different regions, S^T of the next
-// tile only waits for dV and runs while the element-wise warps compute dS.
+// TMEM (512 columns). d = 128: region A [0,128) holds S^T, then P^T as bf16
+// (query q at column 64*(q/64) + (q%64)/2); region B [128,256) holds dP^T,
+// then dS^T as bf16 in the same packing; dV [256,384), dK [384,512). dQ takes
+// region B after dK has read dS^T. Because P^T and dS^T live in different
+// regions, S^T of the next tile only waits for dV and runs while the
+// element-wise warps compute dS. d <= 64: two S / P buffers [0,128) and
+// [128,256) (query tiles alternate), region B [256,384), dV, dK after it;
+// S^T of the next tile is issued into the other buffer before dV of this one,
+// and dQ of a tile lands in the first d columns of its own S buffer once dV
+// has read P from it, so no MMA of tile i+1 waits for the element-wise warps
+// of tile i.
 // Every hand-off is an mbarrier; every wait is bounded and reports a timeout.
 #include <cuda_bf16.h>
 
@@ -80,10 +86,10 @@ struct Roles {
   // sub-partition (16K registers = 512 per lane), and the budgets draw on
   // the registers the block was launched with.
   static constexpr uint32_t R_E = 136;
-  // (the block-mask walk costs the control and dQ warps a few registers at
-  // d <= 64, where their loops are otherwise tightest)
-  static constexpr uint32_t R_DQ = (D == 128 || !kMask) ? 144 : 128;
-  static constexpr uint32_t R_CTL = (D == 128 || !kMask) ? 96 : 112;
+  // (at d <= 64 a dQ row is half as long, and the control warps' pipelined
+  // issue loop and the block-mask walk need the registers it frees)
+  static constexpr uint32_t R_DQ = D == 128 ? 144 : 120;
+  static constexpr uint32_t R_CTL = D == 128 ? 96 : 120;
   static_assert(EG * R_E + R_DQ + R_CTL <= WGS * LAUNCH_REGS,
                 "register split exceeds the launch budget");
   static constexpr int DQ_READERS = 128;            // arrivals on B_DQREAD
@@ -100,7 +106,13 @@ struct BwdLayout {
   static constexpr int CHUNK = kTile * ROWB;    // bytes of one [128][CH] box
   static constexpr int TILE = NCH * CHUNK;      // bytes of one [128][D] bf16 tile
   static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128B : kSwizzle64B;
-  static constexpr int STAGES = 2;
+  // At d <= 64 tensor memory holds two S / P buffers, so S of the next query
+  // tile is computed while the element-wise warps still work on this one
+  // (and dQ of a tile lands in its S buffer once dV has read P); the Q / dO
+  // loads then run three stages deep to keep ahead of it.
+  static constexpr bool PIPE_S = D <= 64;
+  static constexpr int SBUF = PIPE_S ? 2 : 1;
+  static constexpr int STAGES = PIPE_S ? 3 : 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
   static constexpr int Q_OFF = V_OFF + TILE;              // [STAGES] tiles
@@ -122,30 +134,32 @@ struct BwdLayout {
   static constexpr bool EXACT = D == 128;
   static constexpr int ALLOC =
       EXACT ? BYTES : ((BYTES + 1024) > 118 * 1024 ? BYTES + 1024 : 118 * 1024);
-  // TMEM columns
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr bool DQ_OVER_DP = D == 128;
-  static constexpr int DQ_BUFS = DQ_OVER_DP ? 1 : 2;
-  static constexpr uint32_t T_DQ = DQ_OVER_DP ? T_DP : 256 + 2 * D;  // buffer b at T_DQ + b*D
+  // TMEM columns: S / P buffer b at T_S + 128 b; dP / dS; dV; dK. dQ takes
+  // region B (dP / dS) at d = 128, after dK has read dS; at d <= 64 the
+  // first D columns of its tile's S buffer, after dV has read P.
+  static constexpr uint32_t T_S = 0, T_DP = 128 * SBUF, T_DV = T_DP + 128, T_DK = T_DV + D;
+  static constexpr bool DQ_OVER_DP = !PIPE_S;
   static constexpr uint32_t T_COLS = 512;
-  static_assert(DQ_OVER_DP || T_DQ + DQ_BUFS * D <= T_COLS, "TMEM columns exceeded");
+  static_assert(T_DK + D <= T_COLS, "TMEM columns exceeded");
 };
 
+// Barrier slots: up to three Q / dO stages, up to two S buffers.
 enum Bar {
-  B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_SFULL = 5, B_DPFULL, B_PFULL, B_DSFULL, B_DVDONE,
+  B_KV = 0, B_QFULL = 1, B_QEMPTY = 4, B_SFULL = 7, B_DPFULL = 9, B_PFULL, B_DSFULL, B_DVDONE,
   B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2, B_DONE = B_DQREAD + 2, B_FINAL, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
 struct BwdParams {
-  const float* lse2;  // [BH][Np], LSE * log2(e), +inf past N
+  const float* lse2;  // [BH][Np], -LSE * log2(e), -inf past N
   const float* dvec;  // [BH][Np], D, 0 past N
   float* dq_acc;      // [BH][T][D/4][128][4]
   __nv_bfloat16* dk;  // rows at qs.row(bh, key), D channels each
   __nv_bfloat16* dv;
-  RowStrides qs;      // strides of dk and dv (those of q, k, v)
+  RowStrides ks;      // strides of dk and dv (those of k and v)
   int* status;
-  int N, Np, T, BH;
+  int N, Np, T, BH;   // query rows, rows padded to tiles, query tiles, heads
+  int Nk, Tk, q_off;  // keys, key tiles; query row r is position q_off + r
   int G;              // heads per scheduling group (see the CTA order in the kernel)
   int causal;
   const uint8_t* bmask;  // [T][T] tile kinds (0 none, 1 all, 2 key <= query in the tile), or null
@@ -191,19 +205,22 @@ template <int QC>
 __host__ __device__ constexpr uint32_t p_col(int q) { return QC * (q / QC) + (q % QC) / 2; }
 
 // P for this thread's key row over QC queries: p_u = 2^(S_u * scale*log2e -
-// LSE_u*log2e), packed as bf16 pairs. Queries u < thr are masked (kMasked);
-// off the diagonal tile nothing is, and the compare-and-select is skipped.
+// LSE_u*log2e), packed as bf16 pairs; the exponent's argument is formed two
+// queries at a time by one packed fp32 FMA (fma.rn.f32x2) against the row
+// term -LSE*log2e. Queries u < thr are masked (kMasked); off the diagonal
+// tile nothing is, and the compare-and-select is skipped.
 template <bool kMasked, int QC>
-__device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[QC], const float* lse,
+__device__ __forceinline__ void p_from_scores(const uint32_t (&sr)[QC], const float* nlse,
                                               float scale_log2, int thr, uint32_t (&pk)[QC / 2]) {
+  const uint64_t c2 = f2(scale_log2, scale_log2);
 #pragma unroll
   for (int u = 0; u < QC; u += 4) {
-    // one 16-byte broadcast load per four queries (shared-memory wavefronts are scarce)
-    const float4 l4 = *reinterpret_cast<const float4*>(lse + u);
-    float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), scale_log2, -l4.x));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), scale_log2, -l4.y));
-    float p2 = ex2_approx(fmaf(__uint_as_float(sr[u + 2]), scale_log2, -l4.z));
-    float p3 = ex2_approx(fmaf(__uint_as_float(sr[u + 3]), scale_log2, -l4.w));
+    // one 16-byte broadcast load per four queries: -LSE*log2e as two pairs
+    const ulonglong2 l4 = *reinterpret_cast<const ulonglong2*>(nlse + u);
+    const float2 x01 = f2_split(fma2(f2(__uint_as_float(sr[u]), __uint_as_float(sr[u + 1])), c2, l4.x));
+    const float2 x23 = f2_split(fma2(f2(__uint_as_float(sr[u + 2]), __uint_as_float(sr[u + 3])), c2, l4.y));
+    float p0 = ex2_approx(x01.x), p1 = ex2_approx(x01.y);
+    float p2 = ex2_approx(x23.x), p3 = ex2_approx(x23.y);
     if (kMasked) {
       if (u < thr) p0 = 0.f;
       if (u + 1 < thr) p1 = 0.f;
@@ -243,7 +260,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   // heads interleaved. The CTAs in flight then touch only a few heads' Q, dO
   // and dQ accumulator, which stay in L2 while every key tile of those heads
   // passes over them; the last group may be smaller.
-  const int per_group = p.T * p.G;
+  const int per_group = p.Tk * p.G;
   const int g0 = (blockIdx.x / per_group) * p.G;
   const int r = blockIdx.x % per_group;
   const int gs = min(p.G, p.BH - g0);
@@ -259,12 +276,17 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   uint32_t* s_kind2 = s_act + L::MASK_WORDS;
   const bool mask_bits =
       kMask && (p.T + R::THREADS - 1) / R::THREADS * (R::THREADS / 32) <= L::MASK_WORDS;
-  auto tile_kind = [&](int i) -> int {
+  // Queries u of query tile i with u < thr are masked for key row t: keys
+  // past N_k mask every query; the causal filter masks queries whose
+  // position q_off + 128 i + u is before the key's j0 + t (thr0 = j0 + t -
+  // q_off); a block mask's kind-2 tile masks u < t.
+  auto tile_thr = [&](int i, int t, int thr0) -> int {
     if constexpr (kMask) {
-      if (mask_bits) return bit_set(s_kind2, i) ? 2 : 1;
-      return p.bmask[static_cast<size_t>(i) * p.T + jt];
+      if (mask_bits) return bit_set(s_kind2, i) ? t : 0;
+      return p.bmask[static_cast<size_t>(i) * p.T + jt] == 2 ? t : 0;
     } else {
-      return !p.causal ? 1 : (i > jt ? 1 : (i == jt ? 2 : 0));
+      const int th = thr0 - i * kTile;
+      return th < 0 ? 0 : th;  // (above 128 every query of the tile is masked)
     }
   };
   auto next_tile = [&](int i) -> int {  // first tile after i that takes part (T if none)
@@ -274,7 +296,10 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       }
       return i;
     } else {
-      return p.causal ? max(i + 1, jt) : i + 1;
+      // under the causal filter the first query tile that sees this key tile:
+      // its last row's position q_off + 128 i + 127 must reach key j0
+      const int lo = j0 - p.q_off;
+      return max(i + 1, (p.causal && lo > kTile - 1) ? lo / kTile : 0);
     }
   };
   int i_first = kMask ? p.T : next_tile(-1);
@@ -288,13 +313,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_KV], 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(&bars[B_QFULL + s], 1);
       mbar_init(&bars[B_QEMPTY + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_DQFULL + s], 1);
       mbar_init(&bars[B_DQREAD + s], R::DQ_READERS);
+      mbar_init(&bars[B_SFULL + s], 1);
     }
-    mbar_init(&bars[B_SFULL], 1);
     mbar_init(&bars[B_DPFULL], 1);
     mbar_init(&bars[B_PFULL], R::E_THREADS);
     mbar_init(&bars[B_DSFULL], R::E_THREADS);
@@ -332,7 +359,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
   if (warp == R::TMA_WARP) {
     // ------------------------------------------------ TMA producer
     if (elect_one_sync()) {
-      const int hh = bh % p.qs.H, hb = bh / p.qs.H;  // head and batch: TMA coordinates
+      const int hh = bh % p.ks.H, hb = bh / p.ks.H;  // head and batch: TMA coordinates
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
@@ -345,9 +372,10 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       bool ok = true;
       int issued = 0;
       for (int it = 0, i = i_first; i < p.T; ++it, i = next_tile(i)) {
-        const int s = it & 1;
-        if (it >= 2 &&
-            !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
+        const int s = it % L::STAGES;
+        if (it >= L::STAGES &&
+            !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - L::STAGES) / L::STAGES) & 1, p.wait_cycles,
+                             abort_flag)))
           break;
         const int i0 = i * kTile;
         uint64_t* bar = &bars[B_QFULL + s];
@@ -367,15 +395,19 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       if (!ok) fail();
       // Every load issued has landed before the CTA can exit (bounded).
       mbar_wait(&bars[B_KV], 0, p.wait_cycles, never);
-      for (int w = issued > 2 ? issued - 2 : 0; w < issued; ++w)
-        mbar_wait(&bars[B_QFULL + (w & 1)], (w >> 1) & 1, p.wait_cycles, never);
+      for (int w = issued > L::STAGES ? issued - L::STAGES : 0; w < issued; ++w)
+        mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_cycles, never);
     }
     __syncwarp();
   } else if (warp == R::MMA_WARP) {
     // ------------------------------------------------ MMA issuer
-    // Issue order per query tile i: dV(i), S(i+1), dK(i), dQ(i), dP(i+1); S(0)
-    // and dP(0) before the loop. Each wait guards one TMEM or shared-memory
-    // region against the MMA that overwrites it.
+    // Each wait guards one TMEM or shared-memory region against the MMA that
+    // overwrites it. d = 128, per query tile i: dV(i), S(i+1), dK(i), dQ(i),
+    // dP(i+1), with S(0) and dP(0) before the loop; S(i+1) overwrites P(i)
+    // and so waits for dV(i). d <= 64 (two S buffers): S(i+1), dV(i), dK(i),
+    // dQ(i), dP(i+1): S(i+1) goes into the other buffer as soon as its last
+    // reader (the read-out of dQ(i-1)) is done, so the element-wise warps
+    // find it ready when they finish dS(i).
     if (elect_one_sync()) {
       const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sdS = sbase + L::DS_OFF;
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
@@ -384,15 +416,17 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       auto wait = [&](int b, uint32_t parity) {
         return mbar_wait(&bars[b], parity, p.wait_cycles, abort_flag);
       };
-      auto stage_q = [&](int it) { return sbase + L::Q_OFF + (it & 1) * L::TILE; };
-      auto stage_do = [&](int it) { return sbase + L::DO_OFF + (it & 1) * L::TILE; };
-      // S^T(it) = K_j Q_i^T -> region A
+      auto stage_q = [&](int it) { return sbase + L::Q_OFF + (it % L::STAGES) * L::TILE; };
+      auto stage_do = [&](int it) { return sbase + L::DO_OFF + (it % L::STAGES) * L::TILE; };
+      auto qfull = [&](int it) { return wait(B_QFULL + it % L::STAGES, (it / L::STAGES) & 1); };
+      auto sbuf = [&](int it) { return L::T_S + 128 * (it % L::SBUF); };
+      // S^T(it) = K_j Q_i^T -> S buffer it % SBUF
       auto issue_s = [&](int it) {
         const uint32_t sQ = stage_q(it);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::T_S, desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
-        if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL]);
+          mma_ss(tmem + sbuf(it), desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
+        if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL + it % L::SBUF]);
       };
       // dP^T(it) = V_j dO_i^T -> region B
       auto issue_dp = [&](int it) {
@@ -402,61 +436,87 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
           mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
         mma_commit(&bars[B_DPFULL]);
       };
+      // dV_j += P^T dO_i, P^T read from the tile's S buffer (K = 128 queries)
+      auto issue_dv = [&](int it) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::T_DV, tmem + sbuf(it) + p_col<QC>(16 * kk),
+                 desc_mnmajor<D>(stage_do(it), kk), ID_KV, (it > 0 || kk > 0));
+        mma_commit(&bars[B_DVDONE]);
+      };
+      // dK_j += dS^T Q_i, dS^T read from region B
+      auto issue_dk = [&](int it) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk),
+                 desc_mnmajor<D>(stage_q(it), kk), ID_KV, (it > 0 || kk > 0));
+        mma_commit(&bars[B_DKDONE]);
+      };
+      // dQ_i = dS K_j (dS from shared memory) -> region B (d = 128) or the
+      // tile's S buffer (d <= 64); Q_i / dO_i's stage is free afterwards
+      auto issue_dq = [&](int it) {
+        const uint32_t dst = L::DQ_OVER_DP ? L::T_DP : sbuf(it);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + dst, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
+        mma_commit(&bars[B_DQFULL + (it & 1)]);
+        mma_commit(&bars[B_QEMPTY + it % L::STAGES]);
+      };
       bool ok = true;
-      if (i_first < p.T && (ok = wait(B_KV, 0) && wait(B_QFULL, 0))) {
+      if (i_first < p.T && (ok = wait(B_KV, 0) && qfull(0))) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
       for (int it = 0, i = i_first; ok && i < p.T; ++it, i = next_tile(i)) {
-        const int s = it & 1;
         const bool more = next_tile(i) < p.T;
-        // dV_j += P^T dO_i, P^T read from region A (K = 128 queries, 16 per step)
-        if (!(ok = wait(B_PFULL, it & 1))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DV, tmem + L::T_S + p_col<QC>(16 * kk), desc_mnmajor<D>(stage_do(it), kk),
-                 ID_KV, (it > 0 || kk > 0));
-        mma_commit(&bars[B_DVDONE]);
-        if (more) {
-          // S^T(it+1) overwrites P^T(it), which dV(it) reads.
-          if (!(ok = wait(B_QFULL + (s ^ 1), ((it + 1) >> 1) & 1))) break;
+        if constexpr (L::PIPE_S) {
+          if (more) {
+            // S(it+1) reuses the buffer of tile it-1, free once dQ(it-1) is read out
+            if (!(ok = qfull(it + 1))) break;
+            if (it >= 1 && !(ok = wait(B_DQREAD + ((it - 1) & 1), ((it - 1) >> 1) & 1))) break;
+            tc_fence_after();
+            issue_s(it + 1);
+          }
+          if (!(ok = wait(B_PFULL, it & 1))) break;
+          tc_fence_after();
+          issue_dv(it);
+          if (!(ok = wait(B_DSFULL, it & 1))) break;
+          tc_fence_after();
+          issue_dk(it);
+          // dQ(it) overwrites P(it), which dV(it) reads
           if (!(ok = wait(B_DVDONE, it & 1))) break;
           tc_fence_after();
-          issue_s(it + 1);
-        }
-        // dK_j += dS^T Q_i, dS^T read from region B
-        if (!(ok = wait(B_DSFULL, it & 1))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk), desc_mnmajor<D>(stage_q(it), kk),
-                 ID_KV, (it > 0 || kk > 0));
-        mma_commit(&bars[B_DKDONE]);
-        // dQ_i = dS K_j (dS from shared memory)
-        const int b = it % L::DQ_BUFS;
-        if (L::DQ_OVER_DP) {
-          if (!(ok = wait(B_DKDONE, it & 1))) break;  // dQ(it) overwrites dS^T(it)
-        } else if (it >= L::DQ_BUFS) {
-          if (!(ok = wait(B_DQREAD + b, (it / L::DQ_BUFS - 1) & 1))) break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DQ + b * D, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q,
-                 kk > 0);
-        mma_commit(&bars[B_DQFULL + b]);
-        mma_commit(&bars[B_QEMPTY + s]);
-        if (more) {
-          // dP^T(it+1) overwrites region B: dQ(it) at d = 128, dS^T(it) otherwise.
-          if (L::DQ_OVER_DP) {
-            if (!(ok = wait(B_DQREAD, it & 1))) break;
-          } else {
+          issue_dq(it);
+          if (more) {
+            // dP(it+1) overwrites dS^T(it), which dK(it) reads
             if (!(ok = wait(B_DKDONE, it & 1))) break;
+            tc_fence_after();
+            issue_dp(it + 1);
           }
+        } else {
+          if (!(ok = wait(B_PFULL, it & 1))) break;
           tc_fence_after();
-          issue_dp(it + 1);
+          issue_dv(it);
+          if (more) {
+            // S^T(it+1) overwrites P^T(it), which dV(it) reads.
+            if (!(ok = qfull(it + 1))) break;
+            if (!(ok = wait(B_DVDONE, it & 1))) break;
+            tc_fence_after();
+            issue_s(it + 1);
+          }
+          if (!(ok = wait(B_DSFULL, it & 1))) break;
+          tc_fence_after();
+          issue_dk(it);
+          if (!(ok = wait(B_DKDONE, it & 1))) break;  // dQ(it) overwrites dS^T(it)
+          tc_fence_after();
+          issue_dq(it);
+          if (more) {
+            // dP^T(it+1) overwrites region B, where dQ(it) lands
+            if (!(ok = wait(B_DQREAD + (it & 1), (it >> 1) & 1))) break;
+            tc_fence_after();
+            issue_dp(it + 1);
+          }
         }
       }
       if (ok) {
@@ -480,18 +540,19 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     };
     bool ok = true;
     for (int it = 0, i = i_first; i < p.T; ++it, i = next_tile(i)) {
-      const int b = it % L::DQ_BUFS;
-      if (!(ok = wait_w(B_DQFULL + b, (it / L::DQ_BUFS) & 1))) break;
+      const int b = it & 1;
+      if (!(ok = wait_w(B_DQFULL + b, (it >> 1) & 1))) break;
       tc_fence_after();
       // The whole row first, so the columns are released before the atomics.
       uint32_t r[D];
 #pragma unroll
       for (int c = 0; c < D; c += 32)
-        tmem_ld32(lane_base + L::T_DQ + b * D + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
+        tmem_ld32(lane_base + (L::DQ_OVER_DP ? L::T_DP : L::T_S + 128 * (it % L::SBUF)) + c,
+                  *reinterpret_cast<uint32_t(*)[32]>(r + c));
       tmem_ld_wait(r);
       tc_fence_before();
       mbar_arrive(&bars[B_DQREAD + b]);
-      if (i * kTile + t < p.N) {
+      if (i * kTile + t < p.N) {  // a query row of this head
         float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
         // Metered: a burst of reductions fills the sub-partition's memory
         // instruction queue, and the element-wise warps' TMEM and shared-memory
@@ -514,6 +575,8 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int key = j0 + t;
     const int qb = QC * g;
+    // causal threshold of this key row at query tile 0 (none without the filter)
+    const int thr0 = p.causal ? key - p.q_off : -(1 << 30);
     // Outcome of a wait, made uniform across the warp: the TMEM accesses that
     // follow are warp-collective, so a warp must never split on a timeout.
     auto wait_w = [&](int b, uint32_t parity) {
@@ -522,21 +585,23 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     bool ok = true;
     int it = 0;
     for (int i = i_first; i < p.T; ++it, i = next_tile(i)) {
-      const int s = it & 1;
-      if (!(ok = wait_w(B_QFULL + s, (it >> 1) & 1))) break;  // LSE_i, D_i in shared memory
+      const int s = it % L::STAGES;
+      // LSE_i, D_i in shared memory
+      if (!(ok = wait_w(B_QFULL + s, (it / L::STAGES) & 1))) break;
       const float* lse_s = s_lse + s * 128;
       const float* d_s = s_dv + s * 128;
       // queries with local index < thr are masked for this key row (kind 2:
       // the key must not lie after the query inside the tile)
-      const int thr = key >= p.N ? 128 : (tile_kind(i) == 2 ? t : 0);
+      const int thr = key >= p.Nk ? kTile : tile_thr(i, t, thr0);
 
       // ---- P^T = exp2(S^T * scale*log2e - LSE*log2e) -> bf16 into region A
-      if (!(ok = wait_w(B_SFULL, it & 1))) break;
+      const uint32_t t_s = L::T_S + 128 * (it % L::SBUF);  // this tile's S / P buffer
+      if (!(ok = wait_w(B_SFULL + it % L::SBUF, (it / L::SBUF) & 1))) break;
       tc_fence_after();
       uint32_t pk[QC / 2];  // this thread's QC P values as bf16 pairs, kept for the dS pass
       {
         uint32_t sr[QC];
-        tmem_ld<QC>(lane_base + L::T_S + qb, sr);
+        tmem_ld<QC>(lane_base + t_s + qb, sr);
         tmem_ld_wait(sr);
         // Only the diagonal tile and the key tile past N mask anything.
         if (__any_sync(0xffffffffu, thr > qb))
@@ -548,7 +613,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       // overwrite the first half of them
 #pragma unroll
       for (int c = 0; c < QC / 2; c += 16)
-        tmem_st16(lane_base + L::T_S + p_col<QC>(qb) + c,
+        tmem_st16(lane_base + t_s + p_col<QC>(qb) + c,
                   *reinterpret_cast<uint32_t(*)[16]>(pk + c));
       tmem_st_wait();
       tc_fence_before();
@@ -565,13 +630,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 #pragma unroll
         for (int u = 0; u < QC; u += 4) {
           const int q0 = qb + u;
-          const float4 d4 = *reinterpret_cast<const float4*>(d_s + q0);
+          const ulonglong2 d4 = *reinterpret_cast<const ulonglong2*>(d_s + q0);
           const float2 pa = unpack_bf16x2(pk[u / 2]);
           const float2 pb = unpack_bf16x2(pk[u / 2 + 1]);
-          dk[u / 2] = pack_bf16x2(pa.x * (__uint_as_float(dr[u]) - d4.x),
-                                  pa.y * (__uint_as_float(dr[u + 1]) - d4.y));
-          dk[u / 2 + 1] = pack_bf16x2(pb.x * (__uint_as_float(dr[u + 2]) - d4.z),
-                                      pb.y * (__uint_as_float(dr[u + 3]) - d4.w));
+          const float2 x01 = f2_split(mul2(f2(pa.x, pa.y),
+              sub2(f2(__uint_as_float(dr[u]), __uint_as_float(dr[u + 1])), d4.x)));
+          const float2 x23 = f2_split(mul2(f2(pb.x, pb.y),
+              sub2(f2(__uint_as_float(dr[u + 2]), __uint_as_float(dr[u + 3])), d4.y)));
+          dk[u / 2] = pack_bf16x2(x01.x, x01.y);
+          dk[u / 2 + 1] = pack_bf16x2(x23.x, x23.y);
         }
       }
       // dS^T for dK (TMEM A operand); all dP^T columns of the group were read above
@@ -598,9 +665,9 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       tc_fence_after();
       // Epilogue: dV_j and scale * dK_j rows -> bf16, group g writing channels
       // [g*E_CH, (g+1)*E_CH). All lanes load; only the stores are predicated.
-      const bool key_ok = key < p.N;
-      __nv_bfloat16* dv_row = p.dv + p.qs.row(bh, key_ok ? key : 0);
-      __nv_bfloat16* dk_row = p.dk + p.qs.row(bh, key_ok ? key : 0);
+      const bool key_ok = key < p.Nk;
+      __nv_bfloat16* dv_row = p.dv + p.ks.row(bh, key_ok ? key : 0);
+      __nv_bfloat16* dk_row = p.dk + p.ks.row(bh, key_ok ? key : 0);
       constexpr int W = R::E_CH >= 32 ? 32 : R::E_CH;
       const bool any = it > 0;  // a key tile that meets no query tile has dK = dV = 0
 #pragma unroll 1
@@ -646,8 +713,9 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 
 template <int D>
 cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, void* dv, int BH,
-                              int N, bool causal, float scale, uint64_t wait_cycles, int inject,
-                              const uint8_t* bmask, const RowStrides& qs, cudaStream_t s) {
+                              const Extent& ex, bool causal, float scale, uint64_t wait_cycles,
+                              int inject, const uint8_t* bmask, const RowStrides& ks,
+                              cudaStream_t s) {
   using L = BwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = bmask ? attn_bwd_bf16_sm100_kernel<D, true> : attn_bwd_bf16_sm100_kernel<D, false>;
@@ -672,10 +740,13 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.status = ws.status;
-  p.N = N;
+  p.N = ex.nq;
   p.Np = ws.Np;
   p.T = ws.Np / kTile;
   p.BH = BH;
+  p.Nk = ex.nk;
+  p.Tk = (ex.nk + kTile - 1) / kTile;
+  p.q_off = ex.q_off;
   // Heads per group: as many as fit, with their Q and dO tiles (bf16) and dQ
   // accumulator (fp32), in about a third of L2.
   int dev = 0, l2 = 0;
@@ -686,12 +757,12 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.bmask = bmask;
-  p.qs = qs;
+  p.ks = ks;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_cycles = wait_cycles;
   p.inject_fault = inject;
-  const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
+  const unsigned grid = static_cast<unsigned>(p.Tk) * static_cast<unsigned>(BH);
   kern<<<grid, Roles<D>::THREADS, L::ALLOC, s>>>(m.a, m.b, m.c, m.d, p);
   return cudaGetLastError();
 }
@@ -699,19 +770,19 @@ cudaError_t launch_bwd_bf16_d(const TmaMaps& m, const Workspace& ws, void* dk, v
 }  // namespace
 
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
-                            int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, const uint8_t* block_mask, const RowStrides& qs,
-                            cudaStream_t s) {
+                            const Extent& ex, int d, bool causal, float scale,
+                            uint64_t wait_limit_cycles, int inject_fault,
+                            const uint8_t* block_mask, const RowStrides& ks, cudaStream_t s) {
   switch (d) {
     case 32:
-      return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, block_mask, qs, s);
+      return launch_bwd_bf16_d<32>(maps, ws, dk, dv, BH, ex, causal, scale, wait_limit_cycles,
+                                   inject_fault, block_mask, ks, s);
     case 64:
-      return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                   inject_fault, block_mask, qs, s);
+      return launch_bwd_bf16_d<64>(maps, ws, dk, dv, BH, ex, causal, scale, wait_limit_cycles,
+                                   inject_fault, block_mask, ks, s);
     case 128:
-      return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, N, causal, scale, wait_limit_cycles,
-                                    inject_fault, block_mask, qs, s);
+      return launch_bwd_bf16_d<128>(maps, ws, dk, dv, BH, ex, causal, scale, wait_limit_cycles,
+                                    inject_fault, block_mask, ks, s);
     default:
       return cudaErrorInvalidValue;
   }

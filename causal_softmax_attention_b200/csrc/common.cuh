@@ -37,7 +37,7 @@ inline RowStrides contiguous_strides(int H, int N, int d) {
 // Workspace carved out of the caller's buffer for one backward call.
 struct Workspace {
   int* status;     // device status word
-  float* lse_pad;  // [BH][Np]: LSE (f32 path) or LSE * log2(e) (bf16 path); +inf past N
+  float* lse_pad;  // [BH][Np]: LSE, +inf past N (f32 path); -LSE * log2(e), -inf past N (bf16)
   float* d_pad;    // [BH][Np]: D_i = sum_c dO_ic O_ic; 0 past N
   float* dq_acc;   // [BH][Np][d] fp32 dQ accumulator (bf16 path only)
   int Np;          // N rounded up to whole 128-row tiles
@@ -62,13 +62,23 @@ cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse,
                               cudaStream_t s);
 cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const RowStrides& qs,
                               const Workspace& ws, cudaStream_t s);
+// Query and key extents of a head: N_q query rows, N_k keys; query row r
+// stands for position q_off + r and key j for position j, and the causal
+// filter keeps a score when the query's position is at least the key's. The
+// square problem is {N, N, 0}.
+struct Extent {
+  int nq, nk, q_off;
+};
+
+// qs: strides of q and dq; ks: of k, v, dk, dv; os: of o and dout.
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
-                           int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
-                           const RowStrides& os, cudaStream_t s);
+                           int BH, const Extent& ex, int d, bool causal, float scale,
+                           const RowStrides& qs, const RowStrides& ks, const RowStrides& os,
+                           cudaStream_t s);
 cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
-                           float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                           float scale, const RowStrides& qs, const RowStrides& os,
-                           const Workspace& ws, cudaStream_t s);
+                           float* dq, float* dk, float* dv, int BH, const Extent& ex, int d,
+                           bool causal, float scale, const RowStrides& qs, const RowStrides& ks,
+                           const RowStrides& os, const Workspace& ws, cudaStream_t s);
 
 // Backward-over-backward on the CUDA cores (contiguous fp32 [BH][N][d]);
 // needs the preprocess's lse_pad and d_pad in `ws`, and writes the two row
@@ -87,13 +97,15 @@ struct TmaMaps {
 };
 // block_mask: device [T][T] tile kinds (0 none, 1 all, 2 key <= query inside
 // the tile), T = ceil(N / 128), or null for the causal / full filter.
-cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
-                            int d, bool causal, float scale, const uint8_t* block_mask,
-                            const RowStrides& os, cudaStream_t s);
+// (q and o have ex.nq rows per head, k and v ex.nk; a block mask is square,
+// ex.nq == ex.nk, q_off == 0)
+cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH,
+                            const Extent& ex, int d, bool causal, float scale,
+                            const uint8_t* block_mask, const RowStrides& os, cudaStream_t s);
 cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, void* dv, int BH,
-                            int N, int d, bool causal, float scale, uint64_t wait_limit_cycles,
-                            int inject_fault, const uint8_t* block_mask, const RowStrides& qs,
-                            cudaStream_t s);
+                            const Extent& ex, int d, bool causal, float scale,
+                            uint64_t wait_limit_cycles, int inject_fault,
+                            const uint8_t* block_mask, const RowStrides& ks, cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 

@@ -45,7 +45,8 @@ template <int DP>
 __global__ void __launch_bounds__(128)
     fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                    const float* __restrict__ v, float* __restrict__ o, float* __restrict__ lse,
-                   int N, int d, int causal, float scale, RowStrides qs, RowStrides os) {
+                   Extent ex, int d, int causal, float scale, RowStrides qs, RowStrides ks,
+                   RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;  // rows per block
   __shared__ float sK[kRowsTile][DP];
@@ -54,23 +55,23 @@ __global__ void __launch_bounds__(128)
   const int row = blockIdx.x * R + threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
   const float* qh = q + qs.head(bh);
-  const float* kh = k + qs.head(bh);
-  const float* vh = v + qs.head(bh);
+  const float* kh = k + ks.head(bh);
+  const float* vh = v + ks.head(bh);
 
   float qr[32], acc[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
-    qr[c] = (row < N && ch < d) ? qh[row * qs.sn + ch] : 0.f;
+    qr[c] = (row < ex.nq && ch < d) ? qh[row * qs.sn + ch] : 0.f;
     acc[c] = 0.f;
   }
   float m = -INFINITY, z = 0.f;
-  const int last_row = min(N - 1, blockIdx.x * R + R - 1);
-  const int key_end = causal ? last_row + 1 : N;
+  const int last_row = min(ex.nq - 1, blockIdx.x * R + R - 1);
+  const int key_end = causal ? min(ex.nk, last_row + ex.q_off + 1) : ex.nk;
   for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sK, kh, k0, N, d, qs.sn);
-    load_tile<DP>(sV, vh, k0, N, d, qs.sn);
+    load_tile<DP>(sK, kh, k0, ex.nk, d, ks.sn);
+    load_tile<DP>(sV, vh, k0, ex.nk, d, ks.sn);
     __syncthreads();
     float s[kRowsTile];
     float mx = -INFINITY;
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(128)
       for (int c = 0; c < 32; ++c) part_dot = fmaf(qr[c], sK[u][32 * part + c], part_dot);
       const float dot = group_sum<TPR>(part_dot);
       const int key = k0 + u;
-      const bool keep = key < N && (!causal || key <= row);
+      const bool keep = key < ex.nk && (!causal || key <= row + ex.q_off);
       s[u] = keep ? dot * scale : -INFINITY;
       mx = fmaxf(mx, s[u]);
     }
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(128)
     z = z * alpha + zt;
     m = m_new;
   }
-  if (row < N) {
+  if (row < ex.nq) {
     const float inv = 1.f / z;
     float* orow = o + os.row(bh, row);
 #pragma unroll
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(128)
       const int ch = 32 * part + c;
       if (ch < d) orow[ch] = acc[c] * inv;
     }
-    if (part == 0) lse[static_cast<size_t>(bh) * N + row] = m + logf(z);
+    if (part == 0) lse[static_cast<size_t>(bh) * ex.nq + row] = m + logf(z);
   }
 }
 
@@ -119,8 +120,8 @@ __global__ void __launch_bounds__(128)
     bwd_dkdv_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                         const float* __restrict__ v, const float* __restrict__ dout,
                         const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
-                        float* __restrict__ dk, float* __restrict__ dv, int N, int Np, int d,
-                        int causal, float scale, RowStrides qs, RowStrides os) {
+                        float* __restrict__ dk, float* __restrict__ dv, Extent ex, int Np, int d,
+                        int causal, float scale, RowStrides qs, RowStrides ks, RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;
   __shared__ float sQ[kRowsTile][DP];
@@ -129,22 +130,23 @@ __global__ void __launch_bounds__(128)
   const int bh = blockIdx.y;
   const int key = blockIdx.x * R + threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
-  const long long off = qs.head(bh), ooff = os.head(bh);
+  const long long off = qs.head(bh), koff = ks.head(bh), ooff = os.head(bh);
   float kr[32], vr[32], gk[32], gv[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
-    const bool in = key < N && ch < d;
-    kr[c] = in ? k[off + key * qs.sn + ch] : 0.f;
-    vr[c] = in ? v[off + key * qs.sn + ch] : 0.f;
+    const bool in = key < ex.nk && ch < d;
+    kr[c] = in ? k[koff + key * ks.sn + ch] : 0.f;
+    vr[c] = in ? v[koff + key * ks.sn + ch] : 0.f;
     gk[c] = gv[c] = 0.f;
   }
+  // the first query row that can see this block's first key: row + q_off >= key
   const int first_key = blockIdx.x * R;
-  const int q_begin = causal ? (first_key / kRowsTile) * kRowsTile : 0;
-  for (int q0 = q_begin; q0 < N; q0 += kRowsTile) {
+  const int q_begin = causal ? (max(0, first_key - ex.q_off) / kRowsTile) * kRowsTile : 0;
+  for (int q0 = q_begin; q0 < ex.nq; q0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sQ, q + off, q0, N, d, qs.sn);
-    load_tile<DP>(sdO, dout + ooff, q0, N, d, os.sn);
+    load_tile<DP>(sQ, q + off, q0, ex.nq, d, qs.sn);
+    load_tile<DP>(sdO, dout + ooff, q0, ex.nq, d, os.sn);
     if (threadIdx.x < kRowsTile) {
       sL[threadIdx.x] = lse_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
       sD[threadIdx.x] = d_pad[static_cast<size_t>(bh) * Np + q0 + threadIdx.x];
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(128)
       }
       const float s = group_sum<TPR>(ps) * scale;
       const float dp = group_sum<TPR>(pd);
-      const bool keep = qi < N && key < N && (!causal || qi >= key);
+      const bool keep = qi < ex.nq && key < ex.nk && (!causal || qi + ex.q_off >= key);
       const float p = keep ? expf(s - sL[u]) : 0.f;
       const float ds = p * (dp - sD[u]);
 #pragma unroll
@@ -171,13 +173,13 @@ __global__ void __launch_bounds__(128)
       }
     }
   }
-  if (key < N) {
+  if (key < ex.nk) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       const int ch = 32 * part + c;
       if (ch < d) {
-        dk[off + key * qs.sn + ch] = gk[c] * scale;
-        dv[off + key * qs.sn + ch] = gv[c];
+        dk[koff + key * ks.sn + ch] = gk[c] * scale;
+        dv[koff + key * ks.sn + ch] = gv[c];
       }
     }
   }
@@ -189,8 +191,8 @@ __global__ void __launch_bounds__(128)
     bwd_dq_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                       const float* __restrict__ v, const float* __restrict__ dout,
                       const float* __restrict__ lse_pad, const float* __restrict__ d_pad,
-                      float* __restrict__ dq, int N, int Np, int d, int causal, float scale,
-                      RowStrides qs, RowStrides os) {
+                      float* __restrict__ dq, Extent ex, int Np, int d, int causal, float scale,
+                      RowStrides qs, RowStrides ks, RowStrides os) {
   constexpr int TPR = DP / 32;
   constexpr int R = 128 / TPR;
   __shared__ float sK[kRowsTile][DP];
@@ -203,19 +205,19 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const int ch = 32 * part + c;
-    const bool in = row < N && ch < d;
+    const bool in = row < ex.nq && ch < d;
     qr[c] = in ? q[off + row * qs.sn + ch] : 0.f;
     dor[c] = in ? dout[ooff + row * os.sn + ch] : 0.f;
     g[c] = 0.f;
   }
   const float Li = lse_pad[static_cast<size_t>(bh) * Np + min(row, Np - 1)];
   const float Di = d_pad[static_cast<size_t>(bh) * Np + min(row, Np - 1)];
-  const int last_row = min(N - 1, blockIdx.x * R + R - 1);
-  const int key_end = causal ? last_row + 1 : N;
+  const int last_row = min(ex.nq - 1, blockIdx.x * R + R - 1);
+  const int key_end = causal ? min(ex.nk, last_row + ex.q_off + 1) : ex.nk;
   for (int k0 = 0; k0 < key_end; k0 += kRowsTile) {
     __syncthreads();
-    load_tile<DP>(sK, k + off, k0, N, d, qs.sn);
-    load_tile<DP>(sV, v + off, k0, N, d, qs.sn);
+    load_tile<DP>(sK, k + ks.head(bh), k0, ex.nk, d, ks.sn);
+    load_tile<DP>(sV, v + ks.head(bh), k0, ex.nk, d, ks.sn);
     __syncthreads();
 #pragma unroll 4
     for (int u = 0; u < kRowsTile; ++u) {
@@ -228,14 +230,14 @@ __global__ void __launch_bounds__(128)
       }
       const float s = group_sum<TPR>(ps) * scale;
       const float dp = group_sum<TPR>(pd);
-      const bool keep = row < N && key < N && (!causal || key <= row);
+      const bool keep = row < ex.nq && key < ex.nk && (!causal || key <= row + ex.q_off);
       const float p = keep ? expf(s - Li) : 0.f;
       const float ds = p * (dp - Di);
 #pragma unroll
       for (int c = 0; c < 32; ++c) g[c] = fmaf(ds, sK[u][32 * part + c], g[c]);
     }
   }
-  if (row < N) {
+  if (row < ex.nq) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       const int ch = 32 * part + c;
@@ -246,49 +248,50 @@ __global__ void __launch_bounds__(128)
 
 template <int DP>
 cudaError_t fwd_f32_dp(const float* q, const float* k, const float* v, float* o, float* lse,
-                       int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
-                       const RowStrides& os, cudaStream_t s) {
+                       int BH, const Extent& ex, int d, bool causal, float scale,
+                       const RowStrides& qs, const RowStrides& ks, const RowStrides& os,
+                       cudaStream_t s) {
   constexpr int R = 128 / (DP / 32);
-  dim3 grid((N + R - 1) / R, BH);
-  fwd_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, o, lse, N, d, causal, scale, qs, os);
+  dim3 grid((ex.nq + R - 1) / R, BH);
+  fwd_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, o, lse, ex, d, causal, scale, qs, ks, os);
   return cudaGetLastError();
 }
 
 template <int DP>
 cudaError_t bwd_f32_dp(const float* q, const float* k, const float* v, const float* dout,
-                       float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                       float scale, const RowStrides& qs, const RowStrides& os,
-                       const Workspace& ws, cudaStream_t s) {
+                       float* dq, float* dk, float* dv, int BH, const Extent& ex, int d,
+                       bool causal, float scale, const RowStrides& qs, const RowStrides& ks,
+                       const RowStrides& os, const Workspace& ws, cudaStream_t s) {
   constexpr int R = 128 / (DP / 32);
-  dim3 grid((N + R - 1) / R, BH);
-  bwd_dkdv_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dk, dv, N,
-                                               ws.Np, d, causal, scale, qs, os);
+  bwd_dkdv_f32_kernel<DP><<<dim3((ex.nk + R - 1) / R, BH), 128, 0, s>>>(
+      q, k, v, dout, ws.lse_pad, ws.d_pad, dk, dv, ex, ws.Np, d, causal, scale, qs, ks, os);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_f32_kernel<DP><<<grid, 128, 0, s>>>(q, k, v, dout, ws.lse_pad, ws.d_pad, dq, N, ws.Np,
-                                             d, causal, scale, qs, os);
+  bwd_dq_f32_kernel<DP><<<dim3((ex.nq + R - 1) / R, BH), 128, 0, s>>>(
+      q, k, v, dout, ws.lse_pad, ws.d_pad, dq, ex, ws.Np, d, causal, scale, qs, ks, os);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
-                           int BH, int N, int d, bool causal, float scale, const RowStrides& qs,
-                           const RowStrides& os, cudaStream_t s) {
-  if (d <= 32) return fwd_f32_dp<32>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
-  if (d <= 64) return fwd_f32_dp<64>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
-  return fwd_f32_dp<128>(q, k, v, o, lse, BH, N, d, causal, scale, qs, os, s);
+                           int BH, const Extent& ex, int d, bool causal, float scale,
+                           const RowStrides& qs, const RowStrides& ks, const RowStrides& os,
+                           cudaStream_t s) {
+  if (d <= 32) return fwd_f32_dp<32>(q, k, v, o, lse, BH, ex, d, causal, scale, qs, ks, os, s);
+  if (d <= 64) return fwd_f32_dp<64>(q, k, v, o, lse, BH, ex, d, causal, scale, qs, ks, os, s);
+  return fwd_f32_dp<128>(q, k, v, o, lse, BH, ex, d, causal, scale, qs, ks, os, s);
 }
 
 cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
-                           float* dq, float* dk, float* dv, int BH, int N, int d, bool causal,
-                           float scale, const RowStrides& qs, const RowStrides& os,
-                           const Workspace& ws, cudaStream_t s) {
+                           float* dq, float* dk, float* dv, int BH, const Extent& ex, int d,
+                           bool causal, float scale, const RowStrides& qs, const RowStrides& ks,
+                           const RowStrides& os, const Workspace& ws, cudaStream_t s) {
   if (d <= 32)
-    return bwd_f32_dp<32>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
+    return bwd_f32_dp<32>(q, k, v, dout, dq, dk, dv, BH, ex, d, causal, scale, qs, ks, os, ws, s);
   if (d <= 64)
-    return bwd_f32_dp<64>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
-  return bwd_f32_dp<128>(q, k, v, dout, dq, dk, dv, BH, N, d, causal, scale, qs, os, ws, s);
+    return bwd_f32_dp<64>(q, k, v, dout, dq, dk, dv, BH, ex, d, causal, scale, qs, ks, os, ws, s);
+  return bwd_f32_dp<128>(q, k, v, dout, dq, dk, dv, BH, ex, d, causal, scale, qs, ks, os, ws, s);
 }
 
 }  // namespace csa

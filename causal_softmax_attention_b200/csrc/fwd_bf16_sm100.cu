@@ -92,7 +92,8 @@ struct FwdParams {
   RowStrides os;     // strides of o
   float* lse;        // [BH][N]
   int* status;
-  int N, T, BH;
+  int N, T, BH;      // query rows, query tiles, heads
+  int Nk, Tk, q_off; // keys, key tiles; query row r is position q_off + r
   int G;             // heads per scheduling group (see the CTA order)
   int causal;
   const uint8_t* bmask;  // [T][T] tile kinds (0 none, 1 all, 2 key <= query in the tile), or null
@@ -161,14 +162,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       return !p.causal ? 1 : (j < it_q ? 1 : (j == it_q ? 2 : 0));
     }
   };
-  auto next_tile = [&](int j) -> int {  // first tile after j that takes part (T if none)
+  // last key tile the causal filter lets this query tile see (key position
+  // <= q_off + its last row's index)
+  const int j_last = min(p.Tk - 1, (p.q_off + i0 + kTile - 1) / kTile);
+  auto next_tile = [&](int j) -> int {  // first tile after j that takes part (Tk if none)
     if constexpr (kMask) {
-      if (mask_bits) return next_set_bit(s_act, p.T, j);
-      for (++j; j < p.T && mask_row[j] == 0; ++j) {
+      if (mask_bits) return next_set_bit(s_act, p.Tk, j);
+      for (++j; j < p.Tk && mask_row[j] == 0; ++j) {
       }
       return j;
     } else {
-      return (p.causal && j + 1 > it_q) ? p.T : j + 1;
+      return (p.causal && j + 1 > j_last) ? p.Tk : j + 1;
     }
   };
 
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       bool ok = true;
       int issued = 0;
-      for (int jt = 0, j = j_first; j < p.T; ++jt, j = next_tile(j)) {
+      for (int jt = 0, j = j_first; j < p.Tk; ++jt, j = next_tile(j)) {
         const int s = jt & 1;
         // K_j is free once S_j has been computed, V_j once P_j V_j has.
         if (jt >= 2 &&
@@ -262,12 +266,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(&bars[F_KEMPTY + (jt & 1)]);
       };
       bool ok = true;
-      if (j_first < p.T && (ok = wait(F_Q, 0) && wait(F_KFULL, 0))) {
+      if (j_first < p.Tk && (ok = wait(F_Q, 0) && wait(F_KFULL, 0))) {
         tc_fence_after();
         issue_s(0);
-        if (next_tile(j_first) < p.T && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
+        if (next_tile(j_first) < p.Tk && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
       }
-      for (int jt = 0, j = j_first; ok && j < p.T; ++jt, j = next_tile(j)) {
+      for (int jt = 0, j = j_first; ok && j < p.Tk; ++jt, j = next_tile(j)) {
         if (!(ok = wait(F_PFULL, jt & 1))) break;
         if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
         tc_fence_after();
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  (jt > 0 || kk > 0));
         mma_commit(&bars[F_PVDONE + (jt & 1)]);
         mma_commit(&bars[F_VEMPTY + (jt & 1)]);
-        if (next_tile(next_tile(j)) < p.T) {
+        if (next_tile(next_tile(j)) < p.Tk) {
           // S_{j+2} overwrites P_{j-1}, which P_{j-1} V_{j-1} reads
           if (jt >= 1 && !(ok = wait(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
           if (!(ok = wait(F_KFULL + (jt & 1), ((jt + 2) >> 1) & 1))) break;
@@ -305,12 +309,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float m = -INFINITY, z = 0.f;
     bool ok = true;
     int jt = 0;
-    for (int j = j_first; j < p.T; ++jt, j = next_tile(j)) {
+    for (int j = j_first; j < p.Tk; ++jt, j = next_tile(j)) {
       const int kb = j * kTile + 64 * g;  // first key of this thread's 64 columns
-      // keys with local index >= lim are excluded for this row: keys past N,
-      // and in a kind-2 tile keys after the query inside the tile
-      int lim = p.N - kb;
-      if (tile_kind(j) == 2 && t - 64 * g + 1 < lim) lim = t - 64 * g + 1;
+      // keys with local index >= lim are excluded for this row: keys past
+      // N_k, keys after the query's position (causal), and in a kind-2 tile
+      // of a block mask keys after the query inside the tile
+      int lim = p.Nk - kb;
+      if constexpr (kMask) {
+        if (tile_kind(j) == 2 && t - 64 * g + 1 < lim) lim = t - 64 * g + 1;
+      } else {
+        if (p.causal && p.q_off + qrow - kb + 1 < lim) lim = p.q_off + qrow - kb + 1;
+      }
       const bool masked = __any_sync(0xffffffffu, lim < 64);
       if (!(ok = wait_w(F_SFULL + jt % 3, (jt / 3) & 1))) break;
       tc_fence_after();
@@ -433,9 +442,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int BH, int N,
-                         bool causal, float scale, const uint8_t* bmask, const RowStrides& os,
-                         cudaStream_t s) {
+cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int BH,
+                         const Extent& ex, bool causal, float scale, const uint8_t* bmask,
+                         const RowStrides& os, cudaStream_t s) {
   using L = FwdLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   auto kern = bmask ? attn_fwd_bf16_sm100_kernel<D, true> : attn_fwd_bf16_sm100_kernel<D, false>;
@@ -445,16 +454,19 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.status = status;
-  p.N = N;
-  p.T = (N + kTile - 1) / kTile;
+  p.N = ex.nq;
+  p.T = (ex.nq + kTile - 1) / kTile;
   p.BH = BH;
+  p.Nk = ex.nk;
+  p.Tk = (ex.nk + kTile - 1) / kTile;
+  p.q_off = ex.q_off;
   // Heads per group: as many as fit, with their K and V tiles, in about a
   // third of L2.
   int dev = 0, l2 = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
     l2 = 126 << 20;
-  const size_t head_bytes = static_cast<size_t>(p.T) * kTile * D * 4;
+  const size_t head_bytes = static_cast<size_t>(p.Tk) * kTile * D * 4;
   p.G = static_cast<int>(std::max<size_t>(1, std::min<size_t>(BH, (l2 / 3) / head_bytes)));
   p.causal = causal ? 1 : 0;
   p.bmask = bmask;
@@ -468,14 +480,14 @@ cudaError_t launch_fwd_d(const TmaMaps& m, void* o, float* lse, int* status, int
 
 }  // namespace
 
-cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH, int N,
-                            int d, bool causal, float scale, const uint8_t* block_mask,
-                            const RowStrides& os, cudaStream_t s) {
+cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* status, int BH,
+                            const Extent& ex, int d, bool causal, float scale,
+                            const uint8_t* block_mask, const RowStrides& os, cudaStream_t s) {
   switch (d) {
-    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
-    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
+    case 32: return launch_fwd_d<32>(maps, o, lse, status, BH, ex, causal, scale, block_mask, os, s);
+    case 64: return launch_fwd_d<64>(maps, o, lse, status, BH, ex, causal, scale, block_mask, os, s);
     case 128:
-      return launch_fwd_d<128>(maps, o, lse, status, BH, N, causal, scale, block_mask, os, s);
+      return launch_fwd_d<128>(maps, o, lse, status, BH, ex, causal, scale, block_mask, os, s);
     default: return cudaErrorInvalidValue;
   }
 }

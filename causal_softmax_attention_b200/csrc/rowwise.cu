@@ -2,9 +2,11 @@
 //
 // preprocess: D_i = sum_c dO_ic O_ic for every row (the "sums weighted by the
 //   softmax" of ddx issue #243 item 2, which equal sum_j P_ij dP_ij), a copy
-//   of LSE padded to whole 128-row tiles (scaled by log2(e) for the bf16 path,
-//   +inf past N so padded query rows get P = 0), the zeroed fp32 dQ
-//   accumulator (bf16 path) and the zeroed status word.
+//   of LSE padded to whole 128-row tiles (for the bf16 path as -LSE*log2(e),
+//   the term the tensor-core backward adds to its scaled scores, -inf past N;
+//   for the f32 path LSE itself, +inf past N: either way padded query rows get
+//   P = 0), the zeroed fp32 dQ accumulator (bf16 path) and the zeroed status
+//   word.
 // dq_convert: dQ = scale * accumulator, rounded to bf16.
 //
 // Both are bound by HBM bandwidth: 16-byte vector loads/stores, one thread
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(256)
       d_pad[r] = acc;
       // a row with no kept key (LSE = -inf) must give P = 0, like a padded row
       const float l = i < N ? lse[static_cast<size_t>(bh) * N + i] : INFINITY;
-      lse_pad[r] = l == -INFINITY ? INFINITY : l * kLog2e;
+      lse_pad[r] = l == -INFINITY ? -INFINITY : -(l * kLog2e);
     }
   }
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -96,33 +98,44 @@ __global__ void __launch_bounds__(256)
 }
 
 // Accumulator layout [BH][T][d/4][128][4]: element (row r of tile t, column
-// 4*c4 + e). Each thread converts 8 consecutive columns of one row.
+// 4*c4 + e). One CTA per half tile (64 rows): the rows' accumulator columns
+// are read as 16-byte vectors in storage order (each column group of the 64
+// rows is 1 KB of contiguous memory), transposed through shared memory, and
+// written as bf16 rows, consecutive threads covering consecutive 8-byte
+// pieces of a row. Both sides of HBM traffic are therefore fully coalesced,
+// and every index is 32-bit arithmetic on the CTA's own tile.
+constexpr int kConvRows = 64;
+
+template <int D>
 __global__ void __launch_bounds__(256)
-    dq_convert_kernel(const float4* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int BH,
-                      int N, int T, int d, float scale, RowStrides qs) {
-  const int g8 = d / 8;
-  const size_t total = static_cast<size_t>(BH) * T * g8 * kTile;
-  const size_t nthreads = static_cast<size_t>(gridDim.x) * blockDim.x;
-  for (size_t id = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; id < total;
-       id += nthreads) {
-    const int r = static_cast<int>(id % kTile);
-    size_t rest = id / kTile;
-    const int g = static_cast<int>(rest % g8);
-    rest /= g8;
-    const int tile = static_cast<int>(rest % T);
-    const int bh = static_cast<int>(rest / T);
-    const int i = tile * kTile + r;
-    if (i >= N) continue;
-    const size_t a0 = ((static_cast<size_t>(bh) * T + tile) * (d / 4) + 2 * g) * kTile + r;
-    const float4 x = acc[a0];
-    const float4 y = acc[a0 + kTile];
-    __nv_bfloat162 h[4];
+    dq_convert_kernel(const float4* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int N, int T,
+                      float scale, RowStrides qs) {
+  constexpr int C4 = D / 4;       // 16-byte column groups per row
+  constexpr int LD = C4 + 1;      // padded row length in shared memory (float4)
+  __shared__ float4 tile[kConvRows * LD];
+  const int half = blockIdx.x & 1;
+  const int t = (blockIdx.x >> 1) % T;
+  const int bh = (blockIdx.x >> 1) / T;
+  const int r0 = half * kConvRows;
+  const float4* src = acc + (static_cast<size_t>(bh) * T + t) * (C4 * kTile);
+#pragma unroll
+  for (int f = threadIdx.x; f < C4 * kConvRows; f += 256) {
+    const int c4 = f / kConvRows, r = f % kConvRows;
+    tile[r * LD + c4] = src[c4 * kTile + r0 + r];
+  }
+  __syncthreads();
+  const int row0 = t * kTile + r0;
+  __nv_bfloat16* base = dq + qs.head(bh);
+#pragma unroll
+  for (int f = threadIdx.x; f < C4 * kConvRows; f += 256) {
+    const int r = f / C4, c4 = f % C4;
+    if (row0 + r >= N) continue;
+    const float4 x = tile[r * LD + c4];
+    __nv_bfloat162 h[2];
     h[0] = __floats2bfloat162_rn(x.x * scale, x.y * scale);
     h[1] = __floats2bfloat162_rn(x.z * scale, x.w * scale);
-    h[2] = __floats2bfloat162_rn(y.x * scale, y.y * scale);
-    h[3] = __floats2bfloat162_rn(y.z * scale, y.w * scale);
-    *reinterpret_cast<uint4*>(dq + qs.row(bh, i) + 8 * g) =
-        *reinterpret_cast<const uint4*>(h);
+    *reinterpret_cast<uint2*>(base + static_cast<long long>(row0 + r) * qs.sn + 4 * c4) =
+        *reinterpret_cast<const uint2*>(h);
   }
 }
 
@@ -184,10 +197,15 @@ cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse,
 cudaError_t launch_dq_convert(void* dq, int BH, int N, int d, float scale, const RowStrides& qs,
                               const Workspace& ws, cudaStream_t s) {
   const int T = ws.Np / kTile;
-  const size_t total = static_cast<size_t>(BH) * T * (d / 8) * kTile;
-  dq_convert_kernel<<<grid_for(total), 256, 0, s>>>(reinterpret_cast<const float4*>(ws.dq_acc),
-                                                    static_cast<__nv_bfloat16*>(dq), BH, N, T, d,
-                                                    scale, qs);
+  const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(T) * (kTile / kConvRows);
+  const float4* acc = reinterpret_cast<const float4*>(ws.dq_acc);
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dq);
+  switch (d) {
+    case 32: dq_convert_kernel<32><<<grid, 256, 0, s>>>(acc, out, N, T, scale, qs); break;
+    case 64: dq_convert_kernel<64><<<grid, 256, 0, s>>>(acc, out, N, T, scale, qs); break;
+    case 128: dq_convert_kernel<128><<<grid, 256, 0, s>>>(acc, out, N, T, scale, qs); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

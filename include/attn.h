@@ -12,8 +12,9 @@
  * D_i = sum_c dO_ic O_ic instead.
  *
  * Beyond that: block-sparse masks (attn_*_masked), arbitrary row strides
- * (attn_*_strided) and the backward-over-backward (attn_bwd_bwd), each
- * declared below with its own conventions.
+ * (attn_*_strided), N_q != N_k with a query position offset (attn_*_rect)
+ * and the backward-over-backward (attn_bwd_bwd), each declared below with its
+ * own conventions.
  *
  * Layout. Unless an entry point says otherwise, every matrix argument is a
  * DEVICE pointer to a contiguous [B][H][N][d] row-major array (batch, head,
@@ -23,7 +24,8 @@
  * the SCALED scores s_ij = scale * q_i . k_j (the scale is applied before the
  * max, as in ddx issue #217's repro, `SUM(q.val * k.val) / 2.0`). With
  * causal != 0 position i sees keys j <= i (diagonal included, the repro's
- * `WHERE q.pos >= k.pos`); causal == 0 is full attention. N_q == N_k == N.
+ * `WHERE q.pos >= k.pos`); causal == 0 is full attention. N_q == N_k == N
+ * except in attn_*_rect.
  *
  * Ownership. The caller allocates and frees every buffer, the backward's
  * workspace included. The library never allocates or frees device memory,
@@ -160,6 +162,31 @@ int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
                      int H, int N, int d, const long long* qkv_strides,
                      const long long* o_strides, int causal, float scale, int dtype,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * N_q != N_k: N_q query rows attending to N_k keys. Query row r stands for
+ * position q_offset + r and key j for position j; with causal != 0 a score is
+ * kept when the query's position is at least the key's -- the repro's
+ * `WHERE q.pos >= k.pos` of ddx issue #217 ("Backward of batched attention
+ * builds a contraction over every pair of sequences and heads") read on
+ * absolute positions. q_offset = N_k - N_q is the usual key-value-cache
+ * shape (the last N_q positions); q_offset is ignored without the filter.
+ *   q, o, dout, dq : [B][H][N_q][d] of dtype, contiguous
+ *   k, v, dk, dv   : [B][H][N_k][d] of dtype, contiguous
+ *   lse            : [B][H][N_q] float
+ *   workspace      : >= attn_bwd_workspace_bytes(B, H, N_q, d, dtype) bytes
+ * n_q, n_k >= 1 and 0 <= q_offset <= 2^30, else ATTN_ERR_INVALID; every row
+ * then keeps key 0, so no row is empty. Keys after the last query's position
+ * get dK = dV = 0. Everything else (dtypes, head sizes, checks, statuses) as
+ * attn_fwd / attn_bwd, which are the case n_q = n_k, q_offset = 0.
+ */
+int attn_fwd_rect(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int n_q, int n_k, int d, int q_offset, int causal, float scale,
+                  int dtype, void* stream);
+int attn_bwd_rect(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int n_q, int n_k,
+                  int d, int q_offset, int causal, float scale, int dtype, void* workspace,
+                  size_t workspace_bytes, void* stream);
 
 /*
  * Backward-over-backward (the FlashBoB listing, "Approaching I/O-optimality

@@ -72,8 +72,8 @@ def block_mask_keep(block_mask, n: int, tile: int = 128) -> np.ndarray:
     return (kind == 1) | ((kind == 2) & (j % tile <= i % tile))
 
 
-def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None):
-    """Forward of one head. q, k, v: [N, d] float64.
+def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None, q_offset=0):
+    """Forward of one head. q: [N_q, d], k, v: [N_k, d] float64.
 
     Returns a dict with S (scores, including ``row_shift`` if given), keep,
     m (row max over kept scores), w, z, P, O and LSE = m + log z.
@@ -82,7 +82,9 @@ def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None):
     the softmax; it exists only to test the invariance of everything but LSE
     to such a shift. ``keep`` (boolean [N_q, N_k], optional) replaces the
     causal / full filter; a row that keeps no score has P = 0, O = 0 and
-    LSE = -inf (the log of an empty sum).
+    LSE = -inf (the log of an empty sum). With N_q != N_k the causal filter
+    reads query row r as position ``q_offset + r`` and key column j as
+    position j (the repro's ``WHERE q.pos >= k.pos`` on absolute positions).
     """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -91,7 +93,7 @@ def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None):
     S = scale * (q @ k.T)
     if row_shift is not None:
         S = S + np.asarray(row_shift, np.float64)[:, None]
-    keep = keep_mask(n, k.shape[0], causal) if keep is None else np.asarray(keep, bool)
+    keep = keep_mask(n, k.shape[0], causal, q_offset) if keep is None else np.asarray(keep, bool)
     m = np.where(keep, S, -np.inf).max(axis=1)
     w = np.zeros_like(S)
     w[keep] = np.exp((S - m[:, None])[keep])
@@ -104,14 +106,15 @@ def forward_head(q, k, v, scale, causal=True, row_shift=None, keep=None):
     return {"S": S, "keep": keep, "m": m, "w": w, "z": z, "P": P, "O": O, "LSE": LSE}
 
 
-def backward_head(q, k, v, do, scale, causal=True, row_shift=None, keep=None):
-    """Backward of one head without the shift's gradient.
+def backward_head(q, k, v, do, scale, causal=True, row_shift=None, keep=None, q_offset=0):
+    """Backward of one head without the shift's gradient (q, do: [N_q, d];
+    k, v: [N_k, d]; the filter as in forward_head).
 
     Returns dict(dQ, dK, dV, D, D_rows, dS, fwd) where D = sum_c dO o O (the
     form the GPU uses) and D_rows = sum_j P o dP (the softmax-weighted sum of
     ddx issue #243 item 2); the two agree up to rounding.
     """
-    f = forward_head(q, k, v, scale, causal, row_shift, keep)
+    f = forward_head(q, k, v, scale, causal, row_shift, keep, q_offset)
     do = np.asarray(do, np.float64)
     k = np.asarray(k, np.float64)
     q = np.asarray(q, np.float64)
@@ -164,32 +167,38 @@ def backward_head_with_shift(q, k, v, do, scale, causal=True, row_shift=None,
     return {"dQ": dQ, "dK": dK, "dV": dV, "dm": dm, "dS": dS}
 
 
-def forward(q, k, v, scale, causal=True, keep=None):
-    """Batched forward. q, k, v: [B, H, N, d]. Returns O [B,H,N,d], LSE [B,H,N].
-    ``keep`` (boolean [N, N], optional) is shared by every head."""
+def forward(q, k, v, scale, causal=True, keep=None, q_offset=0):
+    """Batched forward. q: [B, H, N_q, d], k, v: [B, H, N_k, d]. Returns
+    O [B,H,N_q,d], LSE [B,H,N_q]. ``keep`` (boolean [N_q, N_k], optional) is
+    shared by every head; ``q_offset`` as in forward_head."""
     q = np.asarray(q, np.float64)
     B, H, N, d = q.shape
     O = np.empty((B, H, N, v.shape[-1]))
     LSE = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
-            f = forward_head(q[b, h], k[b, h], v[b, h], scale, causal, keep=keep)
+            f = forward_head(q[b, h], k[b, h], v[b, h], scale, causal, keep=keep,
+                             q_offset=q_offset)
             O[b, h] = f["O"]
             LSE[b, h] = f["LSE"]
     return O, LSE
 
 
-def backward(q, k, v, do, scale, causal=True, keep=None):
-    """Batched backward. Returns dQ, dK, dV [B,H,N,d], O, LSE and D [B,H,N].
-    ``keep`` (boolean [N, N], optional) is shared by every head."""
+def backward(q, k, v, do, scale, causal=True, keep=None, q_offset=0):
+    """Batched backward. Returns dQ, O [B,H,N_q,d], dK, dV [B,H,N_k,d], LSE
+    and D [B,H,N_q]. ``keep`` (boolean [N_q, N_k], optional) is shared by
+    every head; ``q_offset`` as in forward_head."""
     q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
     B, H, N, d = q.shape
-    out = {name: np.empty(q.shape) for name in ("dQ", "dK", "dV", "O")}
+    out = {name: np.empty(q.shape) for name in ("dQ", "O")}
+    out.update({name: np.empty(k.shape) for name in ("dK", "dV")})
     out["LSE"] = np.empty((B, H, N))
     out["D"] = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
-            r = backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal, keep=keep)
+            r = backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal, keep=keep,
+                              q_offset=q_offset)
             for name in ("dQ", "dK", "dV", "D"):
                 out[name][b, h] = r[name]
             out["O"][b, h] = r["fwd"]["O"]

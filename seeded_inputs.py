@@ -82,6 +82,18 @@ def draw(B: int, H: int, N: int, d: int, seed: int, dtype: str = "f32",
     return tuple(out)
 
 
+def draw_rect(B: int, H: int, n_q: int, n_k: int, d: int, seed: int, dtype: str = "f32"):
+    """q, k, v, dO for N_q query rows and N_k keys: one seeded CPU generator
+    draws q [B, H, N_q, d], k, v [B, H, N_k, d] and dO [B, H, N_q, d] in that
+    order, N(0, 1) float32, rounded like `draw` for bf16."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = []
+    for n in (n_q, n_k, n_k, n_q):
+        t = torch.randn(B, H, n, d, generator=g, dtype=torch.float32)
+        out.append(t.to(torch.bfloat16) if dtype == "bf16" else t)
+    return tuple(out)
+
+
 def draw_config(cfg: AttnConfig):
     return draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)
 

@@ -193,3 +193,21 @@ def test_double_backward_entry_point_rejects_bad_arguments():
     assert f(*([A] * 5 + [A + 4] + [A] * 7), 1, 2, 300, 64, 1, 0.125, 0, A, need,
              None) == csa.ATTN_ERR_INVALID  # lse must be 16-byte aligned
     assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 0, A + 8, need, None) == csa.ATTN_ERR_INVALID
+
+
+def test_rectangular_entry_points_reject_bad_arguments():
+    # every call returns during argument checking (no CUDA call)
+    f, b = L.attn_fwd_rect, L.attn_bwd_rect
+    ws = 1 << 30
+    assert f(A, A, A, A, A, 1, 1, 0, 64, 64, 0, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 0, 64, 0, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 64, 64, -1, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 64, 64, (1 << 30) + 1, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(None, A, A, A, A, 1, 1, 64, 200, 64, 0, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 200, 96, 0, 1, 0.125, 1, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert b(A, A, A, A, A, A, A, A, A, 1, 1, 64, 200, 64, -3, 1, 0.125, 1, A, ws, None) == csa.ATTN_ERR_INVALID
+    assert b(A, A, A, A, A, A, A, A, A, 1, 1, 64, 0, 64, 0, 1, 0.125, 1, A, ws, None) == csa.ATTN_ERR_INVALID
+    # the workspace is sized by the query rows: one sized for fewer rows is refused
+    small = csa.attn_bwd_workspace_bytes(1, 1, 64, 64, csa.ATTN_BF16)
+    assert b(A, A, A, A, A, A, A, A, A, 1, 1, 300, 64, 64, 0, 1, 0.125, 1, A, small, None) == csa.ATTN_ERR_INVALID
+    assert b(A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 0, 1, math.nan, 1, A, ws, None) == csa.ATTN_ERR_INVALID

@@ -535,6 +535,76 @@ def test_outputs_stay_inside_their_buffers(csa, dtype, N, d):
         assert rel(as_f64(view[name].cpu()), ref["d" + name[1:].upper()], gscale) <= TOL[dtype]
 
 
+# ------------------------------------------------------------------ N_q != N_k
+def run_rect(csa, q, k, v, do, off, causal, scale):
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
+    o, lse = csa.forward_rect(qd, kd, vd, off, causal, scale)
+    dq, dk, dv = csa.backward_rect(qd, kd, vd, o, dod, lse, off, causal, scale)
+    torch.cuda.synchronize()
+    assert csa.attn_fwd_last_status() == 0
+    return {"O": o, "LSE": lse, "dQ": dq, "dK": dk, "dV": dv}
+
+
+@pytest.mark.parametrize("dtype,nq,nk,off,causal,d", [
+    ("bf16", 300, 1000, 700, True, 64),    # the KV-cache shape: the last 300 positions
+    ("bf16", 200, 900, 333, True, 128),    # an offset off the tile grid: partial diagonal tiles
+    ("bf16", 1000, 300, 0, True, 128),     # more queries than keys: rows past 300 see every key
+    ("bf16", 257, 641, 50, True, 32),
+    ("bf16", 200, 700, 0, False, 64),      # full attention, rectangular
+    ("bf16", 700, 130, 0, False, 128),
+    ("bf16", 129, 128, 5000, True, 64),    # every query after every key: the causal filter keeps all
+    ("f32", 100, 333, 233, True, 48),
+    ("f32", 333, 100, 0, True, 64),
+    ("f32", 90, 200, 17, False, 7),
+    ("f32", 70, 300, 101, True, 128),
+])
+def test_rectangular_against_the_oracle(csa, dtype, nq, nk, off, causal, d):
+    from seeded_inputs import draw_rect
+    B, H = 2, 3
+    q, k, v, do = draw_rect(B, H, nq, nk, d, 900 + nq + nk, dtype)
+    scale = d ** -0.5
+    g = run_rect(csa, q, k, v, do, off, causal, scale)
+    ref = oracle.backward(as_f64(q), as_f64(k), as_f64(v), as_f64(do), scale, causal, q_offset=off)
+    gscale = max(np.abs(ref[n]).max() for n in ("dQ", "dK", "dV"))
+    for name in ("O", "dQ", "dK", "dV"):
+        e = rel(as_f64(g[name].cpu()), ref[name], None if name == "O" else gscale)
+        assert e <= TOL[dtype], (name, e)
+    assert np.abs(as_f64(g["LSE"].cpu()) - ref["LSE"]).max() <= (1e-5 if dtype == "f32" else 1e-3)
+    if causal and off + nq < nk:
+        # keys after the last query's position get no gradient
+        assert torch.count_nonzero(g["dK"][:, :, off + nq:]) == 0
+        assert torch.count_nonzero(g["dV"][:, :, off + nq:]) == 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rectangular_square_offset_zero_is_the_square_path(csa, d):
+    # N_q == N_k with offset 0 runs the same kernels as attn_fwd / attn_bwd
+    B, H, N = 1, 2, 3 * 128 + 11
+    q, k, v, do = draw(B, H, N, d, 950 + d, "bf16")
+    a = run_rect(csa, q, k, v, do, 0, True, d ** -0.5)
+    b = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    for name in ("O", "LSE", "dK", "dV"):
+        assert torch.equal(a[name], b[name]), name
+    ref = as_f64(b["dQ"].cpu())
+    assert rel(as_f64(a["dQ"].cpu()), ref) <= 1e-2
+
+
+def test_rectangular_rows_of_a_square_problem(csa):
+    # the last 500 query rows of an 1800-token head with offset 1300: O, LSE
+    # and dQ equal those rows of the square call (same kernels, same tiles
+    # apart from the query tiles' alignment), within the bf16 tolerance
+    B, H, N, nq, d = 1, 2, 1800, 500, 64
+    q, k, v, do = draw(B, H, N, d, 960, "bf16")
+    sq = run_gpu(csa, q, k, v, do, True, d ** -0.5)
+    r = run_rect(csa, q[:, :, N - nq:].contiguous(), k, v, do[:, :, N - nq:].contiguous(),
+                 N - nq, True, d ** -0.5)
+    for name in ("O", "dQ"):
+        ref = as_f64(sq[name][:, :, N - nq:].cpu())
+        assert rel(as_f64(r[name].cpu()), ref) <= 2e-2, name
+    assert np.abs(as_f64(r["LSE"].cpu()) - as_f64(sq["LSE"][:, :, N - nq:].cpu())).max() <= 1e-3
+
+
 # ------------------------------------------------------------------ full-size workloads
 def sampled_parity(csa, name, heads, n_rows=24, tail=128, full_heads=()):
     c = CONFIGS[name]

@@ -205,6 +205,90 @@ def test_torch_autograd_cross_check(causal):
 
 
 # --------------------------------------------------------------------------
+# N_q != N_k: query row r at position q_offset + r, key j at position j
+# --------------------------------------------------------------------------
+def torch_reference_positions(q, k, v, do, scale, causal, q_offset):
+    """Separately written: scores masked by explicit positions (row r is
+    position q_offset + r), softmax, weighted values; torch float64 autograd."""
+    q, k, v = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    s = (q @ k.transpose(-1, -2)) * scale
+    if causal:
+        pos_q = q_offset + torch.arange(q.shape[-2])
+        pos_k = torch.arange(k.shape[-2])
+        s = s.masked_fill(pos_q[:, None] < pos_k[None, :], float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    (o * torch.tensor(do)).sum().backward()
+    return o.detach().numpy(), q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("nq,nk,off,causal", [(5, 8, 3, True), (8, 5, 0, True), (6, 9, 0, False),
+                                              (4, 7, 1, True)])
+def test_rectangular_finite_differences(nq, nk, off, causal):
+    rng = np.random.default_rng(nq * 100 + nk)
+    q, do = rng.standard_normal((nq, 4)), rng.standard_normal((nq, 4))
+    k, v = rng.standard_normal((nk, 4)), rng.standard_normal((nk, 4))
+    r = A.backward_head(q, k, v, do, 0.5, causal, q_offset=off)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        return float((do * A.forward_head(q_, k_, v_, 0.5, causal, q_offset=off)["O"]).sum())
+
+    for which, name in ((0, "dQ"), (1, "dK"), (2, "dV")):
+        args = [q, k, v]
+        g = np.zeros_like(args[which])
+        for idx in np.ndindex(g.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            g[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        assert np.abs(g - r[name]).max() <= 1e-7 * max(1.0, np.abs(r[name]).max()), name
+
+
+@pytest.mark.parametrize("nq,nk,off,causal", [(37, 70, 33, True), (70, 37, 0, True),
+                                              (20, 50, 5, True), (33, 21, 0, False)])
+def test_rectangular_torch_autograd_cross_check(nq, nk, off, causal):
+    q, do = rnd(40, 2, 3, nq, 16), rnd(41, 2, 3, nq, 16)
+    k, v = rnd(42, 2, 3, nk, 16), rnd(43, 2, 3, nk, 16)
+    out = A.backward(q, k, v, do, 0.25, causal, q_offset=off)
+    o, gq, gk, gv = torch_reference_positions(q, k, v, do, 0.25, causal, off)
+    assert out["dK"].shape == k.shape and out["dQ"].shape == q.shape
+    assert rel(out["O"], o) <= 1e-12
+    assert rel(out["dQ"], gq) <= 1e-12
+    assert rel(out["dK"], gk) <= 1e-12
+    assert rel(out["dV"], gv) <= 1e-12
+
+
+def test_rectangular_is_a_row_block_of_the_square_problem():
+    # the last n_q rows of a square causal head, offset n - n_q: the same O,
+    # LSE, dQ rows, and dK, dV equal to those rows' contributions
+    # (backward_row_block, pinned above against the materialised head)
+    n, nq, d = 90, 23, 8
+    q, k, v, do = tiny_case(50, n=n, d=d)
+    r = A.backward_head(q[n - nq:], k, v, do[n - nq:], 0.4, True, q_offset=n - nq)
+    blk = A.backward_row_block(q, k, v, do, 0.4, n - nq, n, True)
+    for name in ("dQ", "dK", "dV", "D"):
+        assert rel(r[name], blk[name]) <= 1e-12, name
+    assert rel(r["fwd"]["O"], blk["O"]) <= 1e-12
+    assert np.allclose(r["fwd"]["LSE"], blk["LSE"], rtol=1e-13)
+
+
+def test_rectangular_special_cases():
+    q, k, v, do = tiny_case(60, n=12, d=4)
+    # square with offset 0 is the square causal problem
+    a = A.backward_head(q, k, v, do, 0.3, True, q_offset=0)
+    b = A.backward_head(q, k, v, do, 0.3, True)
+    assert all(np.array_equal(a[n], b[n]) for n in ("dQ", "dK", "dV"))
+    # an offset past the last key makes the causal filter keep everything
+    c = A.backward_head(q[:5], k, v, do[:5], 0.3, True, q_offset=11)
+    e = A.backward_head(q[:5], k, v, do[:5], 0.3, False)
+    assert all(np.array_equal(c[n], e[n]) for n in ("dQ", "dK", "dV"))
+    # keys no query can see get zero gradients
+    f = A.backward_head(q[:3], k, v, do[:3], 0.3, True, q_offset=4)
+    assert np.count_nonzero(f["dK"][7:]) == 0 and np.count_nonzero(f["dV"][7:]) == 0
+
+
+# --------------------------------------------------------------------------
 # ddx issue #217's repro: its printed table sizes and its float64 JAX check
 # --------------------------------------------------------------------------
 def test_ddx_issue217_repro():
