@@ -74,6 +74,7 @@ from seeded_inputs import CONFIGS, block_mask, block_mask_pairs, draw  # noqa: E
 
 METRIC = "causal attention backward TFLOP/s (bf16, 1×B200) and % of dense tensor peak"
 BOB_METRIC = "causal attention backward-over-backward TFLOP/s (fp32, 1xB200)"
+BOB_METRIC_BF16 = "causal attention backward-over-backward TFLOP/s (bf16, 1xB200)"
 LAYER_METRIC = "causal multi-head attention layer step TFLOP/s (bf16, forward + backward)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 MAIN_KERNEL_SOURCE = os.path.join(ROOT, "causal_softmax_attention_b200", "csrc",
@@ -392,8 +393,8 @@ def oracle_sample_bob(cfg, budget_s):
     """The double-backward oracle on the whole workload (as the --bob arm)."""
     import oracle
     from seeded_inputs import as_f64
-    a = [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed, "f32", cfg.qk_gain)]
-    a += [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed + 500, "f32")[:3]]
+    a = [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)]
+    a += [as_f64(t) for t in draw(cfg.B, cfg.H, cfg.N, cfg.d, cfg.seed + 500, cfg.dtype)[:3]]
     return oracle_sample_repeat(
         f"oracle double_backward (numpy float64) on {cfg.name}",
         lambda: oracle.double_backward(*a, cfg.scale, True), 12.0 * cfg.B * cfg.H * cfg.N ** 2 * cfg.d,
@@ -415,8 +416,24 @@ def oracle_sample_layer(cfg, budget_s, n_sample=256):
 
 def bob_config(cfg, n_gpus):
     return dict(config_dict(cfg, n_gpus), workload=f"{cfg.name}: causal attention "
-                f"backward-over-backward B={cfg.B} H={cfg.H} N={cfg.N} d={cfg.d} f32, "
-                "q,k,v,dO,U ~ N(0,1)")
+                f"backward-over-backward B={cfg.B} H={cfg.H} N={cfg.N} d={cfg.d} {cfg.dtype}, "
+                "q,k,v,dO,U ~ N(0,1)" + (f" (q,k x{cfg.qk_gain})" if cfg.qk_gain != 1.0 else ""))
+
+
+def oracle_sample_bob_prefix(cfg, budget_s, n_sample=1024):
+    """The double-backward oracle (materialised, numpy float64) on the first
+    n_sample positions of one head -- a causal prefix is itself a causal
+    problem -- until `budget_s` seconds of CPU work; FLOPs 12 * n^2 * d."""
+    import oracle
+    from seeded_inputs import as_f64
+    n = min(cfg.N, n_sample)
+    a = [as_f64(t[0, 0, :n]) for t in draw(1, 1, cfg.N, cfg.d, cfg.seed, cfg.dtype, cfg.qk_gain)]
+    a += [as_f64(t[0, 0, :n]) for t in draw(1, 1, cfg.N, cfg.d, cfg.seed + 500, cfg.dtype)[:3]]
+    v, desc, el = oracle_sample_repeat(
+        f"oracle double_backward_head (numpy float64, materialised) on the first {n} positions "
+        f"of one head of {cfg.name}", lambda: oracle.double_backward_head(*a, cfg.scale, True),
+        12.0 * n * n * cfg.d, budget_s)
+    return v, desc, el
 
 
 def layer_config(cfg):
@@ -430,7 +447,7 @@ def layer_config(cfg):
 def mode_metric_config(args, cfg, n_gpus):
     """The metric and config of the measurement the flags select."""
     if args.bob:
-        return BOB_METRIC, bob_config(cfg, n_gpus)
+        return (BOB_METRIC_BF16 if cfg.dtype == "bf16" else BOB_METRIC), bob_config(cfg, n_gpus)
     if args.layer:
         return LAYER_METRIC, layer_config(cfg)
     return METRIC, config_dict(cfg, n_gpus, args.block_mask, args.layout)
@@ -442,7 +459,7 @@ def run_reference(args, cfg, world, rank):
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     def sample(b):
         if args.bob:
-            return oracle_sample_bob(cfg, b)
+            return oracle_sample_bob(cfg, b) if cfg.N <= 4096 else oracle_sample_bob_prefix(cfg, b)
         if args.layer:
             return oracle_sample_layer(cfg, b)
         if args.block_mask:
@@ -584,14 +601,16 @@ def run_bob(args, cfg, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     B, H, N, d = cfg.B, cfg.H, cfg.N, cfg.d
-    ins = draw(B, H, N, d, cfg.seed + 1000 * rank, "f32", cfg.qk_gain)
-    cots = draw(B, H, N, d, cfg.seed + 1000 * rank + 500, "f32")[:3]
+    bf16 = cfg.dtype == "bf16"
+    ins = draw(B, H, N, d, cfg.seed + 1000 * rank, cfg.dtype, cfg.qk_gain)
+    cots = draw(B, H, N, d, cfg.seed + 1000 * rank + 500, cfg.dtype)[:3]
     host = [t.pin_memory() for t in ins + cots]
     q, k, v, do, uq, uk, uv = (t.to(dev) for t in host)
     o, lse = csa.forward(q, k, v, True, cfg.scale)
     outs = [torch.empty_like(q) for _ in range(4)]
-    ws = torch.empty(csa.library().attn_bwd_bwd_workspace_bytes(B, H, N, d, csa.ATTN_F32),
-                     dtype=torch.uint8, device=dev)
+    ws = torch.empty(csa.library().attn_bwd_bwd_workspace_bytes(
+        B, H, N, d, csa.ATTN_BF16 if bf16 else csa.ATTN_F32), dtype=torch.uint8, device=dev)
+    torch.cuda.reset_peak_memory_stats(dev)
     stream = torch.cuda.current_stream(dev)
     flops = 12.0 * B * H * N * N * d
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -645,20 +664,31 @@ def run_bob(args, cfg, world, rank, local):
         return
     if csa.attn_last_status(ws) != 0:
         raise RuntimeError("device status after the double-backward steps")
-    peaks, _ = load_peaks()
-    ffma = ffma_peak_tflops(peaks, dev)
+    peaks, peak_kind = load_peaks()
+    if bf16:
+        peak, peak_source = tensor_peak(peaks, peak_kind, ms_per_step * args.steps * 1e-3)
+        roofline = {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                    "frac": value / world / peak, "traffic": None,
+                    "kernel": "bob_rows_bf16_kernel + bob_cols_bf16_kernel (+ preprocess)",
+                    "peak_source": peak_source,
+                    "frac_of_burst": value / world / float(peaks["bf16_tflops"])}
+    else:
+        ffma = ffma_peak_tflops(peaks, dev)
+        roofline = {"bound": "alu", "achieved": value / world, "peak": ffma, "unit": "TFLOP/s",
+                    "frac": value / world / ffma, "traffic": None,
+                    "kernel": "bob_rows_f32_kernel + bob_cols_f32_kernel (+ preprocess)",
+                    "peak_source": f"derived: {sm_count(dev)} SMs x 128 FP32 lanes x 2 FLOP x sm_max_mhz"}
+    roofline.update({"algorithmic_flops_per_launch": flops, "avg_launch_ms": ms_per_step,
+                     "flops_convention": "12 matrix products per kept pair (24*d), causal N^2/2"})
     line = {
-        "metric": BOB_METRIC,
+        "metric": BOB_METRIC_BF16 if bf16 else BOB_METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": bob_config(cfg, world),
-        "roofline": {"bound": "alu", "achieved": value / world, "peak": ffma, "unit": "TFLOP/s",
-                     "frac": value / world / ffma, "traffic": None,
-                     "kernel": "bob_rows_f32_kernel + bob_cols_f32_kernel (+ preprocess)",
-                     "peak_source": f"derived: {sm_count(dev)} SMs x 128 FP32 lanes x 2 FLOP x sm_max_mhz",
-                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": ms_per_step,
-                     "flops_convention": "12 matrix products per kept pair (24*d), causal N^2/2"},
+        "roofline": roofline,
+        "peak_memory_bytes": torch.cuda.max_memory_allocated(dev),
+        "memory_per_token_bytes": torch.cuda.max_memory_allocated(dev) / (B * H * N),
         "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
@@ -667,19 +697,12 @@ def run_bob(args, cfg, world, rank, local):
         "clocks": clocks.summary(host_t0, host_t1),
     }
     if world == 1 and not args.no_cpu_baseline:
-        import oracle
-        from seeded_inputs import as_f64
-        a = [as_f64(t) for t in ins + cots]
-        t0 = time.perf_counter()
-        n_runs = 0
-        while time.perf_counter() - t0 < args.cpu_seconds:
-            oracle.double_backward(*a, cfg.scale, True)
-            n_runs += 1
-        el = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": flops * n_runs / el / 1e12, "unit": "TFLOP/s",
-                                "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"oracle double_backward (numpy float64) on the whole "
-                                          f"workload, {n_runs} runs in {el:.1f} s"}
+        if N <= 4096:
+            v_cpu, desc, _ = oracle_sample_bob(cfg, args.cpu_seconds)
+        else:
+            v_cpu, desc, _ = oracle_sample_bob_prefix(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
     print(json.dumps(line), flush=True)
 
 

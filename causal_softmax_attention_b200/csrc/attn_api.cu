@@ -417,8 +417,9 @@ size_t bob_extra_off(int B, int H, int N, int d) {
 }
 }  // namespace
 
+// (the same for both dtypes: the bf16 path has no dQ accumulator)
 size_t attn_bwd_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
-  if (check_shape(B, H, N, d, dtype) != ATTN_OK || dtype != ATTN_F32) return 0;
+  if (check_shape(B, H, N, d, dtype) != ATTN_OK) return 0;
   const size_t rows = static_cast<size_t>(B) * H * round_up(N, kTile);
   return bob_extra_off(B, H, N, d) + 2 * ((rows * sizeof(float) + 255) / 256 * 256);
 }
@@ -427,24 +428,39 @@ int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, const void* uq, const void* uk, const void* uv, void* gq,
                  void* gk, void* gv, void* gdout, int B, int H, int N, int d, int causal,
                  float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!tensors_aligned(ATTN_F32, {q, k, v, o, dout, uq, uk, uv, gq, gk, gv, gdout}) ||
+  if (!tensors_aligned(dtype, {q, k, v, o, dout, uq, uk, uv, gq, gk, gv, gdout}) ||
       !all_aligned({lse}))
     return ATTN_ERR_INVALID;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
   int st = check_shape(B, H, N, d, dtype);
   if (st != ATTN_OK) return st;
-  if (dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned16(workspace) ||
       workspace_bytes < attn_bwd_bwd_workspace_bytes(B, H, N, d, dtype))
     return ATTN_ERR_INVALID;
+  const size_t rows = static_cast<size_t>(B) * H * round_up(N, kTile);
+  float* r_pad = reinterpret_cast<float*>(static_cast<char*>(workspace) + bob_extra_off(B, H, N, d));
+  float* g_pad =
+      reinterpret_cast<float*>(reinterpret_cast<char*>(r_pad) + (rows * sizeof(float) + 255) / 256 * 256);
+  if (dtype == ATTN_BF16) {
+    if ((st = check_device_sm100()) != ATTN_OK) return st;
+    // the bf16 preprocess (D, -LSE log2 e) into the f32 layout: no dQ accumulator
+    Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, ATTN_F32));
+    ws.dq_acc = nullptr;
+    const RowStrides rs = dense(H, N, d);
+    CUtensorMap maps[7];
+    const void* src[7] = {q, k, v, dout, uq, uk, uv};
+    for (int i = 0; i < 7; ++i)
+      if (!make_map(&maps[i], src[i], B, N, d, rs)) return ATTN_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, true, rs, ws, s));
+    if (st != ATTN_OK) return st;
+    return from_cuda(launch_bob_bf16(maps, ws, r_pad, g_pad, gq, gk, gv, gdout, B * H, H, N, d,
+                                     causal != 0, scale, s));
+  }
   st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes,
                        dense(H, N, d), stream);
   if (st != ATTN_OK) return st;
   const Workspace ws = carve_workspace(workspace, workspace_layout(B, H, N, d, dtype));
-  const size_t rows = static_cast<size_t>(B) * H * ws.Np;
-  float* r_pad = reinterpret_cast<float*>(static_cast<char*>(workspace) + bob_extra_off(B, H, N, d));
-  float* g_pad =
-      reinterpret_cast<float*>(reinterpret_cast<char*>(r_pad) + (rows * sizeof(float) + 255) / 256 * 256);
   return from_cuda(launch_bob_f32(
       static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
       static_cast<const float*>(dout), static_cast<const float*>(uq),

@@ -107,6 +107,14 @@ cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, 
                             uint64_t wait_limit_cycles, int inject_fault,
                             const uint8_t* block_mask, const RowStrides& ks, cudaStream_t s);
 
+// Backward-over-backward on the tensor cores (bf16, d in {32, 64, 128}):
+// maps = {q, k, v, dout, uq, uk, uv} as for the tensor-core backward (4-D,
+// contiguous [B][H][N][d]); needs the bf16 preprocess's lse_pad and d_pad in
+// `ws`, and writes the two row scalars to r_pad, g_pad ([BH][Np] each).
+cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const Workspace& ws, float* r_pad,
+                            float* g_pad, void* gq, void* gk, void* gv, void* gdo, int BH, int H,
+                            int N, int d, bool causal, float scale, cudaStream_t s);
+
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 
 }  // namespace csa

@@ -169,7 +169,9 @@ cudaError_t launch_preprocess(const void* o, const void* dout, const float* lse,
         ws.d_pad, ws.status, BH, N, ws.Np, d, os);
     return cudaGetLastError();
   }
-  const size_t acc_vecs = rows * d / 4;
+  // (a workspace without a dQ accumulator -- the backward-over-backward's --
+  // skips the zeroing)
+  const size_t acc_vecs = ws.dq_acc != nullptr ? rows * d / 4 : 0;
   const int G = d / 8;
   const unsigned grid = grid_for(rows * G > acc_vecs ? rows * G : acc_vecs);
   const uint4* po = static_cast<const uint4*>(o);

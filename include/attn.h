@@ -198,9 +198,11 @@ int attn_bwd_rect(const void* q, const void* k, const void* v, const void* o, co
  *   gq, gk, gv, gdout : out, DEVICE [B][H][N][d], same dtype as q.
  * o and lse are the forward's outputs for (q, k, v) (attn_fwd). The scores
  * are recomputed tile by tile in two passes (two row-wise scalars first,
- * then the gradients); nothing N x N is stored. f32 only for now (bf16 ->
- * ATTN_ERR_UNSUPPORTED), 1 <= d <= 128, contiguous [B][H][N][d], pointers
- * 4-byte aligned, lse and workspace 16-byte aligned.
+ * then the gradients); nothing N x N is stored. dtype ATTN_F32 (CUDA-core
+ * FFMA kernels, 1 <= d <= 128, pointers 4-byte aligned) or ATTN_BF16
+ * (tensor-core kernels, bf16 in and out with fp32 accumulation, d in
+ * {32, 64, 128}, pointers 16-byte aligned); contiguous [B][H][N][d]; lse
+ * and workspace 16-byte aligned.
  *   workspace : DEVICE scratch of >= attn_bwd_bwd_workspace_bytes bytes
  *               (0 for an unsupported shape or dtype).
  * Three stream-ordered kernels: the backward's preprocess (D, padded LSE),

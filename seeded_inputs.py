@@ -66,6 +66,9 @@ CONFIGS = {
     "prof_d64": AttnConfig("prof_d64", 1, 8, 32768, 64, "bf16", 6, qk_gain=0.5),
     # backward-over-backward at a length where its fp32 kernels fill the GPU
     "bob_4k": AttnConfig("bob_4k", 1, 8, 4096, 64, "f32", 7),
+    # the bf16 tensor-core backward-over-backward at 16,384 tokens, d = 64 and 128
+    "bob_16k": AttnConfig("bob_16k", 1, 8, 16384, 64, "bf16", 8),
+    "bob_16k_d128": AttnConfig("bob_16k_d128", 1, 4, 16384, 128, "bf16", 9),
 }
 
 

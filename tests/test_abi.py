@@ -181,11 +181,16 @@ def test_row_strides_of_views():
 def test_double_backward_entry_point_rejects_bad_arguments():
     # every call returns during argument checking (no CUDA call)
     f = L.attn_bwd_bwd
-    assert L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 64, 1) == 0  # bf16: not built
     need = L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 64, 0)
     assert need >= 2 * 2 * 384 * 4
+    # bf16 (tensor-core kernels) takes the same workspace: no dQ accumulator
+    assert L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 64, 1) == need
+    assert L.attn_bwd_bwd_workspace_bytes(1, 2, 300, 48, 1) == 0  # bf16 d outside {32, 64, 128}
     ptrs = [A] * 13
-    assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(*ptrs, 1, 2, 300, 48, 1, 0.125, 1, A, 1 << 30, None) == csa.ATTN_ERR_UNSUPPORTED
+    assert f(*([A] * 9 + [A + 4] + [A] * 3), 1, 2, 300, 64, 1, 0.125, 1, A, 1 << 30,
+             None) == csa.ATTN_ERR_INVALID  # bf16 tensors must be 16-byte aligned
+    assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 1, A, need - 1, None) == csa.ATTN_ERR_INVALID
     assert f(*ptrs, 1, 2, 300, 64, 1, 0.125, 0, A, need - 1, None) == csa.ATTN_ERR_INVALID
     assert f(*ptrs, 1, 2, 300, 64, 1, math.inf, 0, A, need, None) == csa.ATTN_ERR_INVALID
     assert f(*ptrs, 1, 2, 300, 200, 1, 0.125, 0, A, need, None) == csa.ATTN_ERR_UNSUPPORTED

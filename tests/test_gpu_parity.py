@@ -389,6 +389,31 @@ def test_double_backward_against_the_oracle(csa, B, H, N, d, causal):
         assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["f32"], name
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 2, 2100, 64, True), (1, 1, 2048 + 77, 128, True),
+                                             (2, 1, 300, 32, True), (1, 2, 700, 64, False),
+                                             (2, 2, 129, 128, False), (1, 1, 1, 64, True)])
+def test_double_backward_bf16_against_the_oracle(csa, B, H, N, d, causal):
+    # the tensor-core kernels: 2,100 and 2,125 tokens walk 17 tiles (key tile
+    # 0 meets every query tile); N = 1 has the closed form gQ = gK = gV = 0,
+    # gdO = U_V. The oracle takes the bf16-rounded inputs widened to float64.
+    q, k, v, do = draw(B, H, N, d, 800 + N, "bf16")
+    uq, uk, uv, _ = draw(B, H, N, d, 850 + N, "bf16")
+    scale = d ** -0.5
+    ref = oracle.double_backward(*(as_f64(t) for t in (q, k, v, do, uq, uk, uv)), scale, causal)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod, uqd, ukd, uvd = (t.to(dev) for t in (q, k, v, do, uq, uk, uv))
+    o, lse = csa.forward(qd, kd, vd, causal, scale)
+    outs = [torch.full_like(qd, float("nan")) for _ in range(4)]
+    ws = torch.empty(csa.library().attn_bwd_bwd_workspace_bytes(B, H, N, d, csa.ATTN_BF16),
+                     dtype=torch.uint8, device=dev)
+    csa.attn_bwd_bwd(qd, kd, vd, o, dod, lse, uqd, ukd, uvd, *outs, ws, causal, scale)
+    torch.cuda.synchronize()
+    assert csa.attn_last_status(ws) == csa.ATTN_OK
+    gscale = max(np.abs(ref[n]).max() for n in ("gQ", "gK", "gV", "gdO"))
+    for name, t in zip(("gQ", "gK", "gV", "gdO"), outs):
+        assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["bf16"], name
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
