@@ -15,7 +15,7 @@ import os
 
 import torch
 
-from .build import LIB_PATH
+from .build import DEBUG_LIB_PATH, LIB_PATH
 
 ATTN_OK = 0
 ATTN_ERR_INVALID = -1
@@ -34,12 +34,19 @@ class AttnError(RuntimeError):
         self.status = status
 
 
+# CSA_ATTN_DEBUG=1 loads the ATTN_DEBUG build (device-side bounds checks
+# reporting ATTN_ERR_BOUNDS, outputs filled with NaN before each call).
+DEBUG = os.environ.get("CSA_ATTN_DEBUG") == "1"
+ATTN_ERR_BOUNDS = -5
+
+
 def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+    path = DEBUG_LIB_PATH if DEBUG else LIB_PATH
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python causal_softmax_attention_b200/build.py` "
-            "(there is no CPU fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+            f"{path} is missing: build it with `python causal_softmax_attention_b200/build.py"
+            f"{' --debug' if DEBUG else ''}` (there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "attn_fwd": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]),

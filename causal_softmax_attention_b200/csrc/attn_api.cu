@@ -150,6 +150,24 @@ int check_strides(const long long* st, int H, int d, int dtype, RowStrides* out)
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
 
+// Debug builds fill an output with NaN (all-ones bytes: NaN in bf16 and in
+// fp32) before the kernels run, stream-ordered, so that an element no kernel
+// writes shows up; release builds do nothing. Only contiguous outputs are
+// filled (a strided view's rows need not tile its span).
+bool is_dense(const RowStrides& rs, int n, int d) {
+  return rs.sn == d && rs.sh == static_cast<long long>(n) * d && rs.sb == rs.sh * rs.H;
+}
+
+int poison(void* p, size_t elems, size_t elem_bytes, cudaStream_t s) {
+#ifdef ATTN_DEBUG
+  if (p != nullptr && elems > 0)
+    return from_cuda(cudaMemsetAsync(p, 0xFF, elems * elem_bytes, s));
+#else
+  (void)p, (void)elems, (void)elem_bytes, (void)s;
+#endif
+  return ATTN_OK;
+}
+
 struct FaultInjection {
   int armed = 0;
   unsigned long long limit_cycles = 0;
@@ -174,6 +192,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported dtype / head dimension";
     case ATTN_ERR_CUDA: return "CUDA error (launch failed or device is not sm_100)";
     case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_BOUNDS: return "device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -196,6 +215,11 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (st != ATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
+  if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
+  if (is_dense(os, ex.nq, d) &&
+      (poison(o, static_cast<size_t>(BH) * ex.nq * d, dtype == ATTN_BF16 ? 2 : 4, s) != ATTN_OK ||
+       poison(lse, static_cast<size_t>(BH) * ex.nq, 4, s) != ATTN_OK))
+    return ATTN_ERR_CUDA;
   if (dtype == ATTN_F32)
     return from_cuda(launch_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                     static_cast<const float*>(v), static_cast<float*>(o), lse, BH,
@@ -289,6 +313,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (bmask != nullptr && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if ((st = check_ws(B, H, ex.nq, d, dtype, workspace, workspace_bytes)) != ATTN_OK) return st;
   if (dtype == ATTN_BF16 && (st = check_device_sm100()) != ATTN_OK) return st;
+  {
+    const size_t bh = static_cast<size_t>(B) * H, eb = dtype == ATTN_BF16 ? 2 : 4;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((is_dense(qs, ex.nq, d) && poison(dq, bh * ex.nq * d, eb, s) != ATTN_OK) ||
+        (is_dense(ks, ex.nk, d) && (poison(dk, bh * ex.nk * d, eb, s) != ATTN_OK ||
+                                    poison(dv, bh * ex.nk * d, eb, s) != ATTN_OK)))
+      return ATTN_ERR_CUDA;
+  }
   st = preprocess_impl(o, dout, lse, B, H, ex.nq, d, dtype, workspace, workspace_bytes, os,
                        stream);
   if (st != ATTN_OK) return st;
@@ -437,6 +469,11 @@ int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (workspace == nullptr || !aligned16(workspace) ||
       workspace_bytes < attn_bwd_bwd_workspace_bytes(B, H, N, d, dtype))
     return ATTN_ERR_INVALID;
+  {
+    const size_t n = static_cast<size_t>(B) * H * N * d, eb = dtype == ATTN_BF16 ? 2 : 4;
+    for (void* out : {gq, gk, gv, gdout})
+      if (poison(out, n, eb, static_cast<cudaStream_t>(stream)) != ATTN_OK) return ATTN_ERR_CUDA;
+  }
   const size_t rows = static_cast<size_t>(B) * H * round_up(N, kTile);
   float* r_pad = reinterpret_cast<float*>(static_cast<char*>(workspace) + bob_extra_off(B, H, N, d));
   float* g_pad =

@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(kBobThreads, 1)
         if (!(ok = wait_w(O_XCH, 0))) break;
         rr_ = r_sum + xch[(0 * 2 + (g ^ 1)) * 128 + t];
         gg_ = g_sum + xch[(1 * 2 + (g ^ 1)) * 128 + t] - 2.f * rr_ * dv;
-        if (g == 0) {
+        if (g == 0 && CSA_IN_BOUNDS(row < p.Np && bh < p.BH, p.status)) {
           p.r_pad[vrow] = rr_;
           p.g_pad[vrow] = gg_;
         }
@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       fail();
     } else {
       tc_fence_after();
-      const bool row_ok = row < p.N;
+      const bool row_ok = row < p.N && CSA_IN_BOUNDS(bh < p.BH && it_q < p.T, p.status);
       const size_t orow = (static_cast<size_t>(bh) * p.N + (row_ok ? row : 0)) * D;
       store_acc<D>(lane_base, L::T_A0, p.out0 + orow, row_ok, g, p.scale);
       store_acc<D>(lane_base, L::T_A1, p.out1 + orow, row_ok, g, 1.f);
@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       fail();
     } else {
       tc_fence_after();
-      const bool key_ok = key < p.N;
+      const bool key_ok = key < p.N && CSA_IN_BOUNDS(bh < p.BH && jt < p.T, p.status);
       const size_t orow = (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
       // a key tile that meets no query tile (none, causal or not) still
       // accumulated at least one half: n_loads >= 1 always

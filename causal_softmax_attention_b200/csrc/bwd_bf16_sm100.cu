@@ -377,7 +377,9 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
             !(ok = mbar_wait(&bars[B_QEMPTY + s], ((it - L::STAGES) / L::STAGES) & 1, p.wait_cycles,
                              abort_flag)))
           break;
-        const int i0 = i * kTile;
+        // (a debug build redirects an out-of-range tile to tile 0)
+        const int i0 =
+            (CSA_IN_BOUNDS(i >= 0 && i < p.T && jt < p.Tk && bh < p.BH, p.status) ? i : 0) * kTile;
         uint64_t* bar = &bars[B_QFULL + s];
         mbar_arrive_expect_tx(bar, 2 * L::TILE + 2 * 512);
         for (int c = 0; c < L::NCH; ++c) {
@@ -552,7 +554,8 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       tmem_ld_wait(r);
       tc_fence_before();
       mbar_arrive(&bars[B_DQREAD + b]);
-      if (i * kTile + t < p.N) {  // a query row of this head
+      if (i * kTile + t < p.N &&  // a query row of this head
+          CSA_IN_BOUNDS(i >= 0 && i < p.T && bh < p.BH && t < kTile, p.status)) {
         float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.T + i) * (D / 4) * 512 + t * 4;
         // Metered: a burst of reductions fills the sub-partition's memory
         // instruction queue, and the element-wise warps' TMEM and shared-memory
@@ -682,8 +685,9 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
 #pragma unroll
           for (int u = 0; u < W; ++u) rv[u] = rk[u] = 0u;
         }
+        const bool store_ok = key_ok && CSA_IN_BOUNDS(bh < p.BH && ch + W <= D, p.status);
 #pragma unroll
-        for (int v = 0; v < W / 8 && key_ok; ++v) {
+        for (int v = 0; v < W / 8 && store_ok; ++v) {
           uint4 ov, ok4;
           ov.x = pack_bf16x2(__uint_as_float(rv[8 * v + 0]), __uint_as_float(rv[8 * v + 1]));
           ov.y = pack_bf16x2(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3]));

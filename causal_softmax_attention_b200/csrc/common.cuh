@@ -12,6 +12,18 @@ constexpr int kTile = 128;  // rows of a query or key tile on the tensor-core pa
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = -4;
+constexpr int kStatusBounds = -5;  // a device-side bounds check of a debug build failed
+
+// Debug builds (compiled with ATTN_DEBUG) check tile coordinates and row
+// indices before the global accesses a thread makes; a failed check writes
+// kStatusBounds into the call's status word and the access is skipped or
+// redirected to a valid tile -- never a trap. Release builds compile the
+// checks away (the condition is not even evaluated).
+#ifdef ATTN_DEBUG
+#define CSA_IN_BOUNDS(cond, status) ((cond) ? true : (atomicExch((status), kStatusBounds), false))
+#else
+#define CSA_IN_BOUNDS(cond, status) true
+#endif
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 

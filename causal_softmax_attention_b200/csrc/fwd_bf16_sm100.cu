@@ -233,9 +233,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             !(ok = mbar_wait(&bars[empty + s], ((jt - 2) >> 1) & 1, p.wait_cycles, abort_flag)))
           break;
         mbar_arrive_expect_tx(&bars[full + s], L::TILE);
+        // (a debug build redirects an out-of-range tile to tile 0)
+        const int j_ld = CSA_IN_BOUNDS(j >= 0 && j < p.Tk && bh < p.BH, p.status) ? j : 0;
         for (int c = 0; c < L::NCH; ++c)
           tma_load_4d(smem + off + s * L::TILE + c * L::CHUNK, map, &bars[full + s], c * L::CH,
-                      j * kTile, hh, hb);
+                      j_ld * kTile, hh, hb);
         ++issued;
       }
       if (!ok) fail();
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     } else {
       tc_fence_after();
       const float inv = z > 0.f ? 1.f / z : 0.f;
-      const bool row_ok = qrow < p.N;
+      const bool row_ok = qrow < p.N && CSA_IN_BOUNDS(bh < p.BH && it_q < p.T, p.status);
       __nv_bfloat16* orow =
           p.o + p.os.row(bh, row_ok ? qrow : 0) + g * L::HALF_D;
 #pragma unroll 1

@@ -45,6 +45,14 @@
  * into a status word (the workspace's for the backward, a library-owned one
  * for the forward) and the kernel returns without trapping. Input VALUES are
  * not validated: NaN and infinities propagate as IEEE arithmetic carries them.
+ *
+ * Debug build. The same sources compiled with ATTN_DEBUG (build.py --debug:
+ * libcsa_attn_debug.so, same symbols) check tile coordinates and row indices
+ * in the kernels before the global accesses a thread makes -- a failed check
+ * writes ATTN_ERR_BOUNDS into the status word and skips the access, never a
+ * trap -- and fill the outputs of attn_fwd / attn_bwd / attn_fwd_rect /
+ * attn_bwd_rect / attn_bwd_bwd with NaN (on the call's stream) before their
+ * kernels run, so that an element no kernel writes shows up.
  */
 #ifndef CSA_ATTN_H_
 #define CSA_ATTN_H_
@@ -60,7 +68,8 @@ typedef enum {
   ATTN_ERR_INVALID = -1,
   ATTN_ERR_UNSUPPORTED = -2,
   ATTN_ERR_CUDA = -3,
-  ATTN_ERR_TIMEOUT = -4
+  ATTN_ERR_TIMEOUT = -4,
+  ATTN_ERR_BOUNDS = -5 /* debug builds only: a device-side bounds check failed */
 } attn_status;
 
 typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;

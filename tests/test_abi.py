@@ -216,3 +216,20 @@ def test_rectangular_entry_points_reject_bad_arguments():
     small = csa.attn_bwd_workspace_bytes(1, 1, 64, 64, csa.ATTN_BF16)
     assert b(A, A, A, A, A, A, A, A, A, 1, 1, 300, 64, 64, 0, 1, 0.125, 1, A, small, None) == csa.ATTN_ERR_INVALID
     assert b(A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 0, 1, math.nan, 1, A, ws, None) == csa.ATTN_ERR_INVALID
+
+
+def test_debug_build_exports_the_same_boundary():
+    # the ATTN_DEBUG variant (built beside the release library) exports every
+    # declared symbol, names the bounds status, and checks arguments the same
+    # way before any CUDA call
+    from causal_softmax_attention_b200.build import DEBUG_LIB_PATH
+    dbg = ctypes.CDLL(DEBUG_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    dbg.attn_status_string.restype = ctypes.c_char_p
+    assert b"bounds" in dbg.attn_status_string(csa.ATTN_ERR_BOUNDS)
+    assert b"bounds" in L.attn_status_string(csa.ATTN_ERR_BOUNDS)
+    f = dbg.attn_fwd
+    f.argtypes = L.attn_fwd.argtypes
+    assert f(None, A, A, A, A, 1, 1, 64, 64, 1, 0.125, 1, None) == csa.ATTN_ERR_INVALID
+    assert f(A, A, A, A, A, 1, 1, 64, 96, 1, 0.125, 1, None) == csa.ATTN_ERR_UNSUPPORTED
