@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "attn_fwd_last_status": (i, []),
         "attn_status_string": (ctypes.c_char_p, [i]),
         "attn_test_arm_timeout": (i, [ctypes.c_ulonglong]),
+        "attn_test_exp2": (i, [vp, vp, vp, i, vp]),
         "attn_bwd_noalloc": (i, [vp] * 9 + [i, i, i, i, i, f, i, vp]),
         "attn_bwd_noalloc_last_status": (i, []),
         "attn_fwd_masked": (i, [vp] * 5 + [i, i, i, i, vp, f, i, vp]),
@@ -84,7 +85,8 @@ EXPORTED = ("attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_prepro
             "attn_status_string", "attn_test_arm_timeout", "attn_bwd_noalloc",
             "attn_bwd_noalloc_last_status", "attn_fwd_masked",
             "attn_bwd_masked", "attn_bwd_main_masked", "attn_fwd_strided", "attn_bwd_strided",
-            "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd", "attn_fwd_rect", "attn_bwd_rect")
+            "attn_bwd_bwd_workspace_bytes", "attn_bwd_bwd", "attn_fwd_rect", "attn_bwd_rect",
+            "attn_test_exp2")
 
 
 def library() -> ctypes.CDLL:

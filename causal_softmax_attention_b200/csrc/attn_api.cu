@@ -525,6 +525,12 @@ int attn_fwd_last_status(void) {
   return v;
 }
 
+int attn_test_exp2(const float* x, float* poly, float* mufu, int n, void* stream) {
+  if (x == nullptr || poly == nullptr || mufu == nullptr || n < 0) return ATTN_ERR_INVALID;
+  if (n == 0) return ATTN_OK;
+  return from_cuda(launch_exp2_pair(x, poly, mufu, n, static_cast<cudaStream_t>(stream)));
+}
+
 int attn_test_arm_timeout(unsigned long long wait_limit_cycles) {
   if (wait_limit_cycles == 0) return ATTN_ERR_INVALID;
   std::lock_guard<std::mutex> g(g_fault_mu);

@@ -129,4 +129,7 @@ cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const Workspace& ws, f
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 
+// Test hook: 2^x by the forward's FMA-pipe polynomial and by MUFU ex2.approx.
+cudaError_t launch_exp2_pair(const float* x, float* poly, float* mufu, int n, cudaStream_t s);
+
 }  // namespace csa

@@ -367,13 +367,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         z *= alpha;
       }
-      // P = exp2(S * scale*log2e - m) -> bf16 into the first 32 of this group's columns
+      // P = exp2(S * scale*log2e - m) -> bf16 into the first 32 of this group's
+      // columns. The arguments are formed two at a time by a packed FMA; one
+      // pair in four is exponentiated on the FMA pipe (exp2_fma2), the rest
+      // on MUFU, whose 16 results per clock per SM would otherwise take twice
+      // as long as the tile's two MMAs at d = 64.
       uint32_t pk[32];
       float zt = 0.f;
+      const uint64_t c2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-m, -m);
 #pragma unroll
       for (int u = 0; u < 64; u += 2) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[u]), p.scale_log2, -m));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[u + 1]), p.scale_log2, -m));
+        const float2 x =
+            f2_split(fma2(f2(__uint_as_float(sr[u]), __uint_as_float(sr[u + 1])), c2, nm2));
+        float p0, p1;
+        if ((u / 2) % 4 == 3) {
+          const float2 e = exp2_fma2(x.x, x.y);
+          p0 = e.x;
+          p1 = e.y;
+        } else {
+          p0 = ex2_approx(x.x);
+          p1 = ex2_approx(x.y);
+        }
         if (masked) {
           if (u >= lim) p0 = 0.f;
           if (u + 1 >= lim) p1 = 0.f;
@@ -492,6 +506,30 @@ cudaError_t launch_fwd_bf16(const TmaMaps& maps, void* o, float* lse, int* statu
       return launch_fwd_d<128>(maps, o, lse, status, BH, ex, causal, scale, block_mask, os, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+namespace {
+// Test hook: the forward's two exponentials side by side, 2^x by
+// exp2_fma2 (FMA pipe) and by ex2.approx (MUFU), for n inputs.
+__global__ void exp2_pair_kernel(const float* __restrict__ x, float* __restrict__ poly,
+                                 float* __restrict__ mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  const float2 e = sm100::exp2_fma2(a, b);
+  poly[i] = e.x;
+  mufu[i] = sm100::ex2_approx(a);
+  if (i + 1 < n) {
+    poly[i + 1] = e.y;
+    mufu[i + 1] = sm100::ex2_approx(b);
+  }
+}
+}  // namespace
+
+cudaError_t launch_exp2_pair(const float* x, float* poly, float* mufu, int n, cudaStream_t s) {
+  const int pairs = (n + 1) / 2;
+  exp2_pair_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, poly, mufu, n);
+  return cudaGetLastError();
 }
 
 }  // namespace csa

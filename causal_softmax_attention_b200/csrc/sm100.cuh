@@ -405,6 +405,37 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe instead of the MUFU unit, by Cody and
+// Waite's range reduction: x (clamped to >= -125, so that the result stays
+// a normal number) splits into r = round-to-nearest(x), found by adding and
+// subtracting 1.5 * 2^23, and f = x - r in [-1/2, 1/2]; 2^f comes from a
+// degree-3 polynomial and 2^r is added into the exponent field as an
+// integer (the magic sum's low bits hold r). The coefficients were fitted
+// for relative error on [-1/2, 1/2] by Lawson's iteration (weighted least
+// squares on Chebyshev nodes converging to the minimax fit): max relative
+// error 7.5e-5, far below bf16's 2^-9 rounding of the probabilities it
+// feeds. Exact inputs below -125 (the masked -inf included) give 2^-125.
+__device__ __forceinline__ float2 exp2_fma2(float a, float b) {
+  a = fmaxf(a, -125.f);
+  b = fmaxf(b, -125.f);
+  const uint64_t x = f2(a, b);
+  const uint64_t magic = f2(12582912.f, 12582912.f);
+  const uint64_t t = add2(x, magic);
+  const uint64_t fr = sub2(x, sub2(t, magic));
+  uint64_t q = fma2(f2(0.0551716685295105f, 0.0551716685295105f), fr,
+                    f2(0.2426111400127411f, 0.2426111400127411f));
+  q = fma2(q, fr, f2(0.6932609677314758f, 0.6932609677314758f));
+  q = fma2(q, fr, f2(0.9999280571937561f, 0.9999280571937561f));
+  const float2 tv = f2_split(t), qv = f2_split(q);
+  return make_float2(__uint_as_float(__float_as_uint(qv.x) + (__float_as_uint(tv.x) << 23)),
+                     __uint_as_float(__float_as_uint(qv.y) + (__float_as_uint(tv.y) << 23)));
+}
 
 }  // namespace sm100
 }  // namespace csa

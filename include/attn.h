@@ -277,6 +277,17 @@ const char* attn_status_string(int status);
 int attn_test_arm_timeout(unsigned long long wait_limit_cycles);
 
 /*
+ * Test hook for the forward's exponentials (not part of the method; the pages
+ * have no counterpart): for n DEVICE floats x, writes 2^x computed the two
+ * ways the bf16 forward computes it -- on the FMA pipe by Cody-Waite range
+ * reduction and a degree-3 polynomial (`poly`) and by the MUFU ex2.approx
+ * instruction (`mufu`) -- so that tests can bound the polynomial against
+ * the hardware instruction and exact values. Device pointers, enqueued on
+ * `stream`; NULL pointers or n < 0 -> ATTN_ERR_INVALID.
+ */
+int attn_test_exp2(const float* x, float* poly, float* mufu, int n, void* stream);
+
+/*
  * Backward without any allocation, for callers that cannot call cudaMalloc:
  * code running inside a host framework whose device memory is reserved by that
  * framework's own pool (a plugin or custom operator that may not allocate),

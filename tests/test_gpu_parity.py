@@ -414,6 +414,32 @@ def test_double_backward_bf16_against_the_oracle(csa, B, H, N, d, causal):
         assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["bf16"], name
 
 
+def test_forward_exponential_polynomial(csa):
+    # the forward computes one exponential in four on the FMA pipe (Cody-Waite
+    # reduction, degree-3 polynomial): against exact 2^x and against MUFU's
+    # ex2.approx over the arguments the forward produces (<= 8: the running
+    # maximum is raised once a score exceeds it by 8), the masked -inf
+    # included; below -125 the polynomial clamps to 2^-125
+    x = np.concatenate([np.linspace(-130.0, 8.0, 1 << 20), np.linspace(-1.0, 1.0, 4097),
+                        [-np.inf, -125.5, -125.0, -124.99, -0.5, 0.5, -1e-30, 0.0, 8.0]])
+    x = x.astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    poly, mufu = torch.empty_like(xd), torch.empty_like(xd)
+    st = csa.library().attn_test_exp2(xd.data_ptr(), poly.data_ptr(), mufu.data_ptr(), x.size,
+                                      torch.cuda.current_stream().cuda_stream)
+    assert st == csa.ATTN_OK
+    torch.cuda.synchronize()
+    poly, mufu = poly.cpu().numpy().astype(np.float64), mufu.cpu().numpy().astype(np.float64)
+    exact = np.exp2(x.astype(np.float64))
+    inside = x >= -125.0
+    assert np.all(np.isfinite(poly)) and np.all(poly >= 0.0)
+    assert np.abs(poly[inside] / exact[inside] - 1.0).max() <= 1e-4
+    assert np.all(poly[~inside] <= 2.0 ** -124)
+    normal = x >= -126.0
+    assert np.abs(mufu[normal] / exact[normal] - 1.0).max() <= 1e-6
+    assert np.abs(poly[inside] / mufu[inside] - 1.0).max() <= 1.1e-4
+
+
 def test_linearity_and_causality(csa):
     B, H, N, d = 1, 2, 768, 64
     q, k, v, do = draw(B, H, N, d, 7, "bf16")
