@@ -45,6 +45,11 @@ dQ, dK, dV to every rank inside the timed step.
 per kept score pair (24*d per pair, 12*B*H*N^2*d causal), against the
 derived FFMA peak.
 
+`--rect NQ` times the N_q != N_k backward (attn_bwd_rect): the last NQ
+positions of the configuration's N tokens (query row r at position
+N - NQ + r) attending causally to all N keys -- the key-value-cache shape --
+FLOPs counted over the kept pairs (10*d per pair).
+
 `--block-mask SPEC` (causal, full, window:W, random:P:SEED over 128 x 128
 tiles; bf16) times the block-sparse backward instead: the same three stages
 with the masked main kernel, FLOPs counted over the kept tiles (a kind-1 tile
@@ -444,8 +449,29 @@ def layer_config(cfg):
             "l2": "inputs larger than L2 (no flush needed)"}
 
 
+RECT_METRIC = "causal attention backward TFLOP/s, N_q < N_k (bf16, 1xB200)"
+
+
+def rect_pairs(nq: int, nk: int, off: int) -> int:
+    """Score pairs the causal filter keeps when query row r is position off + r."""
+    r = np.arange(nq, dtype=np.int64)
+    return int(np.minimum(nk, off + r + 1).sum())
+
+
+def rect_config(cfg, nq):
+    off = cfg.N - nq
+    return {"workload": f"{cfg.name} keys with the last {nq} positions as queries: causal attention "
+                        f"backward B={cfg.B} H={cfg.H} N_q={nq} N_k={cfg.N} q_offset={off} "
+                        f"d={cfg.d} {cfg.dtype}, q,k,v,dO ~ N(0,1)",
+            "B": cfg.B, "H": cfg.H, "N_q": nq, "N_k": cfg.N, "q_offset": off, "d": cfg.d,
+            "causal": True, "parallelism": "single GPU",
+            "kept_pairs_per_head": rect_pairs(nq, cfg.N, off)}
+
+
 def mode_metric_config(args, cfg, n_gpus):
     """The metric and config of the measurement the flags select."""
+    if args.rect:
+        return RECT_METRIC, rect_config(cfg, args.rect)
     if args.bob:
         return (BOB_METRIC_BF16 if cfg.dtype == "bf16" else BOB_METRIC), bob_config(cfg, n_gpus)
     if args.layer:
@@ -460,6 +486,8 @@ def run_reference(args, cfg, world, rank):
     def sample(b):
         if args.bob:
             return oracle_sample_bob(cfg, b) if cfg.N <= 4096 else oracle_sample_bob_prefix(cfg, b)
+        if args.rect:
+            return oracle_sample(cfg, b)  # the last query rows of a head: the rectangular problem
         if args.layer:
             return oracle_sample_layer(cfg, b)
         if args.block_mask:
@@ -796,6 +824,71 @@ def run_layer(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------- rectangular arm
+def run_rect(args, cfg, world, rank, local):
+    import causal_softmax_attention_b200 as csa
+    from seeded_inputs import draw_rect
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, nk, d, nq = cfg.B, cfg.H, cfg.N, cfg.d, args.rect
+    off = nk - nq
+    q, k, v, do = (t.to(dev) for t in draw_rect(B, H, nq, nk, d, cfg.seed + 1000 * rank,
+                                                 cfg.dtype))
+    o, lse = csa.forward_rect(q, k, v, off, True, cfg.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = csa.new_workspace(q)
+    stream = torch.cuda.current_stream(dev)
+    flops = 10.0 * d * B * H * rect_pairs(nq, nk, off)
+
+    def step():
+        csa.attn_bwd_rect(q, k, v, o, do, lse, dq, dk, dv, ws, off, True, cfg.scale, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        time.sleep(1.0)
+        host_t0 = time.time()
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        host_t1 = time.time()
+        time.sleep(0.25)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms_per_step = max_over_ranks(statistics.median(step_ms), world)
+    value = whole_job_tflops(flops, world, ms_per_step)
+    if rank != 0:
+        return
+    if csa.attn_last_status(ws) != 0:
+        raise RuntimeError("device status after the rectangular steps")
+    peaks, peak_kind = load_peaks()
+    peak, peak_source = tensor_peak(peaks, peak_kind, sum(step_ms) * 1e-3)
+    line = {
+        "metric": RECT_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic", "config": rect_config(cfg, nq),
+        "statistic": "median of the timed steps' CUDA-event times (max over ranks)",
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / world / peak, "traffic": None,
+                     "kernel": "attn_bwd_rect (whole call: preprocess, main kernel, dQ convert)",
+                     "peak_source": peak_source,
+                     "frac_of_burst": value / world / float(peaks["bf16_tflops"]),
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": ms_per_step,
+                     "flops_convention": "10*d per kept pair (5 MMAs)"},
+        "e2e": None,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(host_t0, host_t1),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------------------- GPU arm
 def run_gpu(args, cfg, world, rank, local):
     import causal_softmax_attention_b200 as csa
@@ -1074,6 +1167,8 @@ def main():
                     help="time one attention layer step (projections + attention, fwd + bwd)")
     ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd", "packed"],
                     help="memory layout of q, k, v, o, dO and the gradients")
+    ap.add_argument("--rect", type=int, default=0, metavar="NQ",
+                    help="time attn_bwd_rect: the last NQ positions as queries over all N keys")
     ap.add_argument("--block-mask", default=None, metavar="SPEC",
                     help="time the block-sparse backward: causal, full, window:W or "
                          "random:P:SEED over 128x128 tiles (bf16 configs)")
@@ -1087,6 +1182,9 @@ def main():
     if args.layer and "--config" not in sys.argv:
         args.config = "c4"  # a layer of 16 heads x 128 channels (C = 2048)
     cfg = CONFIGS[args.config]
+    if args.rect and (args.rect < 1 or args.rect > cfg.N or args.block_mask or args.bob
+                      or args.layer or args.shard_heads or args.layout != "bhnd"):
+        ap.error("--rect NQ needs 1 <= NQ <= N and is a measurement of its own")
     if args.layout != "bhnd" and args.block_mask:
         ap.error("--layout and --block-mask are separate measurements")
     if args.block_mask:
@@ -1109,6 +1207,8 @@ def main():
     try:
         if args.layer:
             run_layer(args, cfg, world, rank, local)
+        elif args.rect:
+            run_rect(args, cfg, world, rank, local)
         elif args.shard_heads:
             run_sharded(args, cfg, world, rank, local)
         elif args.bob:

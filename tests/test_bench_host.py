@@ -79,3 +79,11 @@ def test_default_workload_is_the_largest_single_gpu_config():
               key=lambda c: c.bwd_flops)
     assert big.name == "c5"
     assert sys.modules["bench"] is bench
+
+
+def test_rect_pair_count_is_the_oracle_mask():
+    import oracle
+    for nq, nk, off in ((300, 1000, 700), (1000, 300, 0), (129, 128, 5000), (5, 8, 3)):
+        assert bench.rect_pairs(nq, nk, off) == int(oracle.keep_mask(nq, nk, True, off).sum())
+    # the last N positions as queries are the square causal problem
+    assert bench.rect_pairs(640, 640, 0) == 640 * 641 // 2
