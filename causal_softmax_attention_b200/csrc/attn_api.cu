@@ -113,9 +113,11 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map {d, N, H, B} over a bf16 array whose rows `rs` lays out: box =
-// 128 rows x min(d, 64) channels of one (b, h), swizzled to match the UMMA
-// canonical layout. Rows past N read as zero.
-bool make_map(CUtensorMap* m, const void* base, int B, int N, int d, const RowStrides& rs) {
+// `box_rows` rows (a tile, or the backward-over-backward's 64-row halves) x
+// min(d, 64) channels of one (b, h), swizzled to match the UMMA canonical
+// layout. Rows past N read as zero.
+bool make_map(CUtensorMap* m, const void* base, int B, int N, int d, const RowStrides& rs,
+              int box_rows = kTile) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const int ch = d >= 64 ? 64 : d;
@@ -123,7 +125,7 @@ bool make_map(CUtensorMap* m, const void* base, int B, int N, int d, const RowSt
                         static_cast<cuuint64_t>(rs.H), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(rs.sn) * 2, static_cast<cuuint64_t>(rs.sh) * 2,
                            static_cast<cuuint64_t>(rs.sb) * 2};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(ch), static_cast<cuuint32_t>(kTile), 1, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(ch), static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapSwizzle swz =
       ch * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -487,11 +489,11 @@ int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, con
     CUtensorMap maps[7];
     const void* src[7] = {q, k, v, dout, uq, uk, uv};
     for (int i = 0; i < 7; ++i)
-      if (!make_map(&maps[i], src[i], B, N, d, rs)) return ATTN_ERR_CUDA;
+      if (!make_map(&maps[i], src[i], B, N, d, rs, kBobBoxRows)) return ATTN_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     st = from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, true, rs, ws, s));
     if (st != ATTN_OK) return st;
-    return from_cuda(launch_bob_bf16(maps, ws, r_pad, g_pad, gq, gk, gv, gdout, B * H, H, N, d,
+    return from_cuda(launch_bob_bf16(maps, src, ws, r_pad, g_pad, gq, gk, gv, gdout, B * H, H, N, d,
                                      causal != 0, scale, s));
   }
   st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes,

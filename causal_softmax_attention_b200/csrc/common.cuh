@@ -9,6 +9,7 @@
 namespace csa {
 
 constexpr int kTile = 128;  // rows of a query or key tile on the tensor-core path
+constexpr int kBobBoxRows = 64;  // rows of one backward-over-backward TMA box (half a tile)
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = -4;
@@ -123,9 +124,11 @@ cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, 
 // maps = {q, k, v, dout, uq, uk, uv} as for the tensor-core backward (4-D,
 // contiguous [B][H][N][d]); needs the bf16 preprocess's lse_pad and d_pad in
 // `ws`, and writes the two row scalars to r_pad, g_pad ([BH][Np] each).
-cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const Workspace& ws, float* r_pad,
-                            float* g_pad, void* gq, void* gk, void* gv, void* gdo, int BH, int H,
-                            int N, int d, bool causal, float scale, cudaStream_t s);
+// maps and src: q, k, v, dout, uq, uk, uv (contiguous [BH][N][d] bf16)
+cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const void* const (&src)[7],
+                            const Workspace& ws, float* r_pad, float* g_pad, void* gq, void* gk,
+                            void* gv, void* gdo, int BH, int H, int N, int d, bool causal,
+                            float scale, cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 
