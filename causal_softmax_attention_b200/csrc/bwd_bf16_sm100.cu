@@ -168,28 +168,45 @@ struct BwdParams {
   int inject_fault;   // 1: never signal the first score tile (tests the timeout path)
 };
 
-// K-major operand: rows [128][D] stored as D/CH swizzled boxes, advanced to
-// the kk-th 16-element K step.
+// Operand descriptors are built once per operand base and stepped by
+// constants: a descriptor's start-address field holds address >> 4 in its low
+// 14 bits (the shared window lies below 256 KB), so the descriptor of
+// base + off is the base's plus off >> 4 for any 16-byte multiple off that
+// stays in the window -- one add per MMA operand instead of a mask, a shift
+// and an OR on 64-bit values, in the warp that shares its sub-partition with
+// two element-wise warps.
+//
+// K-major operand: rows [128][D] stored as D/CH swizzled boxes; koff steps it
+// to the kk-th 16-element K step.
 template <int D>
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
+__device__ __forceinline__ uint64_t desc_k0(uint32_t tile) {
   using L = BwdLayout<D>;
-  const int e = kk * 16;
-  const uint32_t addr = tile + (e / L::CH) * L::CHUNK + (e % L::CH) * 2;
-  return smem_desc(addr, 16, 8 * L::ROWB, L::SWZ);
+  return smem_desc(tile, 16, 8 * L::ROWB, L::SWZ);
+}
+template <int D>
+__host__ __device__ constexpr uint32_t koff(int kk) {
+  using L = BwdLayout<D>;
+  return static_cast<uint32_t>(((kk * 16) / L::CH) * L::CHUNK + ((kk * 16) % L::CH) * 2) >> 4;
 }
 
 // The same [128 rows][D] tile read as an MN-major operand (rows = K,
-// columns = M or N), advanced to the kk-th 16-row K step.
+// columns = M or N); mnoff steps it to the kk-th 16-row K step.
 template <int D>
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
+__device__ __forceinline__ uint64_t desc_mn0(uint32_t tile) {
   using L = BwdLayout<D>;
-  return smem_desc(tile + kk * 16 * L::ROWB, L::CHUNK, 8 * L::ROWB, L::SWZ);
+  return smem_desc(tile, L::CHUNK, 8 * L::ROWB, L::SWZ);
+}
+template <int D>
+__host__ __device__ constexpr uint32_t mnoff(int kk) {
+  using L = BwdLayout<D>;
+  return static_cast<uint32_t>(kk * 16 * L::ROWB) >> 4;
 }
 
 // The [128 keys][128 queries] dS tile (two 64-query boxes, 128B swizzle),
-// read as the MN-major A operand of dQ = dS K (M = queries, K = keys).
-__device__ __forceinline__ uint64_t desc_ds_mnmajor(uint32_t tile, int kk) {
-  return smem_desc(tile + kk * 16 * 128, 16384, 1024, kSwizzle128B);
+// read as the MN-major A operand of dQ = dS K (M = queries, K = keys); its
+// kk-th 16-key step lies kk * 2048 bytes on.
+__device__ __forceinline__ uint64_t desc_ds0(uint32_t tile) {
+  return smem_desc(tile, 16384, 1024, kSwizzle128B);
 }
 
 // Byte offset of 16-byte group `g` (8 bf16 columns, 0..15) of row `r` in the
@@ -423,35 +440,39 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
       auto qfull = [&](int it) { return wait(B_QFULL + it % L::STAGES, (it / L::STAGES) & 1); };
       auto sbuf = [&](int it) { return L::T_S + 128 * (it % L::SBUF); };
       // S^T(it) = K_j Q_i^T -> S buffer it % SBUF
+      const uint64_t dK = desc_k0<D>(sK), dV = desc_k0<D>(sV);
+      const uint64_t dKmn = desc_mn0<D>(sK), dDS = desc_ds0(sdS);
       auto issue_s = [&](int it) {
-        const uint32_t sQ = stage_q(it);
+        const uint64_t dQ = desc_k0<D>(stage_q(it));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + sbuf(it), desc_kmajor<D>(sK, kk), desc_kmajor<D>(sQ, kk), ID_S, kk > 0);
+          mma_ss(tmem + sbuf(it), dK + koff<D>(kk), dQ + koff<D>(kk), ID_S, kk > 0);
         if (!(p.inject_fault && it == 0)) mma_commit(&bars[B_SFULL + it % L::SBUF]);
       };
       // dP^T(it) = V_j dO_i^T -> region B
       auto issue_dp = [&](int it) {
-        const uint32_t sdO = stage_do(it);
+        const uint64_t ddO = desc_k0<D>(stage_do(it));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::T_DP, desc_kmajor<D>(sV, kk), desc_kmajor<D>(sdO, kk), ID_S, kk > 0);
+          mma_ss(tmem + L::T_DP, dV + koff<D>(kk), ddO + koff<D>(kk), ID_S, kk > 0);
         mma_commit(&bars[B_DPFULL]);
       };
       // dV_j += P^T dO_i, P^T read from the tile's S buffer (K = 128 queries)
       auto issue_dv = [&](int it) {
+        const uint64_t ddO = desc_mn0<D>(stage_do(it));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DV, tmem + sbuf(it) + p_col<QC>(16 * kk),
-                 desc_mnmajor<D>(stage_do(it), kk), ID_KV, (it > 0 || kk > 0));
+          mma_ts(tmem + L::T_DV, tmem + sbuf(it) + p_col<QC>(16 * kk), ddO + mnoff<D>(kk), ID_KV,
+                 (it > 0 || kk > 0));
         mma_commit(&bars[B_DVDONE]);
       };
       // dK_j += dS^T Q_i, dS^T read from region B
       auto issue_dk = [&](int it) {
+        const uint64_t dQ = desc_mn0<D>(stage_q(it));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk),
-                 desc_mnmajor<D>(stage_q(it), kk), ID_KV, (it > 0 || kk > 0));
+          mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk), dQ + mnoff<D>(kk), ID_KV,
+                 (it > 0 || kk > 0));
         mma_commit(&bars[B_DKDONE]);
       };
       // dQ_i = dS K_j (dS from shared memory) -> region B (d = 128) or the
@@ -460,7 +481,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
         const uint32_t dst = L::DQ_OVER_DP ? L::T_DP : sbuf(it);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + dst, desc_ds_mnmajor(sdS, kk), desc_mnmajor<D>(sK, kk), ID_Q, kk > 0);
+          mma_ss(tmem + dst, dDS + kk * 128, dKmn + mnoff<D>(kk), ID_Q, kk > 0);
         mma_commit(&bars[B_DQFULL + (it & 1)]);
         mma_commit(&bars[B_QEMPTY + it % L::STAGES]);
       };
