@@ -390,12 +390,14 @@ def test_double_backward_against_the_oracle(csa, B, H, N, d, causal):
 
 
 @pytest.mark.parametrize("B,H,N,d,causal", [(1, 2, 2100, 64, True), (1, 1, 2048 + 77, 128, True),
-                                             (2, 1, 300, 32, True), (1, 2, 700, 64, False),
+                                             (2, 1, 300, 32, True), (1, 1, 1100, 32, True),
+                                             (1, 2, 700, 64, False), (2, 3, 260, 64, False),
                                              (2, 2, 129, 128, False), (1, 1, 1, 64, True)])
 def test_double_backward_bf16_against_the_oracle(csa, B, H, N, d, causal):
     # the tensor-core kernels: 2,100 and 2,125 tokens walk 17 tiles (key tile
-    # 0 meets every query tile); N = 1 has the closed form gQ = gK = gV = 0,
-    # gdO = U_V. The oracle takes the bf16-rounded inputs widened to float64.
+    # 0 meets every query tile), 1,100 at d = 32 nine (three score sets in both
+    # sweeps); N = 1 has the closed form gQ = gK = gV = 0, gdO = U_V. The
+    # oracle takes the bf16-rounded inputs widened to float64.
     q, k, v, do = draw(B, H, N, d, 800 + N, "bf16")
     uq, uk, uv, _ = draw(B, H, N, d, 850 + N, "bf16")
     scale = d ** -0.5
