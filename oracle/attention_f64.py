@@ -295,15 +295,24 @@ def backward_blocked(q, k, v, do, scale, causal=True, rows_per_block=1024):
     return out
 
 
-def key_tail(q, k, v, do, scale, j0):
+def key_tail(q, k, v, do, scale, j0, rows_per_block=None):
     """dK and dV of keys j >= j0 of one causal head.
 
     Under the causal filter key j only meets query rows i >= j, so the tail
     needs rows j0..N-1 only (each row's softmax is still over all its keys).
+    rows_per_block splits those rows into blocks whose dK, dV contributions
+    are summed (the same sums over the same rows, holding rows_per_block x N
+    of the score table at a time instead of (N - j0) x N).
     """
     n = q.shape[0]
-    blk = backward_row_block(q, k, v, do, scale, j0, n, causal=True)
-    return {"dK": blk["dK"][j0:], "dV": blk["dV"][j0:]}
+    step = (n - j0) if rows_per_block is None else rows_per_block
+    dk = np.zeros((n - j0, np.asarray(k).shape[1]))
+    dv = np.zeros((n - j0, np.asarray(v).shape[1]))
+    for r0 in range(j0, n, step):
+        blk = backward_row_block(q, k, v, do, scale, r0, min(r0 + step, n), causal=True)
+        dk += blk["dK"][j0:]
+        dv += blk["dV"][j0:]
+    return {"dK": dk, "dV": dv}
 
 
 def causal_pair_count(B: int, H: int, N: int) -> int:

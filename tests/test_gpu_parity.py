@@ -681,7 +681,7 @@ def sampled_parity(csa, name, heads, n_rows=24, tail=128, full_heads=()):
         assert rel(gq, r["dQ"]) <= TOL[c.dtype]
         assert rel(as_f64(g["O"][b, h].cpu())[rows], r["O"]) <= TOL[c.dtype]
         assert np.abs(as_f64(g["LSE"][b, h].cpu())[rows] - r["LSE"]).max() <= 1e-3
-        t = oracle.key_tail(qh, kh, vh, doh, c.scale, c.N - tail)
+        t = oracle.key_tail(qh, kh, vh, doh, c.scale, c.N - tail, rows_per_block=256)
         assert rel(as_f64(g["dK"][b, h].cpu())[-tail:], t["dK"]) <= TOL[c.dtype]
         assert rel(as_f64(g["dV"][b, h].cpu())[-tail:], t["dV"]) <= TOL[c.dtype]
     # identities over all positions: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
@@ -701,4 +701,6 @@ def test_long_sequence_16k_parity(csa):
 
 
 def test_long_sequence_262k_parity(csa):
-    sampled_parity(csa, "c5", heads=[(0, 0), (0, 3)], n_rows=16, tail=64)
+    # sampled dQ rows, and dK / dV of the last 2,048 keys (their 2,048 query
+    # rows, each over all its 262,144 keys, in 256-row oracle blocks)
+    sampled_parity(csa, "c5", heads=[(0, 0), (0, 3)], n_rows=16, tail=2048)

@@ -340,6 +340,10 @@ def test_query_rows_and_row_blocks(causal):
         tail = A.key_tail(q, k, v, do, 0.35, 50)
         assert rel(tail["dK"], full["dK"][50:]) <= 1e-12
         assert rel(tail["dV"], full["dV"][50:]) <= 1e-12
+        # the same tail from row blocks (a ragged last block included)
+        tail = A.key_tail(q, k, v, do, 0.35, 50, rows_per_block=7)
+        assert rel(tail["dK"], full["dK"][50:]) <= 1e-12
+        assert rel(tail["dV"], full["dV"][50:]) <= 1e-12
 
 
 @pytest.mark.parametrize("causal,block", [(True, 16), (True, 23), (False, 16), (True, 1000)])
