@@ -78,6 +78,10 @@ struct Roles {
   static constexpr int DQ_WARP0 = 4 * EG;
   static constexpr int MMA_WARP = DQ_WARP0 + 4;
   static constexpr int TMA_WARP = MMA_WARP + 1;
+  // d = 128: a second issuer for the gradient MMAs (dV, dK, dQ), so that they
+  // never wait behind a score MMA batch that cannot enter the tensor pipe's
+  // queue yet (an MMA issue waits while the queue is full)
+  static constexpr int MMA2_WARP = MMA_WARP + 2;
   static constexpr int THREADS = (MMA_WARP + 4) * 32;
   static constexpr int WGS = THREADS / 128;
   // registers a thread holds at launch (the per-block 64K, in steps of 8)
@@ -146,7 +150,7 @@ struct BwdLayout {
 // Barrier slots: up to three Q / dO stages, up to two S buffers.
 enum Bar {
   B_KV = 0, B_QFULL = 1, B_QEMPTY = 4, B_SFULL = 7, B_DPFULL = 9, B_PFULL, B_DSFULL, B_DVDONE,
-  B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2, B_DONE = B_DQREAD + 2, B_FINAL, B_COUNT
+  B_DKDONE, B_DQFULL, B_DQREAD = B_DQFULL + 2, B_DONE = B_DQREAD + 2, B_FINAL, B_FINAL2, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
@@ -346,6 +350,7 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
     mbar_init(&bars[B_DKDONE], 1);
     mbar_init(&bars[B_DONE], 1);
     mbar_init(&bars[B_FINAL], 1);
+    mbar_init(&bars[B_FINAL2], 1);
     *abort_flag = 0;
     *const_cast<volatile int*>(never) = 0;
     fence_barrier_init();
@@ -418,15 +423,20 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
         mbar_wait(&bars[B_QFULL + w % L::STAGES], (w / L::STAGES) & 1, p.wait_cycles, never);
     }
     __syncwarp();
-  } else if (warp == R::MMA_WARP) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == R::MMA_WARP || (!L::PIPE_S && warp == R::MMA2_WARP)) {
+    // ------------------------------------------------ MMA issuers
     // Each wait guards one TMEM or shared-memory region against the MMA that
-    // overwrites it. d = 128, per query tile i: dV(i), S(i+1), dK(i), dQ(i),
-    // dP(i+1), with S(0) and dP(0) before the loop; S(i+1) overwrites P(i)
-    // and so waits for dV(i). d <= 64 (two S buffers): S(i+1), dV(i), dK(i),
-    // dQ(i), dP(i+1): S(i+1) goes into the other buffer as soon as its last
-    // reader (the read-out of dQ(i-1)) is done, so the element-wise warps
-    // find it ready when they finish dS(i).
+    // overwrites it. d = 128, two issuers: warp MMA_WARP issues the score
+    // MMAs S(i+1) (it overwrites P(i), so it waits for dV(i)) and dP(i+1) (it
+    // overwrites region B, where dQ(i) lands, so it waits for dQ(i)'s
+    // read-out), with S(0) and dP(0) before the loop; warp MMA2_WARP issues
+    // dV(i), dK(i) and dQ(i) (which overwrites dS^T(i), so it waits for
+    // dK(i)). Every barrier is committed by one thread, and each issuer's
+    // queue no longer holds the other's MMAs behind a full tensor pipe.
+    // d <= 64 (two S buffers), one issuer: S(i+1), dV(i), dK(i), dQ(i),
+    // dP(i+1): S(i+1) goes into the other buffer as soon as its last reader
+    // (the read-out of dQ(i-1)) is done, so the element-wise warps find it
+    // ready when they finish dS(i).
     if (elect_one_sync()) {
       const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sdS = sbase + L::DS_OFF;
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
@@ -485,12 +495,15 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
         mma_commit(&bars[B_DQFULL + (it & 1)]);
         mma_commit(&bars[B_QEMPTY + it % L::STAGES]);
       };
+      const bool scores = L::PIPE_S || warp == R::MMA_WARP;  // S and dP
+      const bool grads = L::PIPE_S || warp == R::MMA2_WARP;  // dV, dK, dQ
       bool ok = true;
-      if (i_first < p.T && (ok = wait(B_KV, 0) && qfull(0))) {
+      if (scores && i_first < p.T && (ok = wait(B_KV, 0) && qfull(0))) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
+      if (!scores && i_first < p.T) ok = wait(B_KV, 0);
       for (int it = 0, i = i_first; ok && i < p.T; ++it, i = next_tile(i)) {
         const bool more = next_tile(i) < p.T;
         if constexpr (L::PIPE_S) {
@@ -517,39 +530,41 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
             tc_fence_after();
             issue_dp(it + 1);
           }
-        } else {
-          if (!(ok = wait(B_PFULL, it & 1))) break;
-          tc_fence_after();
-          issue_dv(it);
+        } else if (scores) {
           if (more) {
             // S^T(it+1) overwrites P^T(it), which dV(it) reads.
             if (!(ok = qfull(it + 1))) break;
             if (!(ok = wait(B_DVDONE, it & 1))) break;
             tc_fence_after();
             issue_s(it + 1);
+            // dP^T(it+1) overwrites region B, where dQ(it) lands; its
+            // read-out also means dQ(it) has finished reading dS(it) from
+            // shared memory, which the element-wise warps overwrite next
+            if (!(ok = wait(B_DQREAD + (it & 1), (it >> 1) & 1))) break;
+            tc_fence_after();
+            issue_dp(it + 1);
           }
+        } else {
+          if (!(ok = wait(B_PFULL, it & 1))) break;
+          tc_fence_after();
+          issue_dv(it);
           if (!(ok = wait(B_DSFULL, it & 1))) break;
           tc_fence_after();
           issue_dk(it);
           if (!(ok = wait(B_DKDONE, it & 1))) break;  // dQ(it) overwrites dS^T(it)
           tc_fence_after();
           issue_dq(it);
-          if (more) {
-            // dP^T(it+1) overwrites region B, where dQ(it) lands
-            if (!(ok = wait(B_DQREAD + (it & 1), (it >> 1) & 1))) break;
-            tc_fence_after();
-            issue_dp(it + 1);
-          }
         }
       }
-      if (ok) {
-        mma_commit(&bars[B_DONE]);
-      } else {
+      if (!ok) {
         fail();
+      } else if (grads) {
+        mma_commit(&bars[B_DONE]);
       }
       // Every MMA this thread issued has finished before TMEM is freed.
-      mma_commit(&bars[B_FINAL]);
-      mbar_wait(&bars[B_FINAL], 0, p.wait_cycles, never);
+      const int fin = warp == R::MMA_WARP ? B_FINAL : B_FINAL2;
+      mma_commit(&bars[fin]);
+      mbar_wait(&bars[fin], 0, p.wait_cycles, never);
     }
     __syncwarp();
   }
