@@ -466,8 +466,11 @@ def test_linearity_and_causality(csa):
     assert torch.equal(lp, lse[:, perm])
 
 
-def test_timeout_is_reported_and_context_survives(csa):
-    B, H, N, d = 1, 1, 256, 64
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_timeout_is_reported_and_context_survives(csa, d):
+    # every d: one MMA issuer at d <= 64, two at d = 128; each side's bounded
+    # waits must end once the first score tile never arrives
+    B, H, N = 1, 1, 256
     q, k, v, do = draw(B, H, N, d, 9, "bf16")
     dev = torch.device("cuda")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
