@@ -493,8 +493,18 @@ int attn_bwd_bwd(const void* q, const void* k, const void* v, const void* o, con
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     st = from_cuda(launch_preprocess(o, dout, lse, B * H, N, d, true, rs, ws, s));
     if (st != ATTN_OK) return st;
+    int inject = 0;
+    unsigned long long limit = kWaitLimitCycles;
+    {
+      std::lock_guard<std::mutex> g(g_fault_mu);
+      if (g_fault.armed) {
+        inject = 1;
+        limit = g_fault.limit_cycles;
+        g_fault.armed = 0;
+      }
+    }
     return from_cuda(launch_bob_bf16(maps, src, ws, r_pad, g_pad, gq, gk, gv, gdout, B * H, H, N, d,
-                                     causal != 0, scale, s));
+                                     causal != 0, scale, limit, inject, s));
   }
   st = preprocess_impl(o, dout, lse, B, H, N, d, dtype, workspace, workspace_bytes,
                        dense(H, N, d), stream);

@@ -179,6 +179,7 @@ struct BobParams {
   int N, Np, T, BH, H, G, causal;  // H splits bh into the tensor maps' (head, batch)
   float scale, scale_log2;
   uint64_t wait_cycles;
+  int inject_fault;  // rows kernel: never signal the first score quarter (the timeout test)
 };
 
 // K-major operand slice kk (16 elements of the contraction) of a [rows][D]
@@ -613,7 +614,7 @@ __global__ void __launch_bounds__(kBobThreads, 1)
         if (k < first_acc) {
           const int s = k % T1::NSET;
           issue_scores<D, T1::TS>(tmem + T1::SET0 + s * kTSet, a_tmem, b);
-          mma_commit(&bars[O_SFULL1 + s]);
+          if (!(p.inject_fault && k == 0)) mma_commit(&bars[O_SFULL1 + s]);
         } else {
           const int s = (k - first_acc) % T2::NSET;
           issue_scores<D, T2::TS>(tmem + T2::SET0 + s * kTSet, T2::TS ? a_tmem : a_smem, b);
@@ -937,7 +938,7 @@ template <int D>
 cudaError_t launch_bob_bf16_d(const CUtensorMap (&maps)[7], const void* const (&src)[7],
                               const Workspace& ws, float* r_pad, float* g_pad, void* gq, void* gk,
                               void* gv, void* gdo, int BH, int H, int N, bool causal, float scale,
-                              cudaStream_t s) {
+                              uint64_t wait_limit_cycles, int inject_fault, cudaStream_t s) {
   using L = BobLayout<D>;
   static_assert(L::ALLOC <= 232448, "shared memory window exceeds 227 KB");
   for (auto k : {bob_rows_bf16_kernel<D>, bob_cols_bf16_kernel<D>}) {
@@ -968,7 +969,8 @@ cudaError_t launch_bob_bf16_d(const CUtensorMap (&maps)[7], const void* const (&
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.wait_cycles = kWaitLimitCycles;
+  p.wait_cycles = wait_limit_cycles;
+  p.inject_fault = inject_fault;
   const unsigned grid = static_cast<unsigned>(p.T) * static_cast<unsigned>(BH);
   // rows kernel: resident Q, dO, U_Q (src order q, k, v, dout, uq, uk, uv)
   p.res[0] = bf(src[0]);
@@ -988,6 +990,7 @@ cudaError_t launch_bob_bf16_d(const CUtensorMap (&maps)[7], const void* const (&
   p.res[3] = bf(src[6]);
   p.out0 = static_cast<__nv_bfloat16*>(gk);
   p.out1 = static_cast<__nv_bfloat16*>(gv);
+  p.inject_fault = 0;
   bob_cols_bf16_kernel<D><<<grid, kBobThreads, L::ALLOC, s>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
   return cudaGetLastError();
@@ -998,17 +1001,18 @@ cudaError_t launch_bob_bf16_d(const CUtensorMap (&maps)[7], const void* const (&
 cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const void* const (&src)[7],
                             const Workspace& ws, float* r_pad, float* g_pad, void* gq, void* gk,
                             void* gv, void* gdo, int BH, int H, int N, int d, bool causal,
-                            float scale, cudaStream_t s) {
+                            float scale, uint64_t wait_limit_cycles, int inject_fault,
+                            cudaStream_t s) {
   switch (d) {
     case 32:
       return launch_bob_bf16_d<32>(maps, src, ws, r_pad, g_pad, gq, gk, gv, gdo, BH, H, N, causal,
-                                   scale, s);
+                                   scale, wait_limit_cycles, inject_fault, s);
     case 64:
       return launch_bob_bf16_d<64>(maps, src, ws, r_pad, g_pad, gq, gk, gv, gdo, BH, H, N, causal,
-                                   scale, s);
+                                   scale, wait_limit_cycles, inject_fault, s);
     case 128:
       return launch_bob_bf16_d<128>(maps, src, ws, r_pad, g_pad, gq, gk, gv, gdo, BH, H, N,
-                                    causal, scale, s);
+                                    causal, scale, wait_limit_cycles, inject_fault, s);
     default:
       return cudaErrorInvalidValue;
   }

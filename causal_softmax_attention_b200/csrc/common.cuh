@@ -125,10 +125,13 @@ cudaError_t launch_bwd_bf16(const TmaMaps& maps, const Workspace& ws, void* dk, 
 // contiguous [B][H][N][d]); needs the bf16 preprocess's lse_pad and d_pad in
 // `ws`, and writes the two row scalars to r_pad, g_pad ([BH][Np] each).
 // maps and src: q, k, v, dout, uq, uk, uv (contiguous [BH][N][d] bf16)
+// wait_limit_cycles bounds every device wait; inject_fault withholds the rows
+// kernel's first score signal (the timeout test's hook)
 cudaError_t launch_bob_bf16(const CUtensorMap (&maps)[7], const void* const (&src)[7],
                             const Workspace& ws, float* r_pad, float* g_pad, void* gq, void* gk,
                             void* gv, void* gdo, int BH, int H, int N, int d, bool causal,
-                            float scale, cudaStream_t s);
+                            float scale, uint64_t wait_limit_cycles, int inject_fault,
+                            cudaStream_t s);
 
 int* fwd_status_ptr();  // library-owned forward status word on the current device
 

@@ -266,11 +266,12 @@ const char* attn_status_string(int status);
 
 /*
  * Failure-detection hook for tests. Arms a one-shot fault for the NEXT bf16
- * attn_bwd_main (or attn_bwd) call in this process: that launch withholds the
- * signal that its first score tile is ready and bounds each of its device
- * waits by `wait_limit_cycles` SM clock cycles, so the waits run out, the
- * kernel writes ATTN_ERR_TIMEOUT into the workspace status word, releases its
- * tensor memory and returns. No fault, trap or unbounded wait is involved; the
+ * attn_bwd_main (or attn_bwd) or bf16 attn_bwd_bwd call in this process: that
+ * launch withholds the signal that its first score tile (backward-over-
+ * backward: the rows kernel's first score quarter) is ready and bounds each
+ * of its device waits by `wait_limit_cycles` SM clock cycles, so the waits
+ * run out, the kernel writes ATTN_ERR_TIMEOUT into the workspace status word,
+ * releases its tensor memory and returns. No fault, trap or unbounded wait is involved; the
  * outputs of that call are undefined. Returns ATTN_ERR_INVALID for
  * wait_limit_cycles == 0.
  */

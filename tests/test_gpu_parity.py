@@ -416,6 +416,34 @@ def test_double_backward_bf16_against_the_oracle(csa, B, H, N, d, causal):
         assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["bf16"], name
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_double_backward_timeout_is_reported(csa, d):
+    # the armed one-shot fault withholds the rows kernel's first score
+    # quarter: every bounded wait of both issuers, the TMA warp and the
+    # element-wise warps ends, the status word says so, and the next call is
+    # unaffected
+    B, H, N = 1, 1, 300
+    q, k, v, do = draw(B, H, N, d, 860 + d, "bf16")
+    uq, uk, uv, _ = draw(B, H, N, d, 870 + d, "bf16")
+    dev = torch.device("cuda")
+    qd, kd, vd, dod, uqd, ukd, uvd = (t.to(dev) for t in (q, k, v, do, uq, uk, uv))
+    o, lse = csa.forward(qd, kd, vd, True, d ** -0.5)
+    ws = torch.empty(csa.library().attn_bwd_bwd_workspace_bytes(B, H, N, d, csa.ATTN_BF16),
+                     dtype=torch.uint8, device=dev)
+    outs = [torch.empty_like(qd) for _ in range(4)]
+    assert csa.attn_test_arm_timeout(50_000_000) == csa.ATTN_OK
+    csa.attn_bwd_bwd(qd, kd, vd, o, dod, lse, uqd, ukd, uvd, *outs, ws, True, d ** -0.5)
+    torch.cuda.synchronize()
+    assert csa.attn_last_status(ws) == csa.ATTN_ERR_TIMEOUT
+    csa.attn_bwd_bwd(qd, kd, vd, o, dod, lse, uqd, ukd, uvd, *outs, ws, True, d ** -0.5)
+    torch.cuda.synchronize()
+    assert csa.attn_last_status(ws) == csa.ATTN_OK
+    ref = oracle.double_backward(*(as_f64(t) for t in (q, k, v, do, uq, uk, uv)), d ** -0.5, True)
+    gscale = max(np.abs(ref[n]).max() for n in ("gQ", "gK", "gV", "gdO"))
+    for name, t in zip(("gQ", "gK", "gV", "gdO"), outs):
+        assert rel(as_f64(t.cpu()), ref[name], gscale) <= TOL["bf16"], name
+
+
 def test_forward_exponential_polynomial(csa):
     # the forward computes one exponential in four on the FMA pipe (Cody-Waite
     # reduction, degree-3 polynomial): against exact 2^x and against MUFU's
