@@ -31,11 +31,12 @@
 //               that lane; it copies the whole dQ row out of TMEM, releases
 //               the columns, then adds the row into the fp32 accumulator with
 //               red.global.add while the next tiles are computed.
-//   warp 12     MMA issuer (one elected lane).
+//   warp 12     MMA issuer (one elected lane); at d = 128 only S^T and dP^T.
 //   warp 13     TMA producer (one elected lane): K_j, V_j once; Q_i, dO_i and
 //               the tile's LSE / D rows per query tile, three stages deep at
 //               d <= 64, two at d = 128.
-//   warps 14-15 idle (they complete the fourth warpgroup, which setmaxnreg
+//   warp 14     d = 128: the second MMA issuer (dV, dK, dQ); idle at d <= 64.
+//   warp 15     idle (it completes the fourth warpgroup, which setmaxnreg
 //               needs to move registers to the dQ and element-wise warps).
 // TMEM (512 columns). d = 128: region A [0,128) holds S^T, then P^T as bf16
 // (query q at column 64*(q/64) + (q%64)/2); region B [128,256) holds dP^T,
@@ -65,8 +66,9 @@ using namespace sm100;
 // Warp roles: two element-wise warpgroups (thread t of group g owns TMEM lane
 // t, key row j0 + t, and query columns [QC*g, QC*(g+1))), one dQ warpgroup
 // (thread = query row of the dQ tile; a whole row of up to 128 channels), and
-// a control warpgroup whose warp MMA_WARP issues the MMAs and warp TMA_WARP
-// the TMA loads (its other two warps idle). Four element-wise warpgroups at
+// a control warpgroup whose warp MMA_WARP issues the MMAs (at d = 128 it and
+// warp MMA2_WARP split them) and warp TMA_WARP the TMA loads. Four
+// element-wise warpgroups at
 // d <= 64, with dQ read out by them, measured slower (736 vs 791 TFLOP/s on
 // 8 heads of 32K tokens): that pass is bound by its MUFU and issue slots, not
 // by latency.
