@@ -700,6 +700,9 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       int lim = p.N - kb;                                       // columns u >= lim are masked
       if (p.causal && row - kb + 1 < lim) lim = row - kb + 1;
       const uint32_t col = lane_base + (second ? T2::SET0 : T1::SET0) + b * kTSet + 16 * g;
+      // the masked pass is taken by the whole warp whenever one lane needs
+      // it: the TMEM accesses that follow are warp-collective, and a per-lane
+      // choice lets the compiler issue them from divergent paths
       uint32_t s[16], dp[16], m[16], w[16];
       tmem_ld16(col + kTS, s);
       tmem_ld16(col + kTDP, dp);
@@ -708,13 +711,13 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       tmem_ld_wait(s, dp);
       tmem_ld_wait(m, w);
       if (!second) {
-        if (lim < 16)
+        if (__any_sync(0xffffffffu, lim < 16))
           rows_sums<true>(s, dp, m, w, sl2, nl2, sc2, lim, r_acc, g_acc);
         else
           rows_sums<false>(s, dp, m, w, sl2, nl2, sc2, lim, r_acc, g_acc);
       } else {
         uint32_t o_ds[8], o_ds2[8], o_e[8], o_p[8];
-        if (lim < 16)
+        if (__any_sync(0xffffffffu, lim < 16))
           second_pass<true, true>(s, dp, m, w, sl2, sc2, nl2, dv2, r2, g2, nullptr, lim, o_ds,
                                   o_ds2, o_e, o_p);
         else
@@ -899,6 +902,9 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       if (key >= p.N) thr = 16;
       else if (p.causal) thr = key - (unit_query(u) + qo);
       const uint32_t col = lane_base + T2::SET0 + b * kTSet + 16 * g;
+      // the masked pass is taken by the whole warp whenever one lane needs
+      // it: the TMEM accesses that follow are warp-collective, and a per-lane
+      // choice lets the compiler issue them from divergent paths
       uint32_t s[16], dp[16], m[16], w[16];
       tmem_ld16(col + kTS, s);
       tmem_ld16(col + kTDP, dp);
@@ -907,7 +913,7 @@ __global__ void __launch_bounds__(kBobThreads, 1)
       tmem_ld_wait(s, dp);
       tmem_ld_wait(m, w);
       uint32_t o_ds[8], o_ds2[8], o_e[8], o_p[8];
-      if (thr > 0)
+      if (__any_sync(0xffffffffu, thr > 0))
         second_pass<true, false>(s, dp, m, w, sl2, sc2, 0, 0, 0, 0, vec, thr, o_ds, o_ds2, o_e,
                                  o_p);
       else
