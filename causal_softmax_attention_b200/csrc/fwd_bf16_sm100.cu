@@ -19,12 +19,18 @@
 // before the next P V accumulates, which after the first tiles is rare.
 //
 // Warps (384 threads): 0-7 two softmax warpgroups (thread t of group g owns
-// query row i0 + t = TMEM lane t, key columns [64g, 64g+64) of every S tile
-// and O channels [g*d/2, (g+1)*d/2)); the two halves of a row exchange their
-// maxima through shared memory. Warp 8 issues the MMAs, warp 9 loads K tiles
-// and warp 10 V tiles by TMA; warp 11 idles. TMEM: three S buffers
-// [0,384), O [384, 384+d): S_{j+2} is computed while the softmax works on
-// S_{j+1} and P_j V_j accumulates.
+// query row i0 + t = TMEM lane t and key columns [64g, 64g+64) of every S
+// tile). At d <= 64 each group keeps its own running maximum m_g, sum z_g
+// and accumulator O_g = sum over its keys of P V (the P V MMA runs as two
+// K = 64 halves), so the groups never wait for each other inside the key
+// loop; the epilogue combines the halves once:
+//   M = max(m_0, m_1), a_g = 2^(m_g - M), O = (a_0 O_0 + a_1 O_1) / (a_0 z_0 + a_1 z_1).
+// At d = 128 two accumulators do not fit beside three S buffers: the groups
+// share O (group g owns channels [g*d/2, (g+1)*d/2) for rescaling) and
+// exchange their half-row maxima through shared memory every tile. Warp 8
+// issues the MMAs, warp 9 loads K tiles and warp 10 V tiles by TMA; warp 11
+// idles. TMEM: three S buffers [0,384), then O (or O_0, O_1): S_{j+2} is
+// computed while the softmax works on S_{j+1} and P_j V_j accumulates.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -75,15 +81,24 @@ struct FwdLayout {
   static constexpr int BYTES = MASK_OFF + 2 * 4 * MASK_WORDS;
   static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
   static constexpr int SBUF = 3;                    // S buffers in TMEM
+  // one O accumulator per softmax group (O_g at T_O + g * D), or one shared
+  static constexpr bool SPLIT = D <= 64;
   static constexpr uint32_t T_S = 0, T_O = 128 * SBUF;
   static constexpr uint32_t T_COLS = 512;
-  static constexpr int HALF_D = D / 2;              // O channels per softmax group
-  static_assert(T_O + D <= T_COLS, "TMEM columns exceeded");
+  static constexpr int HALF_D = D / 2;              // O channels per softmax group (shared O)
+  static_assert(T_O + (SPLIT ? 2 : 1) * D <= T_COLS, "TMEM columns exceeded");
 };
 
+// F_PFULL + 2g + (j & 1): group g's half of P_j is in TMEM (F_PFULL alone,
+// both groups arriving, with a shared O). A group can then finish two tiles
+// before the issuer looks (the other group holding the issuer up) without
+// the phases aliasing: its P_{j+2} needs S_{j+2}, issued only after P_j was
+// consumed. F_PVDONE + (j & 1): P_j V_j has completed (with split
+// accumulators: group 0's half), F_PVDONE1 + (j & 1): both halves have.
 enum FBar {
   F_Q = 0, F_KFULL = 1, F_KEMPTY = 3, F_VFULL = 5, F_VEMPTY = 7, F_SFULL = 9,
-  F_PFULL = F_SFULL + 3, F_PVDONE, F_XCHG = F_PVDONE + 2, F_FINAL, F_COUNT
+  F_PFULL = F_SFULL + 3, F_PVDONE = F_PFULL + 4, F_PVDONE1 = F_PVDONE + 2, F_XCHG = F_PVDONE1 + 2,
+  F_FINAL, F_COUNT
 };
 static_assert(F_COUNT <= 32, "barrier slots");
 
@@ -184,9 +199,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&bars[F_VFULL + s], 1);
       mbar_init(&bars[F_VEMPTY + s], 1);
       mbar_init(&bars[F_PVDONE + s], 1);
+      mbar_init(&bars[F_PVDONE1 + s], 1);
     }
+    for (int s = 0; s < 4; ++s)
+      mbar_init(&bars[F_PFULL + s], L::SPLIT ? kSoftmaxThreads / 2 : kSoftmaxThreads);
     for (int s = 0; s < 3; ++s) mbar_init(&bars[F_SFULL + s], 1);
-    mbar_init(&bars[F_PFULL], kSoftmaxThreads);
     mbar_init(&bars[F_XCHG], kSoftmaxThreads);
     mbar_init(&bars[F_FINAL], 1);
     *abort_flag = 0;
@@ -274,20 +291,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (next_tile(j_first) < p.Tk && (ok = wait(F_KFULL + 1, 0))) issue_s(1);
       }
       for (int jt = 0, j = j_first; ok && j < p.Tk; ++jt, j = next_tile(j)) {
-        if (!(ok = wait(F_PFULL, jt & 1))) break;
-        if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
-        tc_fence_after();
         const uint32_t sV = sbase + L::V_OFF + (jt & 1) * L::TILE;
         const uint32_t pbuf = tmem + L::T_S + (jt % 3) * 128;
+        if constexpr (L::SPLIT) {
+          // O_g += P_j[:, group g's 64 keys] V_j[those keys], each half as
+          // soon as its group has written it
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::T_O, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk), ID_O,
-                 (jt > 0 || kk > 0));
-        mma_commit(&bars[F_PVDONE + (jt & 1)]);
+          for (int g = 0; g < 2; ++g) {
+            if (!(ok = wait(F_PFULL + 2 * g + (jt & 1), (jt >> 1) & 1))) break;
+            if (g == 0 && !(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * g; kk < 4 * g + 4; ++kk)
+              mma_ts(tmem + L::T_O + g * D, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk),
+                     ID_O, (jt > 0 || kk > 4 * g));
+            mma_commit(&bars[(g == 0 ? F_PVDONE : F_PVDONE1) + (jt & 1)]);
+          }
+          if (!ok) break;
+        } else {
+          if (!(ok = wait(F_PFULL, jt & 1))) break;
+          if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::T_O, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk), ID_O,
+                   (jt > 0 || kk > 0));
+          mma_commit(&bars[F_PVDONE + (jt & 1)]);
+        }
         mma_commit(&bars[F_VEMPTY + (jt & 1)]);
         if (next_tile(next_tile(j)) < p.Tk) {
           // S_{j+2} overwrites P_{j-1}, which P_{j-1} V_{j-1} reads
-          if (jt >= 1 && !(ok = wait(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
+          constexpr int done = L::SPLIT ? F_PVDONE1 : F_PVDONE;
+          if (jt >= 1 && !(ok = wait(done + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
           if (!(ok = wait(F_KFULL + (jt & 1), ((jt + 2) >> 1) & 1))) break;
           tc_fence_after();
           issue_s(jt + 2);
@@ -339,12 +374,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int u = 0; u < 64; ++u) mx = fmaxf(mx, __uint_as_float(sr[u]));
       }
-      // row maximum over both halves of the row
-      float* xmj = xm + (jt & 1) * 256;
-      xmj[g * 128 + t] = mx;
-      mbar_arrive(&bars[F_XCHG]);
-      if (!(ok = wait_w(F_XCHG, jt & 1))) break;
-      mx = fmaxf(mx, xmj[(g ^ 1) * 128 + t]) * p.scale_log2;
+      if constexpr (L::SPLIT) {
+        mx *= p.scale_log2;  // this group's own running maximum
+      } else {
+        // row maximum over both halves of the row
+        float* xmj = xm + (jt & 1) * 256;
+        xmj[g * 128 + t] = mx;
+        mbar_arrive(&bars[F_XCHG]);
+        if (!(ok = wait_w(F_XCHG, jt & 1))) break;
+        mx = fmaxf(mx, xmj[(g ^ 1) * 128 + t]) * p.scale_log2;
+      }
       float alpha = 1.f;
       const bool raise = mx > m + kRescaleMargin;
       if (raise) {
@@ -352,18 +391,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = mx;
       }
       if (__any_sync(0xffffffffu, raise && jt > 0)) {
-        // O holds sum_{j' < j} P_j' V_j' with the old m: scale it by alpha
-        // once the last of those products has landed.
-        if (!(ok = wait_w(F_PVDONE + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
+        // O (this group's O_g, or its channels of the shared O) holds
+        // sum_{j' < j} P_j' V_j' with the old m: scale it by alpha once the
+        // last of those products has landed.
+        const int done = (L::SPLIT && g == 1) ? F_PVDONE1 : F_PVDONE;
+        if (!(ok = wait_w(done + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
         tc_fence_after();
+        constexpr int OCH = L::SPLIT ? D : L::HALF_D;
+        const uint32_t o_cols = L::T_O + g * (L::SPLIT ? D : L::HALF_D);
 #pragma unroll 1
-        for (int c = 0; c < L::HALF_D; c += 16) {
+        for (int c = 0; c < OCH; c += 16) {
           uint32_t ov[16];
-          tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
+          tmem_ld16(lane_base + o_cols + c, ov);
           tmem_ld_wait(ov);
 #pragma unroll
           for (int u = 0; u < 16; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
-          tmem_st16(lane_base + L::T_O + g * L::HALF_D + c, ov);
+          tmem_st16(lane_base + o_cols + c, ov);
         }
         z *= alpha;
       }
@@ -400,19 +443,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_st16(sbuf + fp_col(64 * g) + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[F_PFULL]);
+      mbar_arrive(&bars[L::SPLIT ? F_PFULL + 2 * g + (jt & 1) : F_PFULL]);
     }
     // Epilogue: the last P V has landed; combine the two halves' sums. A
     // query tile that meets no key tile has O = 0 and LSE = -inf (the log of
     // an empty sum).
     const int n_kv = jt;
-    if (ok && n_kv > 0) ok = wait_w(F_PVDONE + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    if (ok && n_kv > 0)
+      ok = wait_w((L::SPLIT ? F_PVDONE1 : F_PVDONE) + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    // split accumulators: this group's weight a_own and the other's a_oth
+    float a_own = 1.f, a_oth = 0.f;
     if (ok && n_kv > 0) {
-      float* xmz = xm + (n_kv & 1) * 256;
-      xmz[g * 128 + t] = z;
-      mbar_arrive(&bars[F_XCHG]);
-      ok = wait_w(F_XCHG, n_kv & 1);
-      if (ok) z += xmz[(g ^ 1) * 128 + t];
+      if constexpr (L::SPLIT) {
+        // the first use of the exchange buffer and its barrier
+        xm[g * 128 + t] = m;
+        xm[256 + g * 128 + t] = z;
+        mbar_arrive(&bars[F_XCHG]);
+        ok = wait_w(F_XCHG, 0);
+        if (ok) {
+          const float m2 = xm[(g ^ 1) * 128 + t], z2 = xm[256 + (g ^ 1) * 128 + t];
+          const float mm = fmaxf(m, m2);
+          // a group none of whose keys the row sees has m = -inf, z = 0
+          a_own = m == -INFINITY ? 0.f : ex2_approx(m - mm);
+          a_oth = m2 == -INFINITY ? 0.f : ex2_approx(m2 - mm);
+          z = z * a_own + z2 * a_oth;
+          m = mm;
+        }
+      } else {
+        float* xmz = xm + (n_kv & 1) * 256;
+        xmz[g * 128 + t] = z;
+        mbar_arrive(&bars[F_XCHG]);
+        ok = wait_w(F_XCHG, n_kv & 1);
+        if (ok) z += xmz[(g ^ 1) * 128 + t];
+      }
     }
     if (!ok) {
       fail();
@@ -425,7 +488,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < L::HALF_D; c += 16) {
         uint32_t ov[16];
-        if (n_kv > 0) {
+        if (n_kv > 0 && L::SPLIT) {
+          // channels [g*d/2 + c, +16) of a_0 O_0 + a_1 O_1
+          uint32_t o0[16], o1[16];
+          tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, o0);
+          tmem_ld16(lane_base + L::T_O + D + g * L::HALF_D + c, o1);
+          tmem_ld_wait(o0, o1);
+          const float a0 = g == 0 ? a_own : a_oth, a1 = g == 0 ? a_oth : a_own;
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            ov[u] = __float_as_uint(__uint_as_float(o0[u]) * a0 + __uint_as_float(o1[u]) * a1);
+        } else if (n_kv > 0) {
           tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
           tmem_ld_wait(ov);
         } else {
