@@ -20,17 +20,15 @@
 //
 // Warps (384 threads): 0-7 two softmax warpgroups (thread t of group g owns
 // query row i0 + t = TMEM lane t and key columns [64g, 64g+64) of every S
-// tile). At d <= 64 each group keeps its own running maximum m_g, sum z_g
-// and accumulator O_g = sum over its keys of P V (the P V MMA runs as two
-// K = 64 halves), so the groups never wait for each other inside the key
-// loop; the epilogue combines the halves once:
+// tile). Each group keeps its own running maximum m_g, sum z_g and
+// accumulator O_g = sum over its keys of P V (the P V MMA runs as two K = 64
+// halves), so the groups never wait for each other inside the key loop; the
+// epilogue combines the halves once:
 //   M = max(m_0, m_1), a_g = 2^(m_g - M), O = (a_0 O_0 + a_1 O_1) / (a_0 z_0 + a_1 z_1).
-// At d = 128 two accumulators do not fit beside three S buffers: the groups
-// share O (group g owns channels [g*d/2, (g+1)*d/2) for rescaling) and
-// exchange their half-row maxima through shared memory every tile. Warp 8
-// issues the MMAs, warp 9 loads K tiles and warp 10 V tiles by TMA; warp 11
-// idles. TMEM: three S buffers [0,384), then O (or O_0, O_1): S_{j+2} is
-// computed while the softmax works on S_{j+1} and P_j V_j accumulates.
+// Warp 8 issues the MMAs, warp 9 loads K tiles and warp 10 V tiles by TMA;
+// warp 11 idles. TMEM: S buffers from column 0 (three at d <= 64, two at
+// d = 128), then O_0 and O_1: S_{j+1} (and at d <= 64 S_{j+2}) is computed
+// while the softmax works on S_j and P_{j-1} V_{j-1} accumulates.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -71,7 +69,7 @@ struct FwdLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;        // [2] tiles
   static constexpr int V_OFF = K_OFF + 2 * TILE;    // [2] tiles
-  static constexpr int XM_OFF = V_OFF + 2 * TILE;   // [2][2][128] f32: row maxima / sums exchanged
+  static constexpr int XM_OFF = V_OFF + 2 * TILE;   // [2][2][128] f32: the groups' maxima, sums
   static constexpr int BAR_OFF = XM_OFF + 2048;
   static constexpr int MISC_OFF = BAR_OFF + 32 * 8;
   // block-mask bitmaps of the query tile's row (active tiles, kind-2 tiles),
@@ -80,21 +78,21 @@ struct FwdLayout {
   static constexpr int MASK_OFF = MISC_OFF + 64;
   static constexpr int BYTES = MASK_OFF + 2 * 4 * MASK_WORDS;
   static constexpr int ALLOC = (BYTES + 1024) > 118 * 1024 ? (BYTES + 1024) : 118 * 1024;
-  static constexpr int SBUF = 3;                    // S buffers in TMEM
-  // one O accumulator per softmax group (O_g at T_O + g * D), or one shared
-  static constexpr bool SPLIT = D <= 64;
+  // S buffers in TMEM, then one O accumulator per softmax group (O_g at
+  // T_O + g * D); at d = 128 the accumulators leave room for two S buffers
+  static constexpr int SBUF = D == 128 ? 2 : 3;
   static constexpr uint32_t T_S = 0, T_O = 128 * SBUF;
   static constexpr uint32_t T_COLS = 512;
-  static constexpr int HALF_D = D / 2;              // O channels per softmax group (shared O)
-  static_assert(T_O + (SPLIT ? 2 : 1) * D <= T_COLS, "TMEM columns exceeded");
+  static constexpr int HALF_D = D / 2;              // O channels each group writes out
+  static_assert(T_O + 2 * D <= T_COLS, "TMEM columns exceeded");
 };
 
-// F_PFULL + 2g + (j & 1): group g's half of P_j is in TMEM (F_PFULL alone,
-// both groups arriving, with a shared O). A group can then finish two tiles
-// before the issuer looks (the other group holding the issuer up) without
-// the phases aliasing: its P_{j+2} needs S_{j+2}, issued only after P_j was
-// consumed. F_PVDONE + (j & 1): P_j V_j has completed (with split
-// accumulators: group 0's half), F_PVDONE1 + (j & 1): both halves have.
+// F_PFULL + 2g + (j & 1): group g's half of P_j is in TMEM. A group can
+// finish two tiles before the issuer looks (the other group holding the
+// issuer up) without the phases aliasing: its P_{j+2} needs S_{j+2}, issued
+// only after P_j was consumed. F_PVDONE + (j & 1): group 0's half of
+// P_j V_j has completed, F_PVDONE1 + (j & 1): both halves have. F_XCHG: the
+// epilogue's exchange of the groups' maxima and sums.
 enum FBar {
   F_Q = 0, F_KFULL = 1, F_KEMPTY = 3, F_VFULL = 5, F_VEMPTY = 7, F_SFULL = 9,
   F_PFULL = F_SFULL + 3, F_PVDONE = F_PFULL + 4, F_PVDONE1 = F_PVDONE + 2, F_XCHG = F_PVDONE1 + 2,
@@ -145,7 +143,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const volatile int* never = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
-  float* xm = reinterpret_cast<float*>(smem + L::XM_OFF);  // [2 uses][2 groups][128 rows]
+  float* xm = reinterpret_cast<float*>(smem + L::XM_OFF);  // [m, z][2 groups][128 rows]
 
   const int warp = threadIdx.x >> 5;
   // CTA order: heads in groups of G (their K and V stay in L2 while all of
@@ -201,8 +199,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&bars[F_PVDONE + s], 1);
       mbar_init(&bars[F_PVDONE1 + s], 1);
     }
-    for (int s = 0; s < 4; ++s)
-      mbar_init(&bars[F_PFULL + s], L::SPLIT ? kSoftmaxThreads / 2 : kSoftmaxThreads);
+    for (int s = 0; s < 4; ++s) mbar_init(&bars[F_PFULL + s], kSoftmaxThreads / 2);
     for (int s = 0; s < 3; ++s) mbar_init(&bars[F_SFULL + s], 1);
     mbar_init(&bars[F_XCHG], kSoftmaxThreads);
     mbar_init(&bars[F_FINAL], 1);
@@ -266,8 +263,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncwarp();
   } else if (warp == kFwdMmaWarp) {
     // ------------------------------------------------ MMA issuer
-    // Order: S_0, S_1, then per key tile j: P_j V_j, S_{j+2} (into the buffer
-    // that P_{j-1} occupied, once P_{j-1} V_{j-1} has completed).
+    // Order: S_0, S_1, then per key tile j: the two halves of P_j V_j, then
+    // S_{j+2} into the buffer P_{j+2-SBUF} occupied, once that tile's P V has
+    // completed (P_{j-1} with three buffers: never a pipe drain, because P_j
+    // V_j is already queued; P_j with two).
     if (elect_one_sync()) {
       constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_O = idesc_bf16(128, D, false, true);
@@ -279,9 +278,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t sK = sbase + L::K_OFF + (jt & 1) * L::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::T_S + (jt % 3) * 128, fdesc_kmajor<D>(sQ, kk), fdesc_kmajor<D>(sK, kk),
+          mma_ss(tmem + L::T_S + (jt % L::SBUF) * 128, fdesc_kmajor<D>(sQ, kk), fdesc_kmajor<D>(sK, kk),
                  ID_S, kk > 0);
-        mma_commit(&bars[F_SFULL + jt % 3]);
+        mma_commit(&bars[F_SFULL + jt % L::SBUF]);
         mma_commit(&bars[F_KEMPTY + (jt & 1)]);
       };
       bool ok = true;
@@ -292,37 +291,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       for (int jt = 0, j = j_first; ok && j < p.Tk; ++jt, j = next_tile(j)) {
         const uint32_t sV = sbase + L::V_OFF + (jt & 1) * L::TILE;
-        const uint32_t pbuf = tmem + L::T_S + (jt % 3) * 128;
-        if constexpr (L::SPLIT) {
-          // O_g += P_j[:, group g's 64 keys] V_j[those keys], each half as
-          // soon as its group has written it
+        const uint32_t pbuf = tmem + L::T_S + (jt % L::SBUF) * 128;
+        // O_g += P_j[:, group g's 64 keys] V_j[those keys], each half as soon
+        // as its group has written it
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (!(ok = wait(F_PFULL + 2 * g + (jt & 1), (jt >> 1) & 1))) break;
-            if (g == 0 && !(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 4 * g; kk < 4 * g + 4; ++kk)
-              mma_ts(tmem + L::T_O + g * D, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk),
-                     ID_O, (jt > 0 || kk > 4 * g));
-            mma_commit(&bars[(g == 0 ? F_PVDONE : F_PVDONE1) + (jt & 1)]);
-          }
-          if (!ok) break;
-        } else {
-          if (!(ok = wait(F_PFULL, jt & 1))) break;
-          if (!(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
+        for (int g = 0; g < 2; ++g) {
+          if (!(ok = wait(F_PFULL + 2 * g + (jt & 1), (jt >> 1) & 1))) break;
+          if (g == 0 && !(ok = wait(F_VFULL + (jt & 1), (jt >> 1) & 1))) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + L::T_O, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk), ID_O,
-                   (jt > 0 || kk > 0));
-          mma_commit(&bars[F_PVDONE + (jt & 1)]);
+          for (int kk = 4 * g; kk < 4 * g + 4; ++kk)
+            mma_ts(tmem + L::T_O + g * D, pbuf + fp_col(16 * kk), fdesc_mnmajor<D>(sV, kk),
+                   ID_O, (jt > 0 || kk > 4 * g));
+          mma_commit(&bars[(g == 0 ? F_PVDONE : F_PVDONE1) + (jt & 1)]);
         }
+        if (!ok) break;
         mma_commit(&bars[F_VEMPTY + (jt & 1)]);
         if (next_tile(next_tile(j)) < p.Tk) {
-          // S_{j+2} overwrites P_{j-1}, which P_{j-1} V_{j-1} reads
-          constexpr int done = L::SPLIT ? F_PVDONE1 : F_PVDONE;
-          if (jt >= 1 && !(ok = wait(done + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
+          // S_{j+2} overwrites P_{j+2-SBUF}, which that tile's P V reads
+          const int jo = jt + 2 - L::SBUF;
+          if (jo >= 0 && !(ok = wait(F_PVDONE1 + (jo & 1), (jo >> 1) & 1))) break;
           if (!(ok = wait(F_KFULL + (jt & 1), ((jt + 2) >> 1) & 1))) break;
           tc_fence_after();
           issue_s(jt + 2);
@@ -358,9 +346,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (p.causal && p.q_off + qrow - kb + 1 < lim) lim = p.q_off + qrow - kb + 1;
       }
       const bool masked = __any_sync(0xffffffffu, lim < 64);
-      if (!(ok = wait_w(F_SFULL + jt % 3, (jt / 3) & 1))) break;
+      if (!(ok = wait_w(F_SFULL + jt % L::SBUF, (jt / L::SBUF) & 1))) break;
       tc_fence_after();
-      const uint32_t sbuf = lane_base + L::T_S + (jt % 3) * 128;
+      const uint32_t sbuf = lane_base + L::T_S + (jt % L::SBUF) * 128;
       uint32_t sr[64];
       tmem_ld32(sbuf + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(sr));
       tmem_ld32(sbuf + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
@@ -374,16 +362,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int u = 0; u < 64; ++u) mx = fmaxf(mx, __uint_as_float(sr[u]));
       }
-      if constexpr (L::SPLIT) {
-        mx *= p.scale_log2;  // this group's own running maximum
-      } else {
-        // row maximum over both halves of the row
-        float* xmj = xm + (jt & 1) * 256;
-        xmj[g * 128 + t] = mx;
-        mbar_arrive(&bars[F_XCHG]);
-        if (!(ok = wait_w(F_XCHG, jt & 1))) break;
-        mx = fmaxf(mx, xmj[(g ^ 1) * 128 + t]) * p.scale_log2;
-      }
+      mx *= p.scale_log2;  // the tile's maximum over this half-row, log2 units
       float alpha = 1.f;
       const bool raise = mx > m + kRescaleMargin;
       if (raise) {
@@ -391,16 +370,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = mx;
       }
       if (__any_sync(0xffffffffu, raise && jt > 0)) {
-        // O (this group's O_g, or its channels of the shared O) holds
-        // sum_{j' < j} P_j' V_j' with the old m: scale it by alpha once the
-        // last of those products has landed.
-        const int done = (L::SPLIT && g == 1) ? F_PVDONE1 : F_PVDONE;
+        // O_g holds this group's sum_{j' < j} P_j' V_j' with the old m: scale
+        // it by alpha once the last of those products has landed.
+        const int done = g == 1 ? F_PVDONE1 : F_PVDONE;
         if (!(ok = wait_w(done + ((jt - 1) & 1), ((jt - 1) >> 1) & 1))) break;
         tc_fence_after();
-        constexpr int OCH = L::SPLIT ? D : L::HALF_D;
-        const uint32_t o_cols = L::T_O + g * (L::SPLIT ? D : L::HALF_D);
+        const uint32_t o_cols = L::T_O + g * D;
 #pragma unroll 1
-        for (int c = 0; c < OCH; c += 16) {
+        for (int c = 0; c < D; c += 16) {
           uint32_t ov[16];
           tmem_ld16(lane_base + o_cols + c, ov);
           tmem_ld_wait(ov);
@@ -443,38 +420,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_st16(sbuf + fp_col(64 * g) + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[L::SPLIT ? F_PFULL + 2 * g + (jt & 1) : F_PFULL]);
+      mbar_arrive(&bars[F_PFULL + 2 * g + (jt & 1)]);
     }
     // Epilogue: the last P V has landed; combine the two halves' sums. A
     // query tile that meets no key tile has O = 0 and LSE = -inf (the log of
     // an empty sum).
     const int n_kv = jt;
-    if (ok && n_kv > 0)
-      ok = wait_w((L::SPLIT ? F_PVDONE1 : F_PVDONE) + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
-    // split accumulators: this group's weight a_own and the other's a_oth
+    if (ok && n_kv > 0) ok = wait_w(F_PVDONE1 + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    // weights of this group's O_g (a_own) and of the other's (a_oth)
     float a_own = 1.f, a_oth = 0.f;
     if (ok && n_kv > 0) {
-      if constexpr (L::SPLIT) {
-        // the first use of the exchange buffer and its barrier
-        xm[g * 128 + t] = m;
-        xm[256 + g * 128 + t] = z;
-        mbar_arrive(&bars[F_XCHG]);
-        ok = wait_w(F_XCHG, 0);
-        if (ok) {
-          const float m2 = xm[(g ^ 1) * 128 + t], z2 = xm[256 + (g ^ 1) * 128 + t];
-          const float mm = fmaxf(m, m2);
-          // a group none of whose keys the row sees has m = -inf, z = 0
-          a_own = m == -INFINITY ? 0.f : ex2_approx(m - mm);
-          a_oth = m2 == -INFINITY ? 0.f : ex2_approx(m2 - mm);
-          z = z * a_own + z2 * a_oth;
-          m = mm;
-        }
-      } else {
-        float* xmz = xm + (n_kv & 1) * 256;
-        xmz[g * 128 + t] = z;
-        mbar_arrive(&bars[F_XCHG]);
-        ok = wait_w(F_XCHG, n_kv & 1);
-        if (ok) z += xmz[(g ^ 1) * 128 + t];
+      xm[g * 128 + t] = m;
+      xm[256 + g * 128 + t] = z;
+      mbar_arrive(&bars[F_XCHG]);
+      ok = wait_w(F_XCHG, 0);
+      if (ok) {
+        const float m2 = xm[(g ^ 1) * 128 + t], z2 = xm[256 + (g ^ 1) * 128 + t];
+        const float mm = fmaxf(m, m2);
+        // a group none of whose keys the row sees has m = -inf, z = 0
+        a_own = m == -INFINITY ? 0.f : ex2_approx(m - mm);
+        a_oth = m2 == -INFINITY ? 0.f : ex2_approx(m2 - mm);
+        z = z * a_own + z2 * a_oth;
+        m = mm;
       }
     }
     if (!ok) {
@@ -488,7 +455,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < L::HALF_D; c += 16) {
         uint32_t ov[16];
-        if (n_kv > 0 && L::SPLIT) {
+        if (n_kv > 0) {
           // channels [g*d/2 + c, +16) of a_0 O_0 + a_1 O_1
           uint32_t o0[16], o1[16];
           tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, o0);
@@ -498,9 +465,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u)
             ov[u] = __float_as_uint(__uint_as_float(o0[u]) * a0 + __uint_as_float(o1[u]) * a1);
-        } else if (n_kv > 0) {
-          tmem_ld16(lane_base + L::T_O + g * L::HALF_D + c, ov);
-          tmem_ld_wait(ov);
         } else {
 #pragma unroll
           for (int u = 0; u < 16; ++u) ov[u] = 0u;
