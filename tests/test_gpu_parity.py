@@ -154,6 +154,34 @@ def test_running_max_raised_every_key_tile(csa, d):
     assert np.abs(as_f64(gr["LSE"].cpu()) - ref["LSE"]).max() <= 1e-3 * max(1.0, np.abs(ref["LSE"]).max())
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("upper", [True, False])
+def test_forward_key_halves_far_apart(csa, d, upper):
+    # Inside every key tile the keys of one half (upper: local index >= 64)
+    # score about 20 log2 units above the other half for every query. The
+    # forward keeps a running maximum, sum and accumulator per half of each
+    # tile's keys and combines them once with weights 2^(m_g - M); here one
+    # half's weight is ~2^-20, and on the diagonal tile rows below 64 see
+    # only the lower half of that tile but both halves of the earlier ones.
+    B, H, N = 1, 2, 4 * 128 + 45
+    g = torch.Generator("cpu").manual_seed(93 + d + int(upper))
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g) for _ in range(4))
+    u = torch.randn(d, generator=g)
+    u = u / u.norm()
+    scale = d ** -0.5
+    c = 20.0 / (scale * 2.0 * np.log2(np.e))  # q.k gains 2c: 20 log2 units
+    half = (torch.arange(N) % 128) >= 64
+    lift = half if upper else ~half
+    q = q + 2.0 * u
+    k = k + (c * lift.float())[:, None] * u
+    q, k, v, do = (t.to(torch.bfloat16) for t in (q, k, v, do))
+    gr = run_gpu(csa, q, k, v, do, True, scale)
+    ref_o, ref_lse = oracle.forward(as_f64(q), as_f64(k), as_f64(v), scale, True)
+    e = rel(as_f64(gr["O"].cpu()), ref_o, None)
+    assert e <= TOL["bf16"], e
+    assert np.abs(as_f64(gr["LSE"].cpu()) - ref_lse).max() <= 1e-3 * max(1.0, np.abs(ref_lse).max())
+
+
 def run_masked(csa, q, k, v, do, bm, scale):
     dev = torch.device("cuda")
     qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
