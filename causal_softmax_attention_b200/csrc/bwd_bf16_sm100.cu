@@ -478,7 +478,13 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
                  (it > 0 || kk > 0));
         mma_commit(&bars[B_DVDONE]);
       };
-      // dK_j += dS^T Q_i, dS^T read from region B
+      // dK_j += dS^T Q_i, dS^T read from region B. dK(it) is the last reader
+      // of Q_i / dO_i's stage: S^T(it) and dP^T(it) completed before their
+      // results could be consumed, dV(it) was issued before it by the same
+      // thread (or, at d = 128, by the same second issuer), and the
+      // element-wise warps' LSE / D reads ended before dS^T(it) was signalled;
+      // dQ(it) reads only dS and the resident K. So the stage is released
+      // here, an MMA chain earlier than after dQ(it).
       auto issue_dk = [&](int it) {
         const uint64_t dQ = desc_mn0<D>(stage_q(it));
 #pragma unroll
@@ -486,16 +492,16 @@ __global__ void __launch_bounds__(Roles<D>::THREADS, 1)
           mma_ts(tmem + L::T_DK, tmem + L::T_DP + p_col<QC>(16 * kk), dQ + mnoff<D>(kk), ID_KV,
                  (it > 0 || kk > 0));
         mma_commit(&bars[B_DKDONE]);
+        mma_commit(&bars[B_QEMPTY + it % L::STAGES]);
       };
       // dQ_i = dS K_j (dS from shared memory) -> region B (d = 128) or the
-      // tile's S buffer (d <= 64); Q_i / dO_i's stage is free afterwards
+      // tile's S buffer (d <= 64)
       auto issue_dq = [&](int it) {
         const uint32_t dst = L::DQ_OVER_DP ? L::T_DP : sbuf(it);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(tmem + dst, dDS + kk * 128, dKmn + mnoff<D>(kk), ID_Q, kk > 0);
         mma_commit(&bars[B_DQFULL + (it & 1)]);
-        mma_commit(&bars[B_QEMPTY + it % L::STAGES]);
       };
       const bool scores = L::PIPE_S || warp == R::MMA_WARP;  // S and dP
       const bool grads = L::PIPE_S || warp == R::MMA2_WARP;  // dV, dK, dQ
