@@ -670,6 +670,8 @@ def run_rect(csa, q, k, v, do, off, causal, scale):
     ("f32", 333, 100, 0, True, 64),
     ("f32", 90, 200, 17, False, 7),
     ("f32", 70, 300, 101, True, 128),
+    ("bf16", 300, 40, 0, False, 64),       # 40 keys: the forward's second softmax group sees none
+    ("bf16", 100, 40, 20, True, 128),      # ... and, causal, rows before key 40 see fewer
 ])
 def test_rectangular_against_the_oracle(csa, dtype, nq, nk, off, causal, d):
     from seeded_inputs import draw_rect
