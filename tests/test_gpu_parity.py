@@ -214,7 +214,7 @@ def compare_masked(csa, B, H, N, d, bm, seed):
     return g, ref
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 128])
 def test_block_sparse_parity(csa, d):
     # kinds 0 / 1 / 2 anywhere, an empty query tile (O = 0, LSE = -inf), a
     # key tile no query meets (dK = dV = 0), kind 2 off the diagonal
@@ -333,6 +333,7 @@ def run_strided(csa, q, k, v, do, causal, scale, layout):
 
 @pytest.mark.parametrize("dtype,d,layout", [("bf16", 64, "bnhd"), ("bf16", 128, "bnhd"),
                                             ("bf16", 64, "packed"), ("bf16", 32, "packed"),
+                                            ("bf16", 128, "packed"),
                                             ("f32", 48, "bnhd"), ("f32", 7, "packed")])
 def test_strided_layouts_match_the_contiguous_path(csa, dtype, d, layout):
     # the same kernels on the same values: O, LSE, dK, dV bit-identical to the
